@@ -1,0 +1,210 @@
+"""CPU oracle for the MoE dispatch / combine path.
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  The library under
+``combine_permute_b200`` never does, and this package imports nothing from
+it.  Everything here is a plain restatement of what the pages say each
+step computes:
+
+* ``prepare``: sglang PR #19058, "Changes", item 1 (prepare_moe_input:
+  tokens per expert, prefix-sum expert offsets, optional FP8 block-scale
+  offsets, input / output permutations).
+* ``dispatch``: same page, item 2 (shuffle_rows, a dtype-agnostic row
+  gather).
+* ``dispatch_fp8``: the FP8 block-scale MoE path of TensorRT-LLM PR #9592
+  (run_moe_fp8_block_scales), with 1x128 blocks and scale = amax / 448.
+* ``combine``: sglang PR #19058, item 3 (apply_shuffle_mul_sum: gather,
+  scale by the router weight, reduce with fp32 accumulation).
+
+The arithmetic lives in ``moe_oracle.c`` (built with gcc, ``-O2
+-ffp-contract=off``, single-threaded).  ``brute_prepare`` is a second,
+pure-Python statement of the metadata step for tiny inputs, built on a
+stable ``sorted`` instead of the per-expert scan.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from .build import build_oracle, oracle_lib_path
+
+__all__ = [
+    "F32", "F16", "BF16", "lib", "prepare", "dispatch", "dispatch_fp8",
+    "combine", "brute_prepare", "f32_to_bf16", "f32_to_f16", "f16_to_f32",
+    "bf16_to_f32", "f32_to_e4m3", "e4m3_to_f32",
+]
+
+F32, F16, BF16 = 0, 1, 2
+_DT = {"fp32": F32, "fp16": F16, "bf16": BF16}
+
+_lib = None
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_vp = ctypes.c_void_p
+
+
+def lib():
+    """The oracle shared library (built on first use if it is missing)."""
+    global _lib
+    if _lib is None:
+        path = oracle_lib_path()
+        if not os.path.exists(path):
+            build_oracle()
+        L = ctypes.CDLL(path)
+        L.oracle_prepare.restype = ctypes.c_int64
+        L.oracle_prepare.argtypes = [_vp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_int32, _vp, _vp, _vp, _vp, _vp]
+        L.oracle_dispatch.restype = None
+        L.oracle_dispatch.argtypes = [_vp, ctypes.c_int64, ctypes.c_int32, _vp, ctypes.c_int64, _vp]
+        L.oracle_dispatch_fp8.restype = None
+        L.oracle_dispatch_fp8.argtypes = [_vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                          ctypes.c_int32, _vp, _vp, _vp, _vp, ctypes.c_int64,
+                                          _vp, _vp]
+        L.oracle_combine.restype = None
+        L.oracle_combine.argtypes = [_vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                     ctypes.c_int32, _vp, _vp, _vp, ctypes.c_int]
+        for name in ["oracle_f32_to_e4m3_n", "oracle_f32_to_bf16_n", "oracle_f32_to_f16_n",
+                     "oracle_f16_to_f32_n", "oracle_bf16_to_f32_n", "oracle_e4m3_to_f32_n"]:
+            fn = getattr(L, name)
+            fn.restype = None
+            fn.argtypes = [_vp, ctypes.c_int64, _vp]
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def prepare(ids: np.ndarray, E: int, block_align: int = 1):
+    """Routing metadata of ids [T,k] int32.
+
+    Returns a dict with counts [E], offsets [E+1], bso [E+1] (block-scale
+    offsets with alignment ``block_align``), input_perm [T*k],
+    output_perm [T*k] (all int32) and n_invalid (ids outside [0, E)).
+    """
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, k = ids.shape
+    S = T * k
+    counts = np.zeros(E, np.int32)
+    offsets = np.zeros(E + 1, np.int32)
+    bso = np.zeros(E + 1, np.int32)
+    inp = np.zeros(S, np.int32)
+    outp = np.zeros(S, np.int32)
+    n_bad = lib().oracle_prepare(_ptr(ids), T, k, E, block_align, _ptr(counts), _ptr(offsets),
+                                 _ptr(bso), _ptr(inp), _ptr(outp))
+    return dict(counts=counts, offsets=offsets, bso=bso, input_perm=inp, output_perm=outp,
+                n_invalid=int(n_bad))
+
+
+def dispatch(x: np.ndarray, k: int, input_perm: np.ndarray, out: np.ndarray | None = None):
+    """Same-dtype dispatch: out[p] = x[input_perm[p] // k] (rows with -1 untouched)."""
+    x = np.ascontiguousarray(x)
+    input_perm = np.ascontiguousarray(input_perm, dtype=np.int32)
+    S = input_perm.shape[0]
+    if out is None:
+        out = np.zeros((S,) + x.shape[1:], dtype=x.dtype)
+    row_bytes = x.dtype.itemsize * int(np.prod(x.shape[1:]))
+    lib().oracle_dispatch(_ptr(x), row_bytes, k, _ptr(input_perm), S, _ptr(out))
+    return out
+
+
+def dispatch_fp8(x_bits: np.ndarray, x_dtype: str, ids: np.ndarray, meta: dict,
+                 q: np.ndarray | None = None, scales: np.ndarray | None = None):
+    """FP8 E4M3 1x128 block-scale dispatch.
+
+    ``x_bits`` is [T,H] uint16 holding bf16 or fp16 bit patterns.  Returns
+    (q [S,H] uint8, scales [bso[E], H/128] fp32).  Arrays passed in are
+    written in place, so untouched rows keep their previous contents.
+    """
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, H = x_bits.shape
+    k = ids.shape[1]
+    S = T * k
+    nb = H // 128
+    if q is None:
+        q = np.zeros((S, H), np.uint8)
+    if scales is None:
+        scales = np.zeros((int(meta["bso"][-1]), nb), np.float32)
+    lib().oracle_dispatch_fp8(_ptr(x_bits), _DT[x_dtype], T, H, k, _ptr(ids),
+                              _ptr(meta["input_perm"]), _ptr(meta["offsets"]), _ptr(meta["bso"]),
+                              S, _ptr(q), _ptr(scales))
+    return q, scales
+
+
+def combine(y_bits: np.ndarray, y_dtype: str, output_perm: np.ndarray, w: np.ndarray,
+            out_dtype: str):
+    """out[t] = round(sum_j w[t,j] * y[output_perm[t*k+j]]) in fp32, j ascending.
+
+    ``y_bits`` holds the raw storage ([S,H] uint16 for bf16/fp16, float32
+    for fp32).  Returns raw storage of the output dtype.
+    """
+    y_bits = np.ascontiguousarray(y_bits)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    output_perm = np.ascontiguousarray(output_perm, dtype=np.int32)
+    T, k = w.shape
+    H = y_bits.shape[1]
+    out = np.zeros((T, H), np.float32 if out_dtype == "fp32" else np.uint16)
+    lib().oracle_combine(_ptr(y_bits), _DT[y_dtype], T, H, k, _ptr(output_perm), _ptr(w),
+                         _ptr(out), _DT[out_dtype])
+    return out
+
+
+def brute_prepare(ids, E: int, block_align: int = 1):
+    """Pure-Python metadata for tiny inputs (a second statement of prepare).
+
+    The dispatched order is ``sorted`` over (expert, token, slot) tuples of
+    the valid slots, which is the stable order by expert id.
+    """
+    ids = [[int(v) for v in row] for row in ids]
+    T = len(ids)
+    k = len(ids[0]) if T else 0
+    keyed = sorted((e, t, j) for t in range(T) for j, e in enumerate(ids[t]) if 0 <= e < E)
+    input_perm = [t * k + j for (_, t, j) in keyed] + [-1] * (T * k - len(keyed))
+    output_perm = [-1] * (T * k)
+    for p, (_, t, j) in enumerate(keyed):
+        output_perm[t * k + j] = p
+    counts = [sum(1 for (e, _, _) in keyed if e == x) for x in range(E)]
+    offsets = [0]
+    for c in counts:
+        offsets.append(offsets[-1] + c)
+    bso = [0]
+    for c in counts:
+        bso.append(bso[-1] + -(-c // block_align) * block_align)
+    return dict(counts=counts, offsets=offsets, bso=bso, input_perm=input_perm,
+                output_perm=output_perm, n_invalid=T * k - len(keyed))
+
+
+def _conv(name, arr, in_dtype, out_dtype):
+    a = np.ascontiguousarray(np.asarray(arr, dtype=in_dtype).ravel())
+    out = np.empty(a.shape, dtype=out_dtype)
+    getattr(lib(), name)(_ptr(a), a.size, _ptr(out))
+    return out
+
+
+def f32_to_bf16(a):
+    return _conv("oracle_f32_to_bf16_n", a, np.float32, np.uint16)
+
+
+def f32_to_f16(a):
+    return _conv("oracle_f32_to_f16_n", a, np.float32, np.uint16)
+
+
+def f32_to_e4m3(a):
+    return _conv("oracle_f32_to_e4m3_n", a, np.float32, np.uint8)
+
+
+def bf16_to_f32(a):
+    return _conv("oracle_bf16_to_f32_n", a, np.uint16, np.float32)
+
+
+def f16_to_f32(a):
+    return _conv("oracle_f16_to_f32_n", a, np.uint16, np.float32)
+
+
+def e4m3_to_f32(a):
+    return _conv("oracle_e4m3_to_f32_n", a, np.uint8, np.float32)

@@ -1,0 +1,381 @@
+/*
+ * CPU oracle for the MoE dispatch / combine path.
+ *
+ * TEST INFRASTRUCTURE.  This file is the plain, slow, obviously correct
+ * definition that the CUDA library is checked against.  Only the tests, the
+ * smoke check and the benchmark's CPU-baseline leg load it; the library's
+ * product path never does.  It shares no code, header or table with the
+ * CUDA sources.
+ *
+ * Sources (the pages' statement of what each step computes):
+ *   - sglang PR #19058 "[jit_kernel] Add prepare_moe_input JIT kernels",
+ *     section "Changes", item 1 prepare_moe_input:
+ *       compute_problem_sizes_kernel  -> tokens per expert   (oracle_prepare)
+ *       compute_expert_offsets_kernel -> prefix sum           (oracle_prepare)
+ *       compute_expert_blockscale_offsets_kernel (optional)   (oracle_prepare)
+ *       compute_arg_sorts_kernel -> input/output permutation  (oracle_prepare)
+ *     item 2 shuffle_rows: dtype-agnostic row gather        (oracle_dispatch)
+ *     item 3 apply_shuffle_mul_sum: gather + scale + reduce with FP32
+ *       accumulation over fp16 / bf16 / fp32                (oracle_combine)
+ *   - TensorRT-LLM PR #9592 "Enable CuteDSL MoE with Large EP" (Walkthrough
+ *     and review comments): "expanded idx" = t*k + j and "permuted idx" =
+ *     dispatched row, int32 index tensors, and the FP8 block-scale MoE path
+ *     (run_moe_fp8_block_scales), which oracle_dispatch_fp8 instantiates
+ *     with 1x128 blocks and scale = amax / 448.
+ *
+ * Readings where the pages are silent (each one is listed in the design
+ * notes):
+ *   - input_permutation[p] is the flat slot (expanded) index i = t*k + j of
+ *     the p-th dispatched row; output_permutation is its inverse.
+ *   - Within an expert the order is ascending slot index i, i.e. ascending
+ *     token then ascending slot (a stable sort by expert id).
+ *   - expert_offsets has E+1 entries, the last one the number of valid
+ *     slots.
+ *   - Block-scale offsets round each expert's row count up to a multiple of
+ *     A (A = 1 gives the expert offsets).
+ *   - Ids outside [0, E) are excluded from every output: they are not
+ *     counted, their output_permutation entry is -1, the trailing
+ *     input_permutation entries (p >= offsets[E]) are -1, dispatch leaves
+ *     those rows untouched and combine skips those slots.
+ *   - FP8: per dispatched row and per 128-column block, amax = max |x|,
+ *     s = amax / 448 (fp32, round to nearest), q = e4m3(x / s) with x / s an
+ *     fp32 division, round to nearest even, saturating to +-448; a block
+ *     with amax = 0 gets s = 0 and all-zero bytes.  The scale of dispatched
+ *     row p of expert e goes to row bso[e] + (p - offsets[e]).
+ *   - Combine: acc = 0; for j = 0..k-1: acc = acc + w[t,j] * y[row_j, h],
+ *     each product and each sum rounded separately to fp32 (this file must
+ *     be compiled with -ffp-contract=off), then acc rounded to the output
+ *     dtype (round to nearest even; fp32 output is acc itself).
+ */
+
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+enum { ORACLE_F32 = 0, ORACLE_F16 = 1, ORACLE_BF16 = 2 };
+
+/* ------------------------------------------------------------------ */
+/* Scalar formats, written from their bit-level definitions.           */
+/* ------------------------------------------------------------------ */
+
+/* bfloat16 is the upper half of an IEEE binary32. */
+float oracle_bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* IEEE binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+float oracle_f16_to_f32(uint16_t h)
+{
+    int sign = h >> 15;
+    int expo = (h >> 10) & 0x1f;
+    int frac = h & 0x3ff;
+    double v;
+    if (expo == 0)
+        v = ldexp((double)frac, -24);                 /* subnormal: frac * 2^-24 */
+    else if (expo == 31)
+        v = frac ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + frac), expo - 25);  /* (1 + frac/1024) * 2^(expo-15) */
+    return (float)(sign ? -v : v);
+}
+
+/* Round a non-negative double holding an exact value to the nearest
+ * integer, ties to even. */
+static double round_half_even(double q)
+{
+    double fl = floor(q);
+    double diff = q - fl;
+    if (diff > 0.5 || (diff == 0.5 && fmod(fl, 2.0) != 0.0))
+        fl += 1.0;
+    return fl;
+}
+
+/* binary32 -> bfloat16, round to nearest even on the 16 dropped bits. */
+uint16_t oracle_f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7fffffffu) > 0x7f800000u)          /* NaN stays NaN (quiet) */
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t upper = u >> 16;
+    uint32_t lower = u & 0xffffu;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))
+        upper += 1u;                               /* a carry may reach inf: correct */
+    return (uint16_t)upper;
+}
+
+/* binary32 -> binary16, round to nearest even, overflow to infinity. */
+uint16_t oracle_f32_to_f16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+    if ((u & 0x7fffffffu) > 0x7f800000u)
+        return (uint16_t)(sign | 0x7e00u);
+    double a = fabs((double)f);                    /* exact */
+    if (a >= 65520.0)                              /* halfway above 65504 and beyond */
+        return (uint16_t)(sign | 0x7c00u);
+    if (a < ldexp(1.0, -14)) {                     /* subnormal range: step 2^-24 */
+        double q = round_half_even(a / ldexp(1.0, -24));
+        return (uint16_t)(sign | (uint16_t)q);     /* q = 1024 encodes 2^-14 */
+    }
+    int ex;
+    frexp(a, &ex);                                 /* a in [2^(ex-1), 2^ex) */
+    int e = ex - 1;
+    double q = round_half_even(a / ldexp(1.0, e - 10)); /* in [1024, 2048] */
+    return (uint16_t)(sign | (uint16_t)((e + 15) * 1024 + (int)q - 1024));
+}
+
+/*
+ * binary32 -> OCP FP8 E4M3 (the "FN" variant: no infinities, 0x7f / 0xff
+ * are NaN, largest finite 448 = 0x7e).  1 sign bit, 4 exponent bits
+ * (bias 7), 3 fraction bits; subnormals are frac * 2^-9.  Round to nearest
+ * even; finite magnitudes that round above 448 (and infinities) saturate to
+ * 448; NaN maps to NaN.
+ */
+uint8_t oracle_f32_to_e4m3(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    uint8_t sign = (uint8_t)((u >> 24) & 0x80u);
+    if ((u & 0x7fffffffu) > 0x7f800000u)
+        return (uint8_t)(sign | 0x7fu);
+    double a = fabs((double)f);
+    if (a >= 448.0)
+        return (uint8_t)(sign | 0x7eu);
+    if (a < ldexp(1.0, -6)) {                      /* subnormal range: step 2^-9 */
+        double q = round_half_even(a / ldexp(1.0, -9));
+        return (uint8_t)(sign | (uint8_t)q);       /* q = 8 encodes 2^-6 */
+    }
+    int ex;
+    frexp(a, &ex);
+    int e = ex - 1;                                /* a in [2^e, 2^(e+1)), e in [-6, 8] */
+    double q = round_half_even(a / ldexp(1.0, e - 3)); /* in [8, 16] */
+    int code = (e + 7) * 8 + (int)q - 8;
+    if (code > 0x7e)
+        code = 0x7e;
+    return (uint8_t)(sign | (uint8_t)code);
+}
+
+float oracle_e4m3_to_f32(uint8_t b)
+{
+    int sign = b >> 7;
+    int expo = (b >> 3) & 0xf;
+    int frac = b & 7;
+    double v;
+    if (expo == 0xf && frac == 7)
+        v = NAN;
+    else if (expo == 0)
+        v = ldexp((double)frac, -9);
+    else
+        v = ldexp((double)(8 + frac), expo - 10);  /* (1 + frac/8) * 2^(expo-7) */
+    return (float)(sign ? -v : v);
+}
+
+static float load_as_f32(const void *base, int dtype, int64_t idx)
+{
+    if (dtype == ORACLE_F32)
+        return ((const float *)base)[idx];
+    if (dtype == ORACLE_F16)
+        return oracle_f16_to_f32(((const uint16_t *)base)[idx]);
+    return oracle_bf16_to_f32(((const uint16_t *)base)[idx]);
+}
+
+static void store_from_f32(void *base, int dtype, int64_t idx, float v)
+{
+    if (dtype == ORACLE_F32)
+        ((float *)base)[idx] = v;
+    else if (dtype == ORACLE_F16)
+        ((uint16_t *)base)[idx] = oracle_f32_to_f16(v);
+    else
+        ((uint16_t *)base)[idx] = oracle_f32_to_bf16(v);
+}
+
+/* ------------------------------------------------------------------ */
+/* Step A: routing metadata (prepare_moe_input).                       */
+/* ------------------------------------------------------------------ */
+
+/*
+ * ids [T*k] (row-major [T,k]) -> counts [E], offsets [E+1],
+ * bso [E+1] (may be NULL), input_perm [T*k], output_perm [T*k].
+ * Returns the number of slots whose id lies outside [0, E).
+ *
+ * The permutation is built by scanning the slots once per expert, in
+ * ascending expert order and ascending slot order: the p-th slot found is
+ * dispatched row p.  This is O(E * T * k) on purpose: it is the stable
+ * order written out, with nothing shared with a counting sort.
+ */
+int64_t oracle_prepare(const int32_t *ids, int64_t T, int32_t k, int32_t E, int32_t A,
+                       int32_t *counts, int32_t *offsets, int32_t *bso,
+                       int32_t *input_perm, int32_t *output_perm)
+{
+    int64_t S = T * (int64_t)k;
+    for (int64_t i = 0; i < S; ++i) {
+        output_perm[i] = -1;
+        input_perm[i] = -1;
+    }
+    int64_t p = 0;
+    for (int32_t e = 0; e < E; ++e) {
+        int32_t c = 0;
+        for (int64_t i = 0; i < S; ++i) {
+            if (ids[i] == e) {
+                input_perm[p] = (int32_t)i;
+                output_perm[i] = (int32_t)p;
+                ++p;
+                ++c;
+            }
+        }
+        counts[e] = c;
+    }
+    offsets[0] = 0;
+    for (int32_t e = 0; e < E; ++e)
+        offsets[e + 1] = offsets[e] + counts[e];
+    if (bso) {
+        bso[0] = 0;
+        for (int32_t e = 0; e < E; ++e) {
+            int32_t padded = (counts[e] + A - 1) / A * A;
+            bso[e + 1] = bso[e] + padded;
+        }
+    }
+    return S - p;
+}
+
+/* ------------------------------------------------------------------ */
+/* Step B1: dispatch, same dtype (shuffle_rows).                       */
+/* ------------------------------------------------------------------ */
+
+/* out[p, :] = x[input_perm[p] / k, :] for every p with input_perm[p] >= 0. */
+void oracle_dispatch(const void *x, int64_t row_bytes, int32_t k,
+                     const int32_t *input_perm, int64_t S, void *out)
+{
+    const unsigned char *src = (const unsigned char *)x;
+    unsigned char *dst = (unsigned char *)out;
+    for (int64_t p = 0; p < S; ++p) {
+        int32_t i = input_perm[p];
+        if (i < 0)
+            continue;
+        int64_t t = i / k;
+        memcpy(dst + p * row_bytes, src + t * row_bytes, (size_t)row_bytes);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Step B2: dispatch with FP8 E4M3 1x128 block-scale quantisation.     */
+/* ------------------------------------------------------------------ */
+
+/*
+ * x [T,H] bf16 or f16; for each dispatched row p (token t = input_perm[p]/k,
+ * expert e = ids[input_perm[p]]) and each 128-column block b:
+ *   amax = max |x[t, b*128 .. b*128+127]|
+ *   s    = amax / 448            (s = 0 and zero bytes when amax = 0)
+ *   q[p, c] = e4m3(x[t, c] / s)
+ *   scales[(bso[e] + p - offsets[e]) * (H/128) + b] = s
+ * Rows and scale rows that no valid slot maps to are left untouched.
+ */
+void oracle_dispatch_fp8(const uint16_t *x, int x_dtype, int64_t T, int64_t H, int32_t k,
+                         const int32_t *ids, const int32_t *input_perm,
+                         const int32_t *offsets, const int32_t *bso, int64_t S,
+                         uint8_t *q, float *scales)
+{
+    (void)T;
+    int64_t nb = H / 128;
+    for (int64_t p = 0; p < S; ++p) {
+        int32_t i = input_perm[p];
+        if (i < 0)
+            continue;
+        int64_t t = i / k;
+        int32_t e = ids[i];
+        int64_t srow = (int64_t)bso[e] + (p - offsets[e]);
+        for (int64_t b = 0; b < nb; ++b) {
+            float amax = 0.0f;
+            for (int64_t c = b * 128; c < b * 128 + 128; ++c) {
+                float a = fabsf(load_as_f32(x, x_dtype, t * H + c));
+                if (a > amax)
+                    amax = a;
+            }
+            float s = 0.0f;
+            if (amax == 0.0f) {
+                for (int64_t c = b * 128; c < b * 128 + 128; ++c)
+                    q[p * H + c] = 0;
+            } else {
+                s = amax / 448.0f;
+                for (int64_t c = b * 128; c < b * 128 + 128; ++c) {
+                    float v = load_as_f32(x, x_dtype, t * H + c) / s;
+                    q[p * H + c] = oracle_f32_to_e4m3(v);
+                }
+            }
+            scales[srow * nb + b] = s;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Step C1: combine (apply_shuffle_mul_sum).                           */
+/* ------------------------------------------------------------------ */
+
+/*
+ * out[t, h] = round_out( sum_{j=0..k-1} w[t,j] * y[output_perm[t*k+j], h] ),
+ * summed in fp32 in ascending j with every operation rounded separately;
+ * slots with output_perm = -1 contribute nothing.
+ */
+void oracle_combine(const void *y, int y_dtype, int64_t T, int64_t H, int32_t k,
+                    const int32_t *output_perm, const float *w, void *out, int out_dtype)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t h = 0; h < H; ++h) {
+            float acc = 0.0f;
+            for (int32_t j = 0; j < k; ++j) {
+                int32_t p = output_perm[t * k + j];
+                if (p < 0)
+                    continue;
+                float prod = w[t * k + j] * load_as_f32(y, y_dtype, (int64_t)p * H + h);
+                acc = acc + prod;
+            }
+            store_from_f32(out, out_dtype, t * H + h, acc);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Array forms of the scalar conversions (for exhaustive sweeps).      */
+/* ------------------------------------------------------------------ */
+
+void oracle_f32_to_e4m3_n(const float *in, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_f32_to_e4m3(in[i]);
+}
+
+void oracle_f32_to_bf16_n(const float *in, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_f32_to_bf16(in[i]);
+}
+
+void oracle_f32_to_f16_n(const float *in, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_f32_to_f16(in[i]);
+}
+
+void oracle_f16_to_f32_n(const uint16_t *in, int64_t n, float *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_f16_to_f32(in[i]);
+}
+
+void oracle_bf16_to_f32_n(const uint16_t *in, int64_t n, float *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_bf16_to_f32(in[i]);
+}
+
+void oracle_e4m3_to_f32_n(const uint8_t *in, int64_t n, float *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_e4m3_to_f32(in[i]);
+}

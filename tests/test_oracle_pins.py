@@ -1,0 +1,374 @@
+"""Pins for the CPU oracle: each check ties the oracle to something other
+than itself — a library routine, a brute force, a closed form, an invariant
+of the definition, or a hand-worked example — so that a dropped term, a
+wrong sign or index, or a transposed operand fails at least one of them.
+
+Sources of the definitions: sglang PR #19058 "[jit_kernel] Add
+prepare_moe_input JIT kernels", section "Changes" (prepare_moe_input,
+shuffle_rows, apply_shuffle_mul_sum); TensorRT-LLM PR #9592 (expanded /
+permuted index naming, FP8 block-scale path).  The e4m3 format facts (bias
+7, max 448, subnormal step 2^-9, no infinities) are those of the OCP FP8
+E4M3 format.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import CONFIGS, make_workload
+
+RNG = np.random.default_rng(12345)
+
+
+# ---------------------------------------------------------------------------
+# scalar formats
+# ---------------------------------------------------------------------------
+
+def test_bf16_decode_exhaustive_vs_torch():
+    bits = np.arange(1 << 16, dtype=np.uint16)
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    got = oracle.bf16_to_f32(bits)
+    np.testing.assert_array_equal(got.view(np.uint32)[~np.isnan(ref)], ref.view(np.uint32)[~np.isnan(ref)])
+    assert np.isnan(got[np.isnan(ref)]).all()
+
+
+def test_f16_decode_exhaustive_vs_numpy():
+    bits = np.arange(1 << 16, dtype=np.uint16)
+    ref = bits.view(np.float16).astype(np.float32)
+    got = oracle.f16_to_f32(bits)
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got.view(np.uint32)[ok], ref.view(np.uint32)[ok])
+    assert np.isnan(got[~ok]).all()
+
+
+def _f32_samples(n):
+    """Random fp32 bit patterns plus values sitting exactly on rounding ties."""
+    u = RNG.integers(0, 1 << 32, size=n, dtype=np.uint64).astype(np.uint32)
+    f = u.view(np.float32)
+    return f[np.isfinite(f)]
+
+
+def test_f32_to_bf16_vs_torch():
+    f = _f32_samples(2_000_000)
+    # ties: low 16 bits exactly 0x8000, both parities of the kept bit
+    tie = (RNG.integers(0, 1 << 16, size=100_000).astype(np.uint32) << 16) | 0x8000
+    f = np.concatenate([f, tie.view(np.float32)])
+    f = f[np.isfinite(f)]
+    ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(oracle.f32_to_bf16(f), ref)
+
+
+def test_f32_to_f16_vs_numpy():
+    f = _f32_samples(2_000_000)
+    # values around the fp16 range: subnormals, ties at 13 dropped bits,
+    # the overflow threshold 65520
+    g = (RNG.standard_normal(500_000) * np.exp2(RNG.integers(-26, 17, 500_000))).astype(np.float32)
+    ties = ((RNG.integers(0, 1 << 19, 100_000).astype(np.uint32) << 13) | 0x1000).view(np.float32)
+    edges = np.array([65504, 65519.996, 65520, 65536, 2**-24, 2**-25, 3 * 2**-26, 2**-14,
+                      2**-14 - 2**-25], np.float32)
+    f = np.concatenate([f, g, ties, edges, -edges])
+    f = f[np.isfinite(f)]
+    with np.errstate(over="ignore"):
+        ref = f.astype(np.float16).view(np.uint16)
+    np.testing.assert_array_equal(oracle.f32_to_f16(f), ref)
+
+
+def _e4m3_grid():
+    """All finite e4m3 magnitudes, decoded by torch (library routine)."""
+    codes = np.arange(0x7f, dtype=np.uint8)  # 0x00..0x7e
+    return torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+
+
+def test_e4m3_decode_all_codes_vs_torch():
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+    got = oracle.e4m3_to_f32(codes)
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok], ref[ok])
+    assert np.isnan(got[~ok]).all() and set(codes[~ok].tolist()) == {0x7f, 0xff}
+
+
+def test_e4m3_closed_forms():
+    # hand-derived from the format: bias 7, 3 fraction bits, max 448
+    cases = [  # (value, code); a list, since 0.0 and -0.0 are equal dict keys
+        (448.0, 0x7E), (1e9, 0x7E), (464.0, 0x7E), (np.inf, 0x7E),     # saturate
+        (-448.0, 0xFE), (-np.inf, 0xFE),
+        (1.0, 0x38), (1.125, 0x39), (1.0625, 0x38),                    # tie 1+1/16 -> even (1.0)
+        (1.1875, 0x3A),                                                # tie 1+3/16 -> even (1.25)
+        (2.0 ** -6, 0x08), (2.0 ** -9, 0x01), (2.0 ** -10, 0x00),      # min normal, min subnormal, tie to 0
+        (3 * 2.0 ** -10, 0x02),                                        # 1.5 steps -> 2 (even)
+        (3 * 2.0 ** -11, 0x01), (0.0, 0x00), (-0.0, 0x80),
+        (240.0, 0x77), (256.0, 0x78), (416.0, 0x7D), (432.0, 0x7E),    # 432 = tie 416|448 -> even 448
+        (-3.5, 0xC6),
+    ]
+    got = oracle.f32_to_e4m3(np.array([v for v, _ in cases], np.float32))
+    np.testing.assert_array_equal(got, np.array([c for _, c in cases], np.uint8))
+    assert oracle.f32_to_e4m3(np.array([np.nan], np.float32))[0] & 0x7F == 0x7F
+
+
+def test_e4m3_encode_vs_torch_ties_and_random():
+    grid = _e4m3_grid()
+    # midpoints between neighbouring e4m3 values and their fp32 neighbours
+    mids = ((grid[1:].astype(np.float64) + grid[:-1]) / 2).astype(np.float32)
+    near = np.concatenate([mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(1e9)),
+                           grid, np.nextafter(grid[1:], np.float32(0)), np.nextafter(grid, np.float32(1e9))])
+    rnd = (RNG.standard_normal(3_000_000) * np.exp2(RNG.integers(-14, 10, 3_000_000))).astype(np.float32)
+    f = np.concatenate([near, -near, rnd])
+    f = f[np.abs(f) <= 448]  # torch maps magnitudes above 464 to NaN: compare inside the range only
+    ref = torch.from_numpy(f).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(oracle.f32_to_e4m3(f), ref)
+
+
+def test_e4m3_roundtrip_every_code():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    np.testing.assert_array_equal(oracle.f32_to_e4m3(oracle.e4m3_to_f32(codes)), codes)
+
+
+# ---------------------------------------------------------------------------
+# prepare
+# ---------------------------------------------------------------------------
+
+def test_prepare_hand_worked_example():
+    # ids [[2,0],[1,2],[2,1]], E=3, k=2 -> slots i: e(0)=2 e(1)=0 e(2)=1 e(3)=2 e(4)=2 e(5)=1
+    # expert 0 holds slot 1; expert 1 slots 2,5; expert 2 slots 0,3,4 (ascending)
+    ids = np.array([[2, 0], [1, 2], [2, 1]], np.int32)
+    m = oracle.prepare(ids, E=3, block_align=4)
+    assert m["counts"].tolist() == [1, 2, 3]
+    assert m["offsets"].tolist() == [0, 1, 3, 6]
+    assert m["bso"].tolist() == [0, 4, 8, 12]
+    assert m["input_perm"].tolist() == [1, 2, 5, 0, 3, 4]
+    assert m["output_perm"].tolist() == [3, 0, 1, 4, 5, 2]
+    assert m["n_invalid"] == 0
+
+
+def test_prepare_hand_worked_invalid_and_duplicates():
+    # a token may name an expert twice; ids -1 and 3 (E=3) are invalid
+    ids = np.array([[1, 1], [-1, 0], [3, 1]], np.int32)
+    m = oracle.prepare(ids, E=3)
+    assert m["counts"].tolist() == [1, 3, 0]
+    assert m["offsets"].tolist() == [0, 1, 4, 4]
+    assert m["input_perm"].tolist() == [3, 0, 1, 5, -1, -1]
+    assert m["output_perm"].tolist() == [1, 2, -1, 0, -1, 3]
+    assert m["n_invalid"] == 2
+
+
+@pytest.mark.parametrize("trial", range(60))
+def test_prepare_vs_bruteforce_tiny(trial):
+    rng = np.random.default_rng(trial)
+    T = int(rng.integers(0, 9))
+    k = int(rng.integers(1, 5))
+    E = int(rng.integers(1, 7))
+    A = int(rng.integers(1, 5))
+    ids = rng.integers(-1, E + 1, size=(T, k)).astype(np.int32)  # duplicates and invalid ids included
+    m = oracle.prepare(ids, E, A)
+    b = oracle.brute_prepare(ids, E, A)
+    for key in ("counts", "offsets", "bso", "input_perm", "output_perm"):
+        assert np.asarray(m[key]).tolist() == list(b[key]), key
+    assert m["n_invalid"] == b["n_invalid"]
+
+
+def _check_prepare_invariants(ids, E, A, m):
+    flat = ids.ravel()
+    S = flat.size
+    # library special cases
+    np.testing.assert_array_equal(m["counts"], np.bincount(flat, minlength=E))
+    np.testing.assert_array_equal(m["offsets"][1:], np.cumsum(m["counts"]))
+    ref_perm = torch.argsort(torch.from_numpy(flat.astype(np.int64)), stable=True).numpy()
+    np.testing.assert_array_equal(m["input_perm"], ref_perm)
+    # invariants
+    assert m["offsets"][0] == 0 and m["offsets"][E] == S
+    inp, outp = m["input_perm"], m["output_perm"]
+    assert np.array_equal(np.sort(inp), np.arange(S))
+    np.testing.assert_array_equal(outp[inp], np.arange(S))
+    np.testing.assert_array_equal(inp[outp], np.arange(S))
+    assert (np.diff(flat[inp]) >= 0).all()
+    for e in range(E):
+        seg = inp[m["offsets"][e]:m["offsets"][e + 1]]
+        assert (np.diff(seg) > 0).all()
+        assert (flat[seg] == e).all()
+    pad = np.diff(m["bso"]) - m["counts"]
+    assert (np.diff(m["bso"]) % A == 0).all() and (pad >= 0).all() and (pad < A).all()
+
+
+@pytest.mark.parametrize("name", list(CONFIGS))
+def test_prepare_invariants_on_workloads(name):
+    w = CONFIGS[name]
+    if w.S > 200_000:
+        w = w.scaled(200_000 // w.k)
+    ids, _, _, _ = make_workload(w, with_x=False, with_y=False)
+    A = w.block_align if w.block_align > 1 else 128
+    m = oracle.prepare(ids, w.E, A)
+    _check_prepare_invariants(ids, w.E, A, m)
+    m1 = oracle.prepare(ids, w.E, 1)
+    np.testing.assert_array_equal(m1["bso"], m1["offsets"])
+
+
+# ---------------------------------------------------------------------------
+# dispatch
+# ---------------------------------------------------------------------------
+
+def test_dispatch_same_dtype_vs_index_select():
+    w = CONFIGS["uniform_t4096_h7168_e256_k8"].scaled(64)
+    ids, _, x, _ = make_workload(w, with_y=False)
+    m = oracle.prepare(ids, w.E)
+    xb = x.view(torch.int16).numpy()
+    got = oracle.dispatch(xb, w.k, m["input_perm"])
+    ref = torch.from_numpy(xb).index_select(0, torch.from_numpy(m["input_perm"] // w.k).long()).numpy()
+    np.testing.assert_array_equal(got, ref)
+    # every token row appears exactly k times
+    rows, mult = np.unique(got.view(np.dtype((np.void, got.shape[1] * 2))), return_counts=True)
+    assert (mult == w.k).all() and rows.size == w.T
+
+
+def test_dispatch_leaves_invalid_rows_untouched():
+    ids = np.array([[0, 5], [1, 0]], np.int32)  # id 5 invalid with E=2
+    m = oracle.prepare(ids, 2)
+    x = np.array([[1, 2], [3, 4]], np.float32)
+    out = np.full((4, 2), -7.0, np.float32)
+    oracle.dispatch(x, 2, m["input_perm"], out)
+    np.testing.assert_array_equal(out, [[1, 2], [3, 4], [3, 4], [-7, -7]])
+
+
+# ---------------------------------------------------------------------------
+# fp8 dispatch
+# ---------------------------------------------------------------------------
+
+def _fp8_case(T=48, H=512, E=16, k=4, dtype="bf16", seed=7):
+    rng = np.random.default_rng(seed)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(seed)).to(tdt)
+    x[3, 128:256] = 0           # an all-zero block
+    x[5, :128] *= 1e-3          # a block of tiny values
+    return ids, x
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_dispatch_fp8_vs_torch_witness(dtype):
+    T, H, E, k, A = 48, 512, 16, 4, 8
+    ids, x = _fp8_case(T, H, E, k, dtype)
+    m = oracle.prepare(ids, E, A)
+    q, scales = oracle.dispatch_fp8(x.view(torch.int16).numpy().view(np.uint16), dtype, ids, m)
+    xf = x.float().view(T, H // 128, 128)
+    amax = xf.abs().amax(dim=2)                       # torch reduction
+    s_ref = amax / 448.0                              # torch fp32 division
+    safe = torch.where(s_ref == 0, torch.ones_like(s_ref), s_ref)
+    q_tok = (xf / safe[..., None]).to(torch.float8_e4m3fn).view(torch.uint8).view(T, H)
+    q_tok[(s_ref == 0).repeat_interleave(128, dim=1)] = 0
+    inp = m["input_perm"]
+    np.testing.assert_array_equal(q, q_tok.numpy()[inp // k])
+    e_of_p = ids.ravel()[inp]
+    srow = m["bso"][e_of_p] + np.arange(T * k) - m["offsets"][e_of_p]
+    np.testing.assert_array_equal(scales[srow], s_ref.numpy()[inp // k])
+    # padding rows of the scale tensor were never written
+    written = np.zeros(scales.shape[0], bool)
+    written[srow] = True
+    assert (scales[~written] == 0).all()
+
+
+def test_dispatch_fp8_decode_error_bound_and_amax_code():
+    T, H, E, k = 32, 1024, 8, 2
+    ids, x = _fp8_case(T, H, E, k, "bf16", seed=11)
+    m = oracle.prepare(ids, E, 1)
+    q, scales = oracle.dispatch_fp8(x.view(torch.int16).numpy().view(np.uint16), "bf16", ids, m)
+    xr = x.double().numpy()[m["input_perm"] // k]
+    s = np.repeat(scales, 128, axis=1).astype(np.float64)
+    dec = oracle.e4m3_to_f32(q).reshape(q.shape).astype(np.float64) * s
+    # |x - decode(q) * s| <= half an e4m3 step of v = x / s (step 2^(e-3) for
+    # v in [2^e, 2^(e+1)), 2^-9 below 2^-6), plus the fp32 rounding of x / s
+    v = np.abs(xr / np.where(s == 0, 1, s))
+    half_step = np.where(v >= 2.0 ** -6, np.exp2(np.floor(np.log2(np.maximum(v, 2.0 ** -6))) - 4), 2.0 ** -10)
+    assert (np.abs(dec - xr) <= half_step * s + np.abs(xr) * 2.0 ** -23).all()
+    # the element that attains amax encodes to +-448 exactly
+    blocks = np.abs(xr).reshape(T * k, H // 128, 128)
+    hit = blocks.argmax(axis=2)
+    qb = q.reshape(T * k, H // 128, 128)
+    codes = np.take_along_axis(qb, hit[..., None], axis=2)[..., 0]
+    live = blocks.max(axis=2) > 0
+    assert ((codes[live] & 0x7F) == 0x7E).all()
+
+
+# ---------------------------------------------------------------------------
+# combine
+# ---------------------------------------------------------------------------
+
+def _bits(t):
+    return t.view(torch.int16).numpy().view(np.uint16) if t.dtype != torch.float32 else t.numpy()
+
+
+def _from_bits(a, dtype):
+    if dtype == "fp32":
+        return torch.from_numpy(a)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
+    return torch.from_numpy(a.view(np.int16)).view(tdt)
+
+
+def test_combine_hand_worked_example():
+    # two tokens, k=2, H=3; y rows in dispatched order; weights powers of two
+    y = torch.tensor([[1, 2, 3], [4, 5, 6], [8, 16, 32], [0.5, -1, 2]], dtype=torch.bfloat16)
+    out_perm = np.array([2, 0, 3, 1], np.int32)      # token0 -> rows 2,0 ; token1 -> rows 3,1
+    w = np.array([[0.5, 0.25], [2.0, 0.125]], np.float32)
+    got = _from_bits(oracle.combine(_bits(y), "bf16", out_perm, w, "fp32"), "fp32")
+    # token0: 0.5*[8,16,32] + 0.25*[1,2,3] = [4.25, 8.5, 16.75]
+    # token1: 2*[0.5,-1,2] + 0.125*[4,5,6] = [1.5, -1.375, 4.75]
+    assert got.tolist() == [[4.25, 8.5, 16.75], [1.5, -1.375, 4.75]]
+
+
+@pytest.mark.parametrize("y_dtype,out_dtype", [("bf16", "bf16"), ("fp16", "fp16"), ("fp16", "fp32"),
+                                               ("bf16", "fp32"), ("fp32", "bf16"), ("fp32", "fp32")])
+def test_combine_identity_round_trip(y_dtype, out_dtype):
+    """dispatch then combine with weights summing to 1 returns x."""
+    T, H, E, k = 40, 256, 12, 4
+    rng = np.random.default_rng(3)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    tdt = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}[y_dtype]
+    # values on the bf16 grid, so that every output dtype can hold x exactly
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(5)).to(torch.bfloat16).to(tdt)
+    m = oracle.prepare(ids, E)
+    y = oracle.dispatch(_bits(x), k, m["input_perm"])
+    w = rng.random((T, k)).astype(np.float32)
+    w /= w.sum(axis=1, keepdims=True)
+    got = _from_bits(oracle.combine(y, y_dtype, m["output_perm"], w, out_dtype), out_dtype)
+    if out_dtype == y_dtype and out_dtype != "fp32":
+        assert torch.equal(got, x)
+    elif out_dtype == "fp32":
+        torch.testing.assert_close(got, x.float(), rtol=1e-6, atol=0)
+    else:
+        assert torch.equal(got, x.to(got.dtype))
+
+
+def test_combine_one_hot_selects_row_exactly():
+    T, H, k = 16, 128, 6
+    rng = np.random.default_rng(9)
+    y = torch.randn(T * k, H, generator=torch.Generator().manual_seed(1)).to(torch.float16)
+    out_perm = rng.permutation(T * k).astype(np.int32)
+    pick = rng.integers(0, k, T)
+    w = np.zeros((T, k), np.float32)
+    w[np.arange(T), pick] = 1.0
+    got = _from_bits(oracle.combine(_bits(y), "fp16", out_perm, w, "fp16"), "fp16")
+    ref = y[torch.from_numpy(out_perm.reshape(T, k)[np.arange(T), pick]).long()]
+    assert torch.equal(got, ref)
+
+
+def test_combine_within_fp64_error_bound():
+    """|oracle - exact| <= k * 2^-24 * sum_j |w y| + half an output ulp."""
+    w_ = CONFIGS["uniform_t4096_h7168_e256_k8"].scaled(24)
+    ids, wt, _, y = make_workload(w_, with_x=False)
+    m = oracle.prepare(ids, w_.E)
+    got32 = oracle.combine(_bits(y), "bf16", m["output_perm"], wt, "fp32")
+    yy = y.double().numpy()[m["output_perm"]].reshape(w_.T, w_.k, w_.H)
+    exact = np.einsum("tk,tkh->th", wt.astype(np.float64), yy)
+    mag = np.einsum("tk,tkh->th", np.abs(wt.astype(np.float64)), np.abs(yy))
+    assert (np.abs(got32 - exact) <= w_.k * 2.0 ** -24 * mag + 1e-30).all()
+    gotb = _from_bits(oracle.combine(_bits(y), "bf16", m["output_perm"], wt, "bf16"), "bf16")
+    # the bf16 output is the fp32 result rounded once (torch RNE as witness)
+    assert torch.equal(gotb, torch.from_numpy(got32).to(torch.bfloat16))
+
+
+def test_combine_skips_invalid_slots():
+    y = torch.tensor([[1.0, 2.0], [3.0, 4.0]], dtype=torch.float32)
+    out_perm = np.array([1, -1, 0, -1], np.int32)
+    w = np.array([[0.5, 100.0], [2.0, 100.0]], np.float32)
+    got = oracle.combine(y.numpy(), "fp32", out_perm, w, "fp32")
+    np.testing.assert_array_equal(got, [[1.5, 2.0], [2.0, 4.0]])
