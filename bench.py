@@ -1,0 +1,500 @@
+"""Benchmark of the MoE dispatch / combine path on B200.
+
+One step = one pass of the whole path over one batch: routing metadata
+(moe_prepare), dispatch (moe_dispatch_rows, or moe_dispatch_rows_fp8 for the
+fp8 workload) and combine (moe_combine), on seeded synthetic inputs already
+resident in HBM.  Prints ONE JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Multi-GPU runs (torchrun, one process per GPU) are independent replicas:
+the path has no exchange step, so every rank runs the same workload on its
+own GPU and the value is the total over ranks ("scaling": "weak"), timed as
+the maximum over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import CONFIGS, make_workload  # noqa: E402
+
+DEFAULT_WORKLOAD = "uniform_t4096_h7168_e256_k8"
+METRIC = "dispatch+combine tokens/s and effective HBM GB/s (% of B200 peak), 1 GPU"
+SPEC_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+DTYPE_BYTES = {"bf16": 2, "fp16": 2, "fp32": 4, "fp8_e4m3": 1}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(w):
+    """Minimal HBM bytes of each step: every input read once, every output
+    written once (the x row is read once though written k times)."""
+    S, T, H, E = w.S, w.T, w.H, w.E
+    bx = DTYPE_BYTES[w.x_dtype]
+    bd = DTYPE_BYTES[w.dispatch_dtype]
+    by = DTYPE_BYTES[w.y_dtype]
+    bo = DTYPE_BYTES[w.out_dtype]
+    fp8 = w.dispatch_dtype == "fp8_e4m3"
+    prepare = 4 * S + 4 * E + 4 * (E + 1) + 8 * S + (4 * (E + 1) if fp8 else 0)
+    dispatch = T * H * bx + S * H * bd + 4 * S
+    if fp8:
+        dispatch += 4 * S + 4 * S * (H // 128) + 8 * (E + 1)  # ids, scales, offsets
+    combine = S * H * by + 4 * S + 4 * S + T * H * bo
+    return {"prepare": prepare, "dispatch": dispatch, "combine": combine}
+
+
+def src_hash():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "combine_permute_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel_key):
+    """dram read+write bytes per launch from the committed ncu summary, if it
+    was taken on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d["kernels"][kernel_key]
+        return e["dram_bytes_per_launch"] if e.get("src_hash") == src_hash() else None
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML during the timed
+    region (read-only)."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index):
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode() if isinstance(uuid, str) else uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _sample(self):
+        mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+        bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        self.samples.append(mhz)
+        for b, name in self.REASONS.items():
+            if bits & b:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                return
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return None
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples),
+                "source": "nvml"}
+
+
+def percentiles(ms):
+    a = np.asarray(ms)
+    return {"p50": float(np.percentile(a, 50)), "p90": float(np.percentile(a, 90)),
+            "p99": float(np.percentile(a, 99)), "mean": float(a.mean())}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline leg)
+# ---------------------------------------------------------------------------
+
+def _oracle_step(oracle, w, ids, wt, xb, yb):
+    A = w.block_align if w.dispatch_dtype == "fp8_e4m3" else 1
+    m = oracle.prepare(ids, w.E, A)
+    if w.dispatch_dtype == "fp8_e4m3":
+        oracle.dispatch_fp8(xb, w.x_dtype, ids, m)
+    else:
+        oracle.dispatch(xb, w.k, m["input_perm"])
+    oracle.combine(yb, w.y_dtype, m["output_perm"], wt, w.out_dtype)
+
+
+def _host_inputs(w, T_sample):
+    import torch
+    ws = w.scaled(T_sample, name=w.name)
+    ids, wt, x, y = make_workload(ws)
+    xb = x.view(torch.int16).numpy().view(np.uint16) if x.dtype != torch.float32 else x.numpy()
+    yb = y.view(torch.int16).numpy().view(np.uint16) if y.dtype != torch.float32 else y.numpy()
+    return ws, ids, wt, xb, yb
+
+
+def time_oracle(w, budget_s=12.0, steps=None):
+    """Time the oracle's full step on the host.  With ``steps`` None: whole
+    workload steps repeated until ``budget_s`` (at least one).  With
+    ``steps`` K: K steps, each on the first T_s tokens, T_s sized so that
+    the K steps take about ``budget_s``."""
+    import oracle
+    oracle.lib()
+    if steps is None:
+        ws, ids, wt, xb, yb = _host_inputs(w, w.T)
+        n, t0 = 0, time.perf_counter()
+        while True:
+            _oracle_step(oracle, ws, ids, wt, xb, yb)
+            n += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        dt = time.perf_counter() - t0
+        return dict(tokens=n * w.T, seconds=dt, sample=f"{n} full steps of {w.name} ({w.T} tokens each)")
+    # calibrate on a small slice, then size the per-step sample
+    cal_T = max(1, min(w.T, 256))
+    ws, ids, wt, xb, yb = _host_inputs(w, cal_T)
+    t0 = time.perf_counter()
+    _oracle_step(oracle, ws, ids, wt, xb, yb)
+    per_tok = (time.perf_counter() - t0) / cal_T
+    T_s = int(max(1, min(w.T, budget_s / max(steps, 1) / max(per_tok, 1e-9))))
+    ws, ids, wt, xb, yb = _host_inputs(w, T_s)
+    return dict(T_s=T_s, run=lambda: _oracle_step(oracle, ws, ids, wt, xb, yb),
+                sample=f"first {T_s} of {w.T} tokens of {w.name} per step")
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    K, W = args.steps, args.warmup
+    plan = time_oracle(w, budget_s=args.ref_budget, steps=K + W)
+    for _ in range(W):
+        plan["run"]()
+    t0 = time.perf_counter()
+    for _ in range(K):
+        plan["run"]()
+    dt = time.perf_counter() - t0
+    value = plan["T_s"] * K / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": K, "warmup": W, "ms_per_step": dt / K * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": _dtype_tag(w),
+        "data": "synthetic",
+        "config": _config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": plan["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _dtype_tag(w):
+    return w.x_dtype if w.dispatch_dtype != "fp8_e4m3" else "bf16->fp8_e4m3"
+
+
+def _config(w, n):
+    return {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "k": w.k,
+            "routing": w.routing.mode, "x_dtype": w.x_dtype, "dispatch_dtype": w.dispatch_dtype,
+            "y_dtype": w.y_dtype, "out_dtype": w.out_dtype, "seed": w.seed,
+            "l2": "no flush: per-step working set > 126 MB L2",
+            "parallelism": "replicas" if n > 1 else "single GPU"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+class Step:
+    """Device buffers and the three calls of one step."""
+
+    def __init__(self, w, dev):
+        import torch
+        import combine_permute_b200 as moe
+        self.moe, self.w, self.dev = moe, w, dev
+        ids_np, wt_np, x, y = make_workload(w, device=dev)
+        self.ids_np, self.wt_np = ids_np, wt_np
+        self.ids = torch.from_numpy(ids_np).to(dev)
+        self.wt = torch.from_numpy(wt_np).to(dev)
+        self.x, self.y = x, y
+        self.fp8 = w.dispatch_dtype == "fp8_e4m3"
+        self.A = w.block_align if self.fp8 else None
+        i32 = dict(dtype=torch.int32, device=dev)
+        S, E = w.S, w.E
+        self.meta_bufs = dict(expert_counts=torch.empty(E, **i32),
+                              expert_offsets=torch.empty(E + 1, **i32),
+                              blockscale_offsets=torch.empty(E + 1, **i32) if self.fp8 else None,
+                              input_permutation=torch.empty(S, **i32),
+                              output_permutation=torch.empty(S, **i32),
+                              diag=torch.empty(2, **i32))
+        nws = moe.moe_prepare_workspace_bytes(w.T, w.k, E)
+        self.ws = torch.zeros(max(nws, 1), dtype=torch.uint8, device=dev)
+        if self.fp8:
+            self.xq = torch.empty((S, w.H), dtype=torch.uint8, device=dev)
+            self.scales = torch.empty((S + E * (w.block_align - 1), w.H // 128),
+                                      dtype=torch.float32, device=dev)
+        else:
+            self.xd = torch.empty((S, w.H), dtype=x.dtype, device=dev)
+        from workloads.routing import torch_dtype
+        self.out = torch.empty((w.T, w.H), dtype=torch_dtype(w.out_dtype), device=dev)
+        self.launches_per_step = (2 if nws > 0 else 1) + 2
+
+    def prepare(self):
+        return self.moe.moe_prepare(self.ids, self.w.E, blockscale_align=self.A, workspace=self.ws,
+                                    **self.meta_bufs)
+
+    def dispatch(self, meta):
+        if self.fp8:
+            self.moe.moe_dispatch_rows_fp8(self.x, self.ids, meta.output_permutation,
+                                           meta.expert_offsets, meta.blockscale_offsets,
+                                           blockscale_align=self.A, out_q=self.xq,
+                                           out_scales=self.scales)
+        else:
+            self.moe.moe_dispatch_rows(self.x, self.w.k, meta.input_permutation,
+                                       meta.output_permutation, out=self.xd)
+
+    def combine(self, meta):
+        self.moe.moe_combine(self.y, meta.output_permutation, self.wt, out=self.out)
+
+    def run(self):
+        meta = self.prepare()
+        self.dispatch(meta)
+        self.combine(meta)
+
+
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    step = Step(w, dev)
+    K, W = args.steps, args.warmup
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(W):
+        step.run()
+    torch.cuda.synchronize(dev)
+
+    # ---- device-resident timed region: K steps, events around every call
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    marks = [[ev() for _ in range(4)] for _ in range(K)]
+    start, end = ev(), ev()
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for i in range(K):
+            m = marks[i]
+            m[0].record(stream)
+            meta = step.prepare()
+            m[1].record(stream)
+            step.dispatch(meta)
+            m[2].record(stream)
+            step.combine(meta)
+            m[3].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    elapsed_ms = max_over_ranks(start.elapsed_time(end))
+    per = {"prepare": [], "dispatch": [], "combine": [], "step": []}
+    for m in marks:
+        per["prepare"].append(m[0].elapsed_time(m[1]))
+        per["dispatch"].append(m[1].elapsed_time(m[2]))
+        per["combine"].append(m[2].elapsed_time(m[3]))
+        per["step"].append(m[0].elapsed_time(m[3]))
+
+    counts = step.meta_bufs["expert_counts"].cpu().numpy()
+    diag = step.meta_bufs["diag"].cpu().numpy().tolist()
+
+    # ---- end to end through the public API from pinned host buffers
+    e2e = run_e2e(step, w, dev, K, W, barrier, max_over_ranks)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = time_oracle(w, budget_s=args.cpu_budget)
+        cpu = {"value": r["tokens"] / r["seconds"], "unit": "tokens/s", "cores": 1,
+               "kind": "oracle", "sample": r["sample"]}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak, peak_kind = measured_peak()
+    alg = algorithmic_bytes(w)
+    kern = {k: statistics.mean(per[k]) for k in ("prepare", "dispatch", "combine")}
+    dominant = max(("dispatch", "combine"), key=lambda k: kern[k])
+    kernel_key = f"{dominant}@{w.name}"
+    achieved = alg[dominant] / (kern[dominant] * 1e-3) / 1e9
+    tokens = w.T * K * world
+    value = tokens / (elapsed_ms * 1e-3)
+    breakdown = {}
+    for k in ("prepare", "dispatch", "combine"):
+        gbs = alg[k] / (kern[k] * 1e-3) / 1e9
+        breakdown[k] = {"us_mean": kern[k] * 1e3, "latency_ms": percentiles(per[k]),
+                        "tokens_per_s": w.T / (kern[k] * 1e-3), "algorithmic_bytes": alg[k],
+                        "effective_gbs": gbs, "frac_of_measured_peak": gbs / peak,
+                        "frac_of_8tbs_spec": gbs / SPEC_HBM_GBS}
+    e2e_alg = sum(alg.values())
+    breakdown["end_to_end"] = {"latency_ms": percentiles(per["step"]),
+                               "effective_gbs": e2e_alg / (elapsed_ms / K * 1e-3) / 1e9,
+                               "frac_of_measured_peak": e2e_alg / (elapsed_ms / K * 1e-3) / 1e9 / peak}
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": _dtype_tag(w), "data": "synthetic",
+        "config": _config(w, world),
+        "roofline": {"bound": "hbm", "kernel": kernel_key, "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": committed_traffic(kernel_key),
+                     "algorithmic_bytes_per_launch": alg[dominant]},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": step.launches_per_step * K,
+        "clocks": clocks.summary(),
+        "breakdown": breakdown,
+        "expert_load": {"max_tokens_per_expert": int(counts.max()),
+                        "min_tokens_per_expert": int(counts.min()),
+                        "mean_tokens_per_expert": float(counts.mean()),
+                        "imbalance_ratio": float(counts.max() / max(counts.mean(), 1e-9))},
+        "diag": diag,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(step, w, dev, K, W, barrier, max_over_ranks):
+    """Same step through the public API with inputs copied in from pinned
+    host memory and the combined output read back, every step."""
+    import torch
+    h_ids = torch.from_numpy(step.ids_np).pin_memory()
+    h_wt = torch.from_numpy(step.wt_np).pin_memory()
+    h_x = step.x.cpu().pin_memory()
+    h_y = step.y.cpu().pin_memory()
+    h_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_ids, h_wt, h_x, h_y))
+    d2h = h_out.numel() * h_out.element_size()
+    stream = torch.cuda.current_stream(dev)
+    n = max(1, min(K, 20))
+
+    def one():
+        step.ids.copy_(h_ids, non_blocking=True)
+        step.wt.copy_(h_wt, non_blocking=True)
+        step.x.copy_(h_x, non_blocking=True)
+        step.y.copy_(h_y, non_blocking=True)
+        step.run()
+        h_out.copy_(step.out, non_blocking=True)
+
+    for _ in range(min(W, 3)):
+        one()
+    torch.cuda.synchronize(dev)
+    barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(n):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = max_over_ranks(s.elapsed_time(e))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    return {"value": w.T * n * world / (ms * 1e-3), "unit": "tokens/s", "steps": n,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
+    ap.add_argument("--ref-budget", type=float, default=90.0,
+                    help="seconds of oracle time for the whole reference run")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    w = CONFIGS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    main()

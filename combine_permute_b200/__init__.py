@@ -1,0 +1,280 @@
+"""Single-GPU MoE dispatch / combine for B200 (sm_100a).
+
+Python face of libmoe.so.  The functions carry the C ABI's names and take
+torch CUDA tensors; they check shapes and types, allocate outputs with torch
+when none are given (torch is the device-memory and stream plumbing here),
+and call the library on the current CUDA stream.  Every step runs in the
+library's CUDA kernels; if libmoe.so is missing, calls raise.
+
+    meta = moe_prepare(topk_ids, num_experts)                 # routing metadata
+    xd = moe_dispatch_rows(x, k, meta.input_permutation,
+                           meta.output_permutation)           # expert-grouped rows
+    out = moe_combine(y, meta.output_permutation, weights)    # weighted k-way sum
+"""
+
+from __future__ import annotations
+
+from typing import NamedTuple, Optional
+
+import torch
+
+from . import _lib
+from ._lib import MoeError  # noqa: F401
+
+__all__ = [
+    "MoeError",
+    "PrepareResult",
+    "moe_prepare",
+    "moe_prepare_workspace_bytes",
+    "moe_dispatch_rows",
+    "moe_dispatch_rows_fp8",
+    "moe_combine",
+    "moe_prepare_dispatch",
+    "moe_version",
+    "library_path",
+]
+
+_DTYPES = {
+    torch.float32: _lib.MOE_F32,
+    torch.float16: _lib.MOE_F16,
+    torch.bfloat16: _lib.MOE_BF16,
+}
+
+
+class PrepareResult(NamedTuple):
+    expert_counts: torch.Tensor        # [E] int32
+    expert_offsets: torch.Tensor       # [E+1] int32
+    blockscale_offsets: Optional[torch.Tensor]  # [E+1] int32 or None
+    input_permutation: torch.Tensor    # [T*k] int32
+    output_permutation: torch.Tensor   # [T*k] int32
+    diag: torch.Tensor                 # [2] int32: invalid ids, wait gave up
+
+
+def library_path() -> str:
+    return _lib.LIB_PATH
+
+
+def moe_version() -> int:
+    return int(_lib.load().moe_version())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, shape=None, device=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    return t
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt not in _DTYPES:
+        raise ValueError(f"unsupported dtype {dt}")
+    return _DTYPES[dt]
+
+
+# One zero-initialised prepare workspace per (device, stream); the library
+# leaves it zeroed after every call.
+_WORKSPACES: dict = {}
+
+
+def _workspace(device: torch.device, nbytes: int) -> Optional[torch.Tensor]:
+    if nbytes == 0:
+        return None
+    key = (device, torch.cuda.current_stream(device).cuda_stream)
+    ws = _WORKSPACES.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        _WORKSPACES[key] = ws
+    return ws
+
+
+def moe_prepare_workspace_bytes(num_tokens: int, top_k: int, num_experts: int) -> int:
+    return int(_lib.load().moe_prepare_workspace_bytes(num_tokens, top_k, num_experts))
+
+
+def _alloc_meta(device, S, E, with_bso, expert_counts, expert_offsets, blockscale_offsets,
+                input_permutation, output_permutation, diag):
+    i32 = dict(dtype=torch.int32, device=device)
+    ec = expert_counts if expert_counts is not None else torch.empty(E, **i32)
+    eo = expert_offsets if expert_offsets is not None else torch.empty(E + 1, **i32)
+    bs = blockscale_offsets
+    if with_bso and bs is None:
+        bs = torch.empty(E + 1, **i32)
+    ip = input_permutation if input_permutation is not None else torch.empty(S, **i32)
+    op = output_permutation if output_permutation is not None else torch.empty(S, **i32)
+    dg = diag if diag is not None else torch.empty(2, **i32)
+    _need(ec, "expert_counts", torch.int32, (E,), device)
+    _need(eo, "expert_offsets", torch.int32, (E + 1,), device)
+    if bs is not None:
+        _need(bs, "blockscale_offsets", torch.int32, (E + 1,), device)
+    _need(ip, "input_permutation", torch.int32, (S,), device)
+    _need(op, "output_permutation", torch.int32, (S,), device)
+    _need(dg, "diag", torch.int32, (2,), device)
+    return PrepareResult(ec, eo, bs, ip, op, dg)
+
+
+def moe_prepare(topk_ids: torch.Tensor, num_experts: int, *, blockscale_align: Optional[int] = None,
+                expert_counts=None, expert_offsets=None, blockscale_offsets=None,
+                input_permutation=None, output_permutation=None, diag=None,
+                workspace: Optional[torch.Tensor] = None) -> PrepareResult:
+    """Routing metadata of topk_ids [T, k] int32 (see include/moe.h).
+
+    Block-scale offsets are produced when ``blockscale_align`` is given.
+    """
+    _need(topk_ids, "topk_ids", torch.int32)
+    if topk_ids.dim() != 2:
+        raise ValueError("topk_ids must be [T, k]")
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    with torch.cuda.device(dev):
+        meta = _alloc_meta(dev, T * k, num_experts, blockscale_align is not None, expert_counts,
+                           expert_offsets, blockscale_offsets, input_permutation,
+                           output_permutation, diag)
+        need = moe_prepare_workspace_bytes(T, k, num_experts) if T * k > 0 else 0
+        if workspace is None:
+            workspace = _workspace(dev, need)
+        elif need:
+            _need(workspace, "workspace", device=dev)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = _lib.load().moe_prepare(
+            topk_ids.data_ptr(), T, k, num_experts, meta.expert_counts.data_ptr(),
+            meta.expert_offsets.data_ptr(), _ptr(meta.blockscale_offsets),
+            blockscale_align or 1, meta.input_permutation.data_ptr(),
+            meta.output_permutation.data_ptr(), meta.diag.data_ptr(), _ptr(workspace), ws_bytes,
+            _stream(dev))
+    _lib.check("moe_prepare", st)
+    return meta
+
+
+def moe_dispatch_rows(x: torch.Tensor, top_k: int, input_permutation: Optional[torch.Tensor] = None,
+                      output_permutation: Optional[torch.Tensor] = None,
+                      out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out[p] = x[input_permutation[p] // k] (see include/moe.h)."""
+    _need(x, "x")
+    if x.dim() != 2:
+        raise ValueError("x must be [T, H]")
+    T, H = x.shape
+    S = T * top_k
+    dev = x.device
+    for name, t in (("input_permutation", input_permutation),
+                    ("output_permutation", output_permutation)):
+        if t is not None:
+            _need(t, name, torch.int32, (S,), dev)
+    if out is None:
+        out = torch.empty((S, H), dtype=x.dtype, device=dev)
+    _need(out, "out", x.dtype, (S, H), dev)
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_dispatch_rows(x.data_ptr(), _dtype_code(x.dtype), T, H, top_k,
+                                           _ptr(input_permutation), _ptr(output_permutation),
+                                           out.data_ptr(), _stream(dev))
+    _lib.check("moe_dispatch_rows", st)
+    return out
+
+
+def moe_dispatch_rows_fp8(x: torch.Tensor, topk_ids: torch.Tensor, output_permutation: torch.Tensor,
+                          expert_offsets: torch.Tensor, blockscale_offsets: torch.Tensor, *,
+                          blockscale_align: int = 1, out_q: Optional[torch.Tensor] = None,
+                          out_scales: Optional[torch.Tensor] = None):
+    """FP8 E4M3 1x128 block-scale dispatch.  Returns (out_q uint8 [T*k, H],
+    out_scales fp32 [rows, H/128]).
+
+    Without ``out_scales`` the scale tensor is allocated with the upper bound
+    T*k + E*(blockscale_align - 1) rows (no device-to-host read).
+    """
+    _need(x, "x")
+    _need(topk_ids, "topk_ids", torch.int32)
+    T, H = x.shape
+    k = topk_ids.shape[1]
+    E = expert_offsets.numel() - 1
+    S = T * k
+    dev = x.device
+    _need(topk_ids, "topk_ids", torch.int32, (T, k), dev)
+    _need(output_permutation, "output_permutation", torch.int32, (S,), dev)
+    _need(expert_offsets, "expert_offsets", torch.int32, (E + 1,), dev)
+    _need(blockscale_offsets, "blockscale_offsets", torch.int32, (E + 1,), dev)
+    if x.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError("fp8 dispatch reads bf16 or fp16 activations")
+    if out_q is None:
+        out_q = torch.empty((S, H), dtype=torch.uint8, device=dev)
+    if out_q.dtype == torch.float8_e4m3fn:
+        out_q = out_q.view(torch.uint8)
+    _need(out_q, "out_q", torch.uint8, (S, H), dev)
+    if out_scales is None:
+        out_scales = torch.empty((S + E * (blockscale_align - 1), H // 128), dtype=torch.float32,
+                                 device=dev)
+    _need(out_scales, "out_scales", torch.float32, None, dev)
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_dispatch_rows_fp8(
+            x.data_ptr(), _dtype_code(x.dtype), T, H, k, E, topk_ids.data_ptr(),
+            output_permutation.data_ptr(), expert_offsets.data_ptr(),
+            blockscale_offsets.data_ptr(), out_q.data_ptr(), out_scales.data_ptr(), _stream(dev))
+    _lib.check("moe_dispatch_rows_fp8", st)
+    return out_q, out_scales
+
+
+def moe_combine(y: torch.Tensor, output_permutation: torch.Tensor, weights: torch.Tensor, *,
+                out_dtype: Optional[torch.dtype] = None,
+                out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out[t] = sum_j weights[t, j] * y[output_permutation[t*k + j]] (fp32
+    accumulation, see include/moe.h)."""
+    _need(y, "y")
+    _need(weights, "weights", torch.float32)
+    T, k = weights.shape
+    S, H = y.shape
+    dev = y.device
+    if S != T * k:
+        raise ValueError("y must have T*k rows")
+    _need(output_permutation, "output_permutation", torch.int32, (S,), dev)
+    _need(weights, "weights", torch.float32, (T, k), dev)
+    if out is None:
+        out = torch.empty((T, H), dtype=out_dtype or y.dtype, device=dev)
+    _need(out, "out", None, (T, H), dev)
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_combine(y.data_ptr(), _dtype_code(y.dtype), T, H, k,
+                                     output_permutation.data_ptr(), weights.data_ptr(),
+                                     out.data_ptr(), _dtype_code(out.dtype), _stream(dev))
+    _lib.check("moe_combine", st)
+    return out
+
+
+def moe_prepare_dispatch(topk_ids: torch.Tensor, num_experts: int, x: torch.Tensor, *,
+                         blockscale_align: Optional[int] = None, out: Optional[torch.Tensor] = None,
+                         expert_counts=None, expert_offsets=None, blockscale_offsets=None,
+                         input_permutation=None, output_permutation=None, diag=None):
+    """moe_prepare + moe_dispatch_rows in one launch for tiny batches.
+    Returns (PrepareResult, dispatched rows)."""
+    _need(topk_ids, "topk_ids", torch.int32)
+    _need(x, "x")
+    T, k = topk_ids.shape
+    H = x.shape[1]
+    dev = x.device
+    _need(x, "x", None, (T, H), dev)
+    meta = _alloc_meta(dev, T * k, num_experts, blockscale_align is not None, expert_counts,
+                       expert_offsets, blockscale_offsets, input_permutation, output_permutation,
+                       diag)
+    if out is None:
+        out = torch.empty((T * k, H), dtype=x.dtype, device=dev)
+    _need(out, "out", x.dtype, (T * k, H), dev)
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_prepare_dispatch(
+            topk_ids.data_ptr(), T, k, num_experts, meta.expert_counts.data_ptr(),
+            meta.expert_offsets.data_ptr(), _ptr(meta.blockscale_offsets), blockscale_align or 1,
+            meta.input_permutation.data_ptr(), meta.output_permutation.data_ptr(),
+            meta.diag.data_ptr(), x.data_ptr(), _dtype_code(x.dtype), H, out.data_ptr(),
+            _stream(dev))
+    _lib.check("moe_prepare_dispatch", st)
+    return meta, out

@@ -1,0 +1,158 @@
+// extern "C" entry points of libmoe: host-side argument validation, then the
+// launchers in prepare.cu / dispatch.cu / combine.cu.  Contracts are stated
+// in include/moe.h.  No entry point allocates memory or synchronises.
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+#include "kernels.h"
+
+namespace {
+
+constexpr int64_t kMaxSlots = (int64_t)1 << 31;
+
+inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+inline bool io_dtype(moe_dtype_t d) { return d == MOE_F32 || d == MOE_F16 || d == MOE_BF16; }
+
+inline moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+inline moe::DType dt(moe_dtype_t d) { return static_cast<moe::DType>(static_cast<int>(d)); }
+
+// Checks shared by every call that takes (T, k).
+inline moe_status_t check_tk(int64_t T, int32_t k) {
+    if (T < 0 || k < 1) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && T * (int64_t)k >= kMaxSlots) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_status_string(moe_status_t s) {
+    switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: outside the supported sizes or types";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA launch or runtime call failed";
+    }
+    return "unknown moe_status_t";
+}
+
+int32_t moe_version(void) { return 10000; }
+
+size_t moe_prepare_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t num_experts) {
+    if (num_tokens < 0 || top_k < 1 || num_experts < 1) return 0;
+    return moe::prepare_workspace_bytes(num_tokens * (int64_t)top_k, num_experts);
+}
+
+moe_status_t moe_prepare(const int32_t *topk_ids, int64_t num_tokens, int32_t top_k,
+                         int32_t num_experts, int32_t *expert_counts, int32_t *expert_offsets,
+                         int32_t *blockscale_offsets, int32_t blockscale_align,
+                         int32_t *input_permutation, int32_t *output_permutation, int32_t *diag,
+                         void *workspace, size_t workspace_bytes, moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (num_experts < 1) return MOE_ERR_INVALID_ARG;
+    if (num_experts > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    if (!expert_counts || !expert_offsets || !input_permutation || !output_permutation)
+        return MOE_ERR_INVALID_ARG;
+    if (num_tokens > 0 && !topk_ids) return MOE_ERR_INVALID_ARG;
+    if (blockscale_offsets && blockscale_align < 1) return MOE_ERR_INVALID_ARG;
+    const int64_t S = num_tokens * (int64_t)top_k;
+    const size_t need = moe::prepare_workspace_bytes(S, num_experts);
+    if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
+        return MOE_ERR_WORKSPACE;
+    return from_cuda(moe::run_prepare(topk_ids, S, num_experts,
+                                      blockscale_offsets ? blockscale_align : 1, expert_counts,
+                                      expert_offsets, blockscale_offsets, input_permutation,
+                                      output_permutation, diag, workspace,
+                                      (cudaStream_t)stream));
+}
+
+moe_status_t moe_dispatch_rows(const void *x, moe_dtype_t dtype, int64_t num_tokens,
+                               int64_t hidden, int32_t top_k, const int32_t *input_permutation,
+                               const int32_t *output_permutation, void *out,
+                               moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (!io_dtype(dtype) || hidden < 1) return MOE_ERR_INVALID_ARG;
+    const int64_t row_bytes = hidden * moe::dtype_bytes(dt(dtype));
+    if (row_bytes % 16 != 0) return MOE_ERR_INVALID_ARG;
+    if (num_tokens == 0) return MOE_OK;
+    if (!x || !out || (!input_permutation && !output_permutation)) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    if (output_permutation)
+        return from_cuda(moe::run_dispatch_scatter(x, num_tokens, row_bytes, top_k,
+                                                   output_permutation, out, (cudaStream_t)stream));
+    return from_cuda(moe::run_dispatch_gather(x, num_tokens, row_bytes, top_k, input_permutation,
+                                              out, (cudaStream_t)stream));
+}
+
+moe_status_t moe_dispatch_rows_fp8(const void *x, moe_dtype_t x_dtype, int64_t num_tokens,
+                                   int64_t hidden, int32_t top_k, int32_t num_experts,
+                                   const int32_t *topk_ids, const int32_t *output_permutation,
+                                   const int32_t *expert_offsets,
+                                   const int32_t *blockscale_offsets, uint8_t *out_q,
+                                   float *out_scales, moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (x_dtype != MOE_BF16 && x_dtype != MOE_F16) return MOE_ERR_UNSUPPORTED;
+    if (hidden < 1 || hidden % 128 != 0 || num_experts < 1) return MOE_ERR_INVALID_ARG;
+    if (num_tokens == 0) return MOE_OK;
+    if (!x || !topk_ids || !output_permutation || !expert_offsets || !blockscale_offsets ||
+        !out_q || !out_scales)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out_q) || ((uintptr_t)out_scales & 3u))
+        return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_dispatch_fp8(x, dt(x_dtype), num_tokens, hidden, top_k, num_experts, topk_ids,
+                                           output_permutation, expert_offsets,
+                                           blockscale_offsets, out_q, out_scales,
+                                           (cudaStream_t)stream));
+}
+
+moe_status_t moe_combine(const void *y, moe_dtype_t y_dtype, int64_t num_tokens, int64_t hidden,
+                         int32_t top_k, const int32_t *output_permutation, const float *weights,
+                         void *out, moe_dtype_t out_dtype, moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (!io_dtype(y_dtype) || !io_dtype(out_dtype) || hidden < 1) return MOE_ERR_INVALID_ARG;
+    if ((hidden * moe::dtype_bytes(dt(y_dtype))) % 16 != 0 ||
+        (hidden * moe::dtype_bytes(dt(out_dtype))) % 16 != 0)
+        return MOE_ERR_INVALID_ARG;
+    if (num_tokens == 0) return MOE_OK;
+    if (!y || !output_permutation || !weights || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(out) || ((uintptr_t)weights & 3u)) return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_combine(y, dt(y_dtype), num_tokens, hidden, top_k,
+                                      output_permutation, weights, out, dt(out_dtype),
+                                      (cudaStream_t)stream));
+}
+
+moe_status_t moe_prepare_dispatch(const int32_t *topk_ids, int64_t num_tokens, int32_t top_k,
+                                  int32_t num_experts, int32_t *expert_counts,
+                                  int32_t *expert_offsets, int32_t *blockscale_offsets,
+                                  int32_t blockscale_align, int32_t *input_permutation,
+                                  int32_t *output_permutation, int32_t *diag, const void *x,
+                                  moe_dtype_t dtype, int64_t hidden, void *out,
+                                  moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (num_experts < 1 || !io_dtype(dtype) || hidden < 1) return MOE_ERR_INVALID_ARG;
+    if (num_experts > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    const int64_t S = num_tokens * (int64_t)top_k;
+    if (S > moe::kFusedMaxSlots) return MOE_ERR_UNSUPPORTED;
+    const int64_t row_bytes = hidden * moe::dtype_bytes(dt(dtype));
+    if (row_bytes % 16 != 0) return MOE_ERR_INVALID_ARG;
+    if (!expert_counts || !expert_offsets || !input_permutation || !output_permutation)
+        return MOE_ERR_INVALID_ARG;
+    if (blockscale_offsets && blockscale_align < 1) return MOE_ERR_INVALID_ARG;
+    if (num_tokens > 0 && (!topk_ids || !x || !out)) return MOE_ERR_INVALID_ARG;
+    if (num_tokens > 0 && (!aligned16(x) || !aligned16(out))) return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_prepare_dispatch(
+        topk_ids, num_tokens, top_k, num_experts, blockscale_offsets ? blockscale_align : 1,
+        expert_counts, expert_offsets, blockscale_offsets, input_permutation, output_permutation,
+        diag, x, row_bytes, out, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,190 @@
+// Dispatch: lay token rows out grouped by expert (sglang PR #19058,
+// "Changes", item 2 shuffle_rows: dtype-agnostic row gather with 128-bit
+// vector accesses), and the same with a fused FP8 E4M3 1x128 block-scale
+// quantisation (the FP8 block-scale MoE path of TensorRT-LLM PR #9592).
+//
+// dispatch_scatter_kernel walks tokens: it reads each x row once into
+// registers (16-byte vectors) and stores it to the token's k dispatched
+// rows, so x crosses HBM once although it is written k times.
+// dispatch_gather_kernel walks dispatched rows and reads the source row
+// through input_permutation (the literal shuffle_rows form).
+// Both are persistent grid-stride kernels sized to fill every SM once.
+#include "kernels.h"
+#include "launch.h"
+#include "moe_device.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kCopyThreads = 128;
+constexpr int kCopyUnroll = 8;  // 16-byte vectors in flight per thread
+
+__global__ void __launch_bounds__(kCopyThreads)
+    dispatch_scatter_kernel(const uint4 *__restrict__ x, int64_t T, int64_t nvec, int k,
+                            const int32_t *__restrict__ out_perm, uint4 *__restrict__ out) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t S = T * k;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        const uint4 *src = x + t * nvec;
+        const int32_t *dst_rows = out_perm + t * k;
+        for (int64_t c0 = threadIdx.x; c0 < nvec; c0 += kCopyThreads * kCopyUnroll) {
+            uint4 v[kCopyUnroll];
+#pragma unroll
+            for (int u = 0; u < kCopyUnroll; ++u) {
+                const int64_t c = c0 + u * kCopyThreads;
+                if (c < nvec) v[u] = ld_stream_v4(src + c);
+            }
+            for (int j = 0; j < k; ++j) {
+                const int p = __ldg(dst_rows + j);
+                if (p < 0 || p >= S) continue;  // invalid slot (or a corrupt entry)
+                uint4 *dst = out + (int64_t)p * nvec;
+#pragma unroll
+                for (int u = 0; u < kCopyUnroll; ++u) {
+                    const int64_t c = c0 + u * kCopyThreads;
+                    if (c < nvec) st_v4(dst + c, v[u]);
+                }
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kCopyThreads)
+    dispatch_gather_kernel(const uint4 *__restrict__ x, int64_t S, int64_t nvec, int k,
+                           const int32_t *__restrict__ in_perm, uint4 *__restrict__ out) {
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int64_t p = blockIdx.x; p < S; p += gridDim.x) {
+        const int i = __ldg(in_perm + p);
+        if (i < 0 || i >= S) continue;
+        const uint4 *src = x + (int64_t)(i / k) * nvec;
+        uint4 *dst = out + p * nvec;
+        for (int64_t c0 = threadIdx.x; c0 < nvec; c0 += kCopyThreads * kCopyUnroll) {
+            uint4 v[kCopyUnroll];
+#pragma unroll
+            for (int u = 0; u < kCopyUnroll; ++u) {
+                const int64_t c = c0 + u * kCopyThreads;
+                if (c < nvec) v[u] = ld_stream_v4(src + c);
+            }
+#pragma unroll
+            for (int u = 0; u < kCopyUnroll; ++u) {
+                const int64_t c = c0 + u * kCopyThreads;
+                if (c < nvec) st_v4(dst + c, v[u]);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// FP8 dispatch.  Each thread owns 16 consecutive elements of a token row (two
+// 16-byte loads); the 8 threads of one 128-column block reduce amax with
+// shuffles, divide by s = amax / 448 in IEEE fp32 and convert pairs with
+// cvt.rn.satfinite.e4m3x2.  The quantised row is computed once per token
+// and stored to its k dispatched rows; the first thread of each block also
+// stores s into the expert's scale segment.
+// ---------------------------------------------------------------------------
+constexpr int kFp8Threads = 256;
+
+template <typename XT>
+__device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
+    const XT *h = reinterpret_cast<const XT *>(&v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = Elem<XT>::to_f32(h[e]);
+}
+
+template <typename XT>
+__global__ void __launch_bounds__(kFp8Threads)
+    dispatch_fp8_kernel(const XT *__restrict__ x, int64_t T, int64_t H, int k, int E,
+                        const int32_t *__restrict__ ids, const int32_t *__restrict__ out_perm,
+                        const int32_t *__restrict__ offsets, const int32_t *__restrict__ bso,
+                        uint8_t *__restrict__ q, float *__restrict__ scales) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t n16 = H / 16;  // 16-element groups per row
+    const int64_t nb = H / 128;
+    const int64_t S = T * k;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        for (int64_t g = threadIdx.x; g < n16; g += kFp8Threads) {
+            const XT *src = x + t * H + g * 16;
+            float f[16];
+            unpack8<XT>(ld_stream_v4(src), f);
+            unpack8<XT>(ld_stream_v4(src + 8), f + 8);
+            float amax = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
+            // the 8 groups of one 128-column block are 8 consecutive lanes,
+            // active together (H is a multiple of 128); lanes past the row
+            // end have left the loop
+            const int64_t rem = n16 - (g - (threadIdx.x & 31));
+            const unsigned m = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+            amax = fmaxf(amax, __shfl_xor_sync(m, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(m, amax, 2));
+            amax = fmaxf(amax, __shfl_xor_sync(m, amax, 4));
+            uint4 packed = make_uint4(0u, 0u, 0u, 0u);
+            float s = 0.0f;
+            if (amax != 0.0f) {
+                s = __fdiv_rn(amax, 448.0f);
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint16_t lo = cvt_e4m3x2(__fdiv_rn(f[4 * e], s), __fdiv_rn(f[4 * e + 1], s));
+                    const uint16_t hi =
+                        cvt_e4m3x2(__fdiv_rn(f[4 * e + 2], s), __fdiv_rn(f[4 * e + 3], s));
+                    w[e] = (uint32_t)lo | ((uint32_t)hi << 16);
+                }
+                packed = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            const bool block_lead = (g & 7) == 0;
+            const int64_t b = g >> 3;
+            for (int j = 0; j < k; ++j) {
+                const int64_t i = t * k + j;
+                const int p = __ldg(out_perm + i);
+                if (p < 0 || p >= S) continue;
+                const int e = __ldg(ids + i);
+                if (e < 0 || e >= E) continue;
+                st_v4(q + (int64_t)p * H + g * 16, packed);
+                if (block_lead) {
+                    const int64_t srow = (int64_t)__ldg(bso + e) + (p - __ldg(offsets + e));
+                    scales[srow * nb + b] = s;
+                }
+            }
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t run_dispatch_scatter(const void *x, int64_t T, int64_t row_bytes, int k,
+                                 const int32_t *out_perm, void *out, cudaStream_t stream) {
+    const int64_t nvec = row_bytes / 16;
+    const int64_t grid = persistent_grid(dispatch_scatter_kernel, kCopyThreads, 0, T);
+    return launch(dispatch_scatter_kernel, grid, kCopyThreads, 0, stream, (const uint4 *)x, T,
+                  nvec, k, out_perm, (uint4 *)out);
+}
+
+cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int k,
+                                const int32_t *in_perm, void *out, cudaStream_t stream) {
+    const int64_t nvec = row_bytes / 16;
+    const int64_t S = T * k;
+    const int64_t grid = persistent_grid(dispatch_gather_kernel, kCopyThreads, 0, S);
+    return launch(dispatch_gather_kernel, grid, kCopyThreads, 0, stream, (const uint4 *)x, S,
+                  nvec, k, in_perm, (uint4 *)out);
+}
+
+cudaError_t run_dispatch_fp8(const void *x, DType x_dtype, int64_t T, int64_t H, int k, int E,
+                             const int32_t *ids, const int32_t *out_perm, const int32_t *offsets,
+                             const int32_t *bso, uint8_t *q, float *scales, cudaStream_t stream) {
+    if (x_dtype == DType::BF16) {
+        auto kern = dispatch_fp8_kernel<__nv_bfloat16>;
+        const int64_t grid = persistent_grid(kern, kFp8Threads, 0, T);
+        return launch(kern, grid, kFp8Threads, 0, stream, (const __nv_bfloat16 *)x, T, H, k, E, ids,
+                      out_perm, offsets, bso, q, scales);
+    }
+    auto kern = dispatch_fp8_kernel<__half>;
+    const int64_t grid = persistent_grid(kern, kFp8Threads, 0, T);
+    return launch(kern, grid, kFp8Threads, 0, stream, (const __half *)x, T, H, k, E, ids, out_perm,
+                  offsets, bso, q, scales);
+}
+
+}  // namespace moe

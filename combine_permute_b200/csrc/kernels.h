@@ -1,0 +1,53 @@
+// Internal launchers behind the C ABI (see include/moe.h for the contracts).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+enum class DType : int { F32 = 0, F16 = 1, BF16 = 2, FP8_E4M3 = 3 };
+
+inline int dtype_bytes(DType d) {
+    return d == DType::F32 ? 4 : (d == DType::FP8_E4M3 ? 1 : 2);
+}
+
+// Prepare: a problem with at most kSingleBlockSlots slots runs as one block;
+// larger ones as tiles of kPrepTile slots in two kernels.
+constexpr int kPrepThreads = 512;
+constexpr int kPrepWarps = kPrepThreads / 32;
+constexpr int kPrepRounds = 8;
+constexpr int kWarpChunk = 32 * kPrepRounds;       // slots per warp per tile
+constexpr int kPrepTile = kPrepThreads * kPrepRounds;  // slots per tile
+constexpr int kSingleBlockSlots = kPrepTile;
+constexpr int kMaxExperts = 1024;
+constexpr int kFusedMaxSlots = 4096;
+
+size_t prepare_workspace_bytes(int64_t S, int E);
+
+cudaError_t run_prepare(const int32_t *ids, int64_t S, int E, int A, int32_t *counts,
+                        int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,
+                        int32_t *diag, void *workspace, cudaStream_t stream);
+
+cudaError_t run_prepare_dispatch(const int32_t *ids, int64_t T, int k, int E, int A,
+                                 int32_t *counts, int32_t *offsets, int32_t *bso,
+                                 int32_t *in_perm, int32_t *out_perm, int32_t *diag,
+                                 const void *x, int64_t row_bytes, void *out,
+                                 cudaStream_t stream);
+
+cudaError_t run_dispatch_scatter(const void *x, int64_t T, int64_t row_bytes, int k,
+                                 const int32_t *out_perm, void *out, cudaStream_t stream);
+
+cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int k,
+                                const int32_t *in_perm, void *out, cudaStream_t stream);
+
+cudaError_t run_dispatch_fp8(const void *x, DType x_dtype, int64_t T, int64_t H, int k, int E,
+                             const int32_t *ids, const int32_t *out_perm, const int32_t *offsets,
+                             const int32_t *bso, uint8_t *q, float *scales, cudaStream_t stream);
+
+cudaError_t run_combine(const void *y, DType y_dtype, int64_t T, int64_t H, int k,
+                        const int32_t *out_perm, const float *w, void *out, DType out_dtype,
+                        cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,87 @@
+// Host-side launch helpers: SM count and occupancy caches, and a launcher
+// that enables programmatic dependent launch on every kernel.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <map>
+#include <mutex>
+#include <tuple>
+
+namespace moe {
+
+inline int current_device() {
+    int d = 0;
+    cudaGetDevice(&d);
+    return d;
+}
+
+inline int sm_count() {
+    static std::mutex mu;
+    static std::map<int, int> cache;
+    const int dev = current_device();
+    std::lock_guard<std::mutex> g(mu);
+    auto it = cache.find(dev);
+    if (it != cache.end()) return it->second;
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 1;
+    cache[dev] = n;
+    return n;
+}
+
+// Resident blocks per SM of `kernel` at this block size and dynamic shared
+// memory, memoised per (kernel, block size, smem, device).  Also raises the
+// kernel's dynamic shared-memory limit when the request is above the 48 KB
+// default.
+template <typename Kernel>
+int blocks_per_sm(Kernel kernel, int threads, size_t smem) {
+    static std::mutex mu;
+    static std::map<std::tuple<const void *, int, size_t, int>, int> cache;
+    const int dev = current_device();
+    const auto key = std::make_tuple((const void *)kernel, threads, smem, dev);
+    std::lock_guard<std::mutex> g(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    if (smem > 48 * 1024)
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess ||
+        n <= 0) {
+        cudaGetLastError();
+        n = 1;
+    }
+    cache[key] = n;
+    return n;
+}
+
+// Grid for a grid-stride kernel over `units` work items: never more blocks
+// than items, never more than fill the GPU once.
+template <typename Kernel>
+int64_t persistent_grid(Kernel kernel, int threads, size_t smem, int64_t units) {
+    const int64_t full = (int64_t)sm_count() * blocks_per_sm(kernel, threads, smem);
+    return units < full ? (units > 0 ? units : 1) : full;
+}
+
+// Launch with programmatic stream serialization (PDL) enabled.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), int64_t grid, int threads, size_t smem,
+                   cudaStream_t stream, Args &&...args) {
+    if (smem > 48 * 1024) blocks_per_sm(kernel, threads, smem);  // sets the smem limit once
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace moe

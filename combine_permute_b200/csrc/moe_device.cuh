@@ -1,0 +1,128 @@
+// Device-side helpers shared by the sm_100a kernels of libmoe.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+constexpr int kWarp = 32;
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch (PTX griddepcontrol, sm_90+).  Every kernel
+// waits for its stream predecessor before touching global memory the
+// predecessor may write or read, and lets its own dependents launch early.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Memory access helpers.
+// ---------------------------------------------------------------------------
+
+// 16-byte read of data that stays constant for the whole kernel, not kept in
+// L1 (each row is read once per block).
+__device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_v4(void *p, const uint4 &v) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// ---------------------------------------------------------------------------
+// Element conversions (CUDA intrinsics, round to nearest even).
+// ---------------------------------------------------------------------------
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    __device__ static float to_f32(float v) { return v; }
+    __device__ static float from_f32(float v) { return v; }
+};
+template <> struct Elem<__half> {
+    __device__ static float to_f32(__half v) { return __half2float(v); }
+    __device__ static __half from_f32(float v) { return __float2half_rn(v); }
+};
+template <> struct Elem<__nv_bfloat16> {
+    __device__ static float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+    __device__ static __nv_bfloat16 from_f32(float v) { return __float2bfloat16_rn(v); }
+};
+
+// Two fp32 values -> two OCP E4M3 bytes (round to nearest even, finite
+// results saturate to +-448).  `lo` lands in the low byte.
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// Block-wide exclusive scan of n <= 4 * blockDim.x ints held in shared
+// memory (in place).  Returns the total.  All threads must call it.
+// `warp_tmp` needs blockDim.x / 32 + 1 ints.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int block_exclusive_scan(int *data, int n, int *warp_tmp) {
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int per = (n + nt - 1) / nt;
+    const int beg = min(n, tid * per), end = min(n, beg + per);
+    int local = 0;
+    for (int i = beg; i < end; ++i) local += data[i];
+    // inclusive warp scan of the per-thread sums
+    const int lane = tid & 31, warp = tid >> 5;
+    int v = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    if (lane == 31) warp_tmp[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        const int nw = nt >> 5;
+        int w = lane < nw ? warp_tmp[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int u = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += u;
+        }
+        if (lane < nw) warp_tmp[lane] = w;  // inclusive warp totals
+        if (lane == nw - 1) warp_tmp[32] = w;
+    }
+    __syncthreads();
+    int run = v - local + (warp > 0 ? warp_tmp[warp - 1] : 0);
+    for (int i = beg; i < end; ++i) {
+        int c = data[i];
+        data[i] = run;
+        run += c;
+    }
+    const int total = warp_tmp[32];
+    __syncthreads();
+    return total;
+}
+
+}  // namespace moe

@@ -1,0 +1,232 @@
+/*
+ * moe.h - C ABI of the single-GPU MoE dispatch / combine library (libmoe.so,
+ * CUDA kernels for sm_100a).
+ *
+ * The path has three steps, named after the kernels of sglang PR #19058
+ * "[jit_kernel] Add prepare_moe_input JIT kernels", section "Changes":
+ *
+ *   1. moe_prepare         routing metadata (prepare_moe_input: tokens per
+ *                          expert, prefix-sum expert offsets, optional FP8
+ *                          block-scale offsets, input/output permutations);
+ *   2. moe_dispatch_rows   the row gather that lays token rows out grouped by
+ *                          expert (shuffle_rows), and moe_dispatch_rows_fp8,
+ *                          the same with a fused FP8 E4M3 1x128 block-scale
+ *                          quantisation (the FP8 block-scale MoE path of
+ *                          TensorRT-LLM PR #9592);
+ *   3. moe_combine         gather + scale by router weight + reduce over the
+ *                          k slots with fp32 accumulation
+ *                          (apply_shuffle_mul_sum).
+ *
+ * Notation: T tokens, H hidden size, E experts, k slots per token (top-k),
+ * S = T*k.  The expanded index of slot j of token t is i = t*k + j; the
+ * permuted index p is the row of the dispatched (expert-grouped) tensor
+ * (TensorRT-LLM PR #9592 names these expanded_idx / permuted_idx).
+ *
+ * Conventions shared by every entry point:
+ *  - All array arguments are caller-owned DEVICE memory, row-major and
+ *    densely packed.  The library never allocates device or host memory and
+ *    keeps no state between calls apart from a per-device cache of launch
+ *    sizes (guarded by a mutex).
+ *  - Every call is asynchronous: it validates its arguments on the host,
+ *    enqueues its kernels on `stream` (NULL = the legacy default stream) and
+ *    returns without synchronising.  Kernels are launched with programmatic
+ *    dependent launch, so consecutive calls on one stream overlap their
+ *    launch latency while still seeing each other's results.
+ *  - Host-side validation failures return MOE_ERR_INVALID_ARG or
+ *    MOE_ERR_UNSUPPORTED and launch nothing.  A failed launch returns
+ *    MOE_ERR_CUDA (the CUDA error is consumed with cudaGetLastError).
+ *  - Outputs must not alias inputs.
+ *  - Index tensors are int32; T*k must be < 2^31.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the same pointer type; this header does not need the CUDA
+ * headers). */
+typedef struct CUstream_st *moe_stream_t;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1, /* null pointer, negative size, bad alignment ... */
+    MOE_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels support    */
+    MOE_ERR_WORKSPACE = 3,   /* workspace missing or too small                */
+    MOE_ERR_CUDA = 4         /* a CUDA launch or runtime call failed          */
+} moe_status_t;
+
+typedef enum {
+    MOE_F32 = 0,
+    MOE_F16 = 1,
+    MOE_BF16 = 2,
+    MOE_FP8_E4M3 = 3 /* OCP E4M3 "FN": no infinities, max finite 448 */
+} moe_dtype_t;
+
+/* Largest expert count the prepare kernels accept. */
+#define MOE_MAX_EXPERTS 1024
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *moe_status_string(moe_status_t status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int32_t moe_version(void);
+
+/*
+ * Bytes of scratch workspace moe_prepare needs for this problem size (0 when
+ * the problem is small enough for the single-block path).  The workspace
+ * must be all-zero before its first use (e.g. one cudaMemsetAsync); every
+ * completed call leaves it all-zero again, so one workspace serves any
+ * number of consecutive calls on one stream.  Calls that may run
+ * concurrently need separate workspaces.  After a call that reported a
+ * CUDA error, zero it again.
+ */
+size_t moe_prepare_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t num_experts);
+
+/*
+ * Routing metadata (sglang PR #19058, "Changes", item 1 prepare_moe_input:
+ * compute_problem_sizes_kernel counts tokens per expert,
+ * compute_expert_offsets_kernel prefix-sums them,
+ * compute_expert_blockscale_offsets_kernel gives the optional FP8
+ * block-scale offsets, compute_arg_sorts_kernel builds the input and output
+ * permutations).
+ *
+ *   topk_ids            [T, k] int32   expert id of every slot.
+ *   expert_counts       [E]    int32   out: slots routed to each expert.
+ *   expert_offsets      [E+1]  int32   out: exclusive prefix sum of the
+ *                                      counts; expert_offsets[E] is the
+ *                                      number of valid slots.
+ *   blockscale_offsets  [E+1]  int32   out, optional (NULL to skip):
+ *                                      exclusive prefix sum of the counts
+ *                                      each rounded up to a multiple of
+ *                                      blockscale_align (>= 1).
+ *   input_permutation   [T*k]  int32   out: input_permutation[p] = i, the
+ *                                      expanded index of dispatched row p;
+ *                                      -1 for p >= expert_offsets[E].
+ *   output_permutation  [T*k]  int32   out: the inverse, output_permutation[i]
+ *                                      = p; -1 for slots with an invalid id.
+ *   diag                [2]    int32   out, optional: diag[0] = number of ids
+ *                                      outside [0, E); diag[1] = 1 if a
+ *                                      bounded inter-block wait gave up (the
+ *                                      other outputs are then invalid), else
+ *                                      0.
+ *   workspace                          scratch of moe_prepare_workspace_bytes()
+ *                                      bytes, 256-byte aligned, zero on entry
+ *                                      (see above); may be NULL when that
+ *                                      size is 0.
+ *
+ * Dispatched order: by expert ascending, and within an expert by expanded
+ * index ascending (token, then slot): a stable counting sort, so the result
+ * is deterministic.  Ids outside [0, E) are not counted and get no row; the
+ * call still succeeds (check diag[0]).  T = 0 writes zero counts/offsets.
+ */
+moe_status_t moe_prepare(const int32_t *topk_ids, int64_t num_tokens, int32_t top_k,
+                         int32_t num_experts, int32_t *expert_counts, int32_t *expert_offsets,
+                         int32_t *blockscale_offsets, int32_t blockscale_align,
+                         int32_t *input_permutation, int32_t *output_permutation, int32_t *diag,
+                         void *workspace, size_t workspace_bytes, moe_stream_t stream);
+
+/*
+ * Dispatch (sglang PR #19058, "Changes", item 2 shuffle_rows: a
+ * dtype-agnostic row gather with 128-bit vector accesses):
+ *
+ *   out[p, :] = x[input_permutation[p] / k, :]   for every p with
+ *                                                 input_permutation[p] >= 0.
+ *
+ *   x       [T, H]   element type `dtype` (F32, F16 or BF16); H * sizeof
+ *                    must be a multiple of 16 bytes, x and out 16-byte
+ *                    aligned.
+ *   out     [T*k, H] same type; rows that no valid slot maps to are not
+ *                    written.
+ *   input_permutation / output_permutation  [T*k] int32 as produced by
+ *                    moe_prepare.  At least one must be non-NULL.  When
+ *                    output_permutation is given the kernel walks tokens and
+ *                    reads every x row once, writing it to its k rows
+ *                    (output_permutation must then be the inverse of the
+ *                    permutation that defines the result); otherwise it
+ *                    walks the dispatched rows and gathers through
+ *                    input_permutation.
+ */
+moe_status_t moe_dispatch_rows(const void *x, moe_dtype_t dtype, int64_t num_tokens,
+                               int64_t hidden, int32_t top_k, const int32_t *input_permutation,
+                               const int32_t *output_permutation, void *out, moe_stream_t stream);
+
+/*
+ * Dispatch with FP8 E4M3 1x128 block-scale quantisation (TensorRT-LLM PR
+ * #9592, FP8 block-scale MoE path, "run_moe_fp8_block_scales"; the optional
+ * FP8 block-scale offsets of sglang PR #19058 place the scales).  For every
+ * valid slot i = t*k + j with p = output_permutation[i] and e = topk_ids[i],
+ * and every 128-column block b:
+ *
+ *   amax = max |x[t, 128b .. 128b+127]|      (in fp32)
+ *   s    = amax / 448                         (fp32, round to nearest)
+ *   out_q[p, c] = e4m3_rn_satfinite(x[t, c] / s)   (fp32 division)
+ *   out_scales[blockscale_offsets[e] + p - expert_offsets[e], b] = s
+ *
+ * A block with amax = 0 gets s = 0 and zero bytes.  Rows of out_q and
+ * scale rows that no valid slot maps to (including the padding rows of each
+ * expert's scale segment) are not written.
+ *
+ *   x          [T, H] BF16 or F16, H a multiple of 128, 16-byte aligned.
+ *   topk_ids   [T, k] int32; output_permutation [T*k] int32;
+ *   expert_offsets / blockscale_offsets [E+1] int32 (from moe_prepare).
+ *   out_q      [T*k, H] uint8 (E4M3 bytes); out_scales [rows, H/128] fp32
+ *              with rows >= blockscale_offsets[E].
+ */
+moe_status_t moe_dispatch_rows_fp8(const void *x, moe_dtype_t x_dtype, int64_t num_tokens,
+                                   int64_t hidden, int32_t top_k, int32_t num_experts,
+                                   const int32_t *topk_ids, const int32_t *output_permutation,
+                                   const int32_t *expert_offsets,
+                                   const int32_t *blockscale_offsets, uint8_t *out_q,
+                                   float *out_scales, moe_stream_t stream);
+
+/*
+ * Combine (sglang PR #19058, "Changes", item 3 apply_shuffle_mul_sum:
+ * gather + scale + reduce, fp32 accumulation, fp16 / bf16 / fp32):
+ *
+ *   out[t, h] = round_out( sum_{j=0}^{k-1} weights[t, j] *
+ *                          y[output_permutation[t*k + j], h] )
+ *
+ * The sum runs over j in ascending order in fp32, each product and each sum
+ * rounded separately (no fused multiply-add); the result is rounded once to
+ * `out_dtype` (round to nearest even).  Slots with output_permutation = -1
+ * contribute nothing.
+ *
+ *   y        [T*k, H] F32, F16 or BF16 (expert outputs in dispatched order).
+ *   weights  [T, k]   fp32 router weights.
+ *   out      [T, H]   F32, F16 or BF16.
+ *   H * sizeof(y element) and H * sizeof(out element) must be multiples of
+ *   16 bytes; y and out 16-byte aligned.
+ */
+moe_status_t moe_combine(const void *y, moe_dtype_t y_dtype, int64_t num_tokens, int64_t hidden,
+                         int32_t top_k, const int32_t *output_permutation, const float *weights,
+                         void *out, moe_dtype_t out_dtype, moe_stream_t stream);
+
+/* Largest T*k that moe_prepare_dispatch accepts. */
+#define MOE_FUSED_MAX_SLOTS 4096
+
+/*
+ * Tiny-batch path: moe_prepare followed by moe_dispatch_rows in ONE kernel
+ * launch, for T*k <= MOE_FUSED_MAX_SLOTS, where launch latency dominates.
+ * Every block recomputes the routing metadata of the whole (small) batch in
+ * shared memory, block 0 writes the metadata outputs, and all blocks copy
+ * their share of rows.  Arguments and results are exactly those of the two
+ * calls (no workspace is needed); `diag` may be NULL.
+ */
+moe_status_t moe_prepare_dispatch(const int32_t *topk_ids, int64_t num_tokens, int32_t top_k,
+                                  int32_t num_experts, int32_t *expert_counts,
+                                  int32_t *expert_offsets, int32_t *blockscale_offsets,
+                                  int32_t blockscale_align, int32_t *input_permutation,
+                                  int32_t *output_permutation, int32_t *diag, const void *x,
+                                  moe_dtype_t dtype, int64_t hidden, void *out,
+                                  moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */
