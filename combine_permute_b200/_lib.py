@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(PKG, "libmoe.so")
 
 # moe_status_t / moe_dtype_t values (include/moe.h)
 MOE_OK = 0
+MOE_ERR_CUDA = 4
 MOE_F32, MOE_F16, MOE_BF16, MOE_FP8_E4M3 = 0, 1, 2, 3
 MAX_EXPERTS = 1024
 FUSED_MAX_SLOTS = 4096
@@ -23,6 +24,7 @@ FUSED_MAX_SLOTS = 4096
 EXPORTED = (
     "moe_status_string",
     "moe_version",
+    "moe_last_cuda_error",
     "moe_prepare_workspace_bytes",
     "moe_prepare",
     "moe_dispatch_rows",
@@ -39,6 +41,7 @@ _int = ctypes.c_int
 _SIGNATURES = {
     "moe_status_string": (ctypes.c_char_p, [_int]),
     "moe_version": (_i32, []),
+    "moe_last_cuda_error": (ctypes.c_char_p, []),
     "moe_prepare_workspace_bytes": (ctypes.c_size_t, [_i64, _i32, _i32]),
     "moe_prepare": (_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp,
                            ctypes.c_size_t, _vp]),
@@ -58,7 +61,10 @@ class MoeError(RuntimeError):
 
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn}: {status_string(status)}")
+        msg = f"{fn}: {status_string(status)}"
+        if status == MOE_ERR_CUDA:
+            msg += f" ({load().moe_last_cuda_error().decode()})"
+        super().__init__(msg)
 
 
 def load():

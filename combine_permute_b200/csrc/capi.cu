@@ -2,8 +2,9 @@
 // launchers in prepare.cu / dispatch.cu / combine.cu.  Contracts are stated
 // in include/moe.h.  No entry point allocates memory or synchronises.
 #include <cuda_runtime.h>
+#include <stdio.h>
 
-#include "../../include/moe.h"
+#include "moe.h"
 #include "kernels.h"
 
 namespace {
@@ -14,7 +15,17 @@ inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
 inline bool io_dtype(moe_dtype_t d) { return d == MOE_F32 || d == MOE_F16 || d == MOE_BF16; }
 
-inline moe_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+// The CUDA error behind the calling thread's last MOE_ERR_CUDA.
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+thread_local char t_last_error_text[256] = "no CUDA error";
+
+inline moe_status_t from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return MOE_OK;
+    t_last_cuda_error = e;
+    snprintf(t_last_error_text, sizeof t_last_error_text, "%s: %s", cudaGetErrorName(e),
+             cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+}
 
 inline moe::DType dt(moe_dtype_t d) { return static_cast<moe::DType>(static_cast<int>(d)); }
 
@@ -42,6 +53,8 @@ const char *moe_status_string(moe_status_t s) {
 
 int32_t moe_version(void) { return 10000; }
 
+const char *moe_last_cuda_error(void) { return t_last_error_text; }
+
 size_t moe_prepare_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t num_experts) {
     if (num_tokens < 0 || top_k < 1 || num_experts < 1) return 0;
     return moe::prepare_workspace_bytes(num_tokens * (int64_t)top_k, num_experts);
@@ -56,11 +69,11 @@ moe_status_t moe_prepare(const int32_t *topk_ids, int64_t num_tokens, int32_t to
     if (st != MOE_OK) return st;
     if (num_experts < 1) return MOE_ERR_INVALID_ARG;
     if (num_experts > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
-    if (!expert_counts || !expert_offsets || !input_permutation || !output_permutation)
-        return MOE_ERR_INVALID_ARG;
-    if (num_tokens > 0 && !topk_ids) return MOE_ERR_INVALID_ARG;
-    if (blockscale_offsets && blockscale_align < 1) return MOE_ERR_INVALID_ARG;
     const int64_t S = num_tokens * (int64_t)top_k;
+    if (!expert_counts || !expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (S > 0 && (!topk_ids || !input_permutation || !output_permutation))
+        return MOE_ERR_INVALID_ARG;
+    if (blockscale_offsets && blockscale_align < 1) return MOE_ERR_INVALID_ARG;
     const size_t need = moe::prepare_workspace_bytes(S, num_experts);
     if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
         return MOE_ERR_WORKSPACE;
@@ -144,10 +157,10 @@ moe_status_t moe_prepare_dispatch(const int32_t *topk_ids, int64_t num_tokens, i
     if (S > moe::kFusedMaxSlots) return MOE_ERR_UNSUPPORTED;
     const int64_t row_bytes = hidden * moe::dtype_bytes(dt(dtype));
     if (row_bytes % 16 != 0) return MOE_ERR_INVALID_ARG;
-    if (!expert_counts || !expert_offsets || !input_permutation || !output_permutation)
-        return MOE_ERR_INVALID_ARG;
+    if (!expert_counts || !expert_offsets) return MOE_ERR_INVALID_ARG;
     if (blockscale_offsets && blockscale_align < 1) return MOE_ERR_INVALID_ARG;
-    if (num_tokens > 0 && (!topk_ids || !x || !out)) return MOE_ERR_INVALID_ARG;
+    if (S > 0 && (!topk_ids || !x || !out || !input_permutation || !output_permutation))
+        return MOE_ERR_INVALID_ARG;
     if (num_tokens > 0 && (!aligned16(x) || !aligned16(out))) return MOE_ERR_INVALID_ARG;
     return from_cuda(moe::run_prepare_dispatch(
         topk_ids, num_tokens, top_k, num_experts, blockscale_offsets ? blockscale_align : 1,

@@ -20,34 +20,96 @@ namespace {
 constexpr int kCopyThreads = 128;
 constexpr int kCopyUnroll = 8;  // 16-byte vectors in flight per thread
 
-__global__ void __launch_bounds__(kCopyThreads)
-    dispatch_scatter_kernel(const uint4 *__restrict__ x, int64_t T, int64_t nvec, int k,
-                            const int32_t *__restrict__ out_perm, uint4 *__restrict__ out) {
+// ---------------------------------------------------------------------------
+// Scatter-form dispatch on the TMA engine.  One warp per block drives a ring
+// of kBulkStages shared-memory stages: lane 0 bulk-loads a row chunk of x
+// (cp.async.bulk global -> shared, completing on an mbarrier), then lane j
+// bulk-stores the staged chunk to dispatched row output_permutation[t*k+j]
+// (cp.async.bulk shared -> global).  A stage is refilled once the stores of
+// its previous chunk have finished reading it (bulk async-group wait).  The
+// row is read from HBM once and written k times with one instruction per
+// copy, so the load/store unit queues never throttle.
+// ---------------------------------------------------------------------------
+constexpr int kBulkStages = 4;
+constexpr uint32_t kBulkChunk = 16384;      // bytes per stage (row chunk)
+constexpr uint32_t kMaxPolls = 1u << 24;    // bounded mbarrier wait (each poll suspends briefly)
+
+__device__ unsigned g_dispatch_error;  // set when a bounded wait gave up
+
+__global__ void __launch_bounds__(32)
+    dispatch_bulk_kernel(const char *__restrict__ x, int64_t T, int64_t row_bytes, int k,
+                         const int32_t *__restrict__ out_perm, char *__restrict__ out) {
+    extern __shared__ __align__(128) unsigned char stage[];  // kBulkStages * kBulkChunk
+    __shared__ __align__(8) uint64_t bar[kBulkStages];
+    const int lane = threadIdx.x;
+    const int64_t nch = (row_bytes + kBulkChunk - 1) / kBulkChunk;
+    const int64_t units = T * nch;
+    const int64_t S = T * k;
+    const int64_t mine =
+        units > (int64_t)blockIdx.x ? (units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    if (lane == 0) {
+        for (int s = 0; s < kBulkStages; ++s) mbar_init(&bar[s], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
     pdl_wait();
     pdl_launch_dependents();
-    const int64_t S = T * k;
-    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        const uint4 *src = x + t * nvec;
-        const int32_t *dst_rows = out_perm + t * k;
-        for (int64_t c0 = threadIdx.x; c0 < nvec; c0 += kCopyThreads * kCopyUnroll) {
-            uint4 v[kCopyUnroll];
+
+    auto load = [&](int64_t n) {  // lane 0: chunk n of this block into stage n % kBulkStages
+        const int64_t u = blockIdx.x + n * (int64_t)gridDim.x;
+        const int64_t t = u / nch, off = (u - t * nch) * kBulkChunk;
+        const uint32_t bytes = (uint32_t)min((int64_t)kBulkChunk, row_bytes - off);
+        const int s = (int)(n % kBulkStages);
+        mbar_expect_tx(&bar[s], bytes);
+        bulk_g2s(stage + (size_t)s * kBulkChunk, x + t * row_bytes + off, bytes, &bar[s]);
+    };
+    int64_t issued = 0;
+    if (lane == 0)
+        for (; issued < kBulkStages && issued < mine; ++issued) load(issued);
+    issued = __shfl_sync(0xffffffffu, issued, 0);
+
+    bool failed = false;
+    int64_t n = 0;
+    for (; n < mine; ++n) {
+        const int64_t u = blockIdx.x + n * (int64_t)gridDim.x;
+        const int64_t t = u / nch, off = (u - t * nch) * kBulkChunk;
+        const uint32_t bytes = (uint32_t)min((int64_t)kBulkChunk, row_bytes - off);
+        const int s = (int)(n % kBulkStages);
+        int p[2];
 #pragma unroll
-            for (int u = 0; u < kCopyUnroll; ++u) {
-                const int64_t c = c0 + u * kCopyThreads;
-                if (c < nvec) v[u] = ld_stream_v4(src + c);
-            }
-            for (int j = 0; j < k; ++j) {
-                const int p = __ldg(dst_rows + j);
-                if (p < 0 || p >= S) continue;  // invalid slot (or a corrupt entry)
-                uint4 *dst = out + (int64_t)p * nvec;
+        for (int h = 0; h < 2; ++h) {
+            const int j = lane + 32 * h;
+            p[h] = j < k ? __ldg(out_perm + t * k + j) : -1;
+        }
+        const bool ok = mbar_wait(&bar[s], (uint32_t)((n / kBulkStages) & 1), kMaxPolls);
+        if (!__all_sync(0xffffffffu, ok)) {
+            failed = true;
+            break;
+        }
+        const unsigned char *src = stage + (size_t)s * kBulkChunk;
 #pragma unroll
-                for (int u = 0; u < kCopyUnroll; ++u) {
-                    const int64_t c = c0 + u * kCopyThreads;
-                    if (c < nvec) st_v4(dst + c, v[u]);
-                }
-            }
+        for (int h = 0; h < 2; ++h)
+            if (p[h] >= 0 && p[h] < S) bulk_s2g(out + (int64_t)p[h] * row_bytes + off, src, bytes);
+        for (int j = lane + 64; j < k; j += 32) {  // top-k above 64
+            const int pj = __ldg(out_perm + t * k + j);
+            if (pj >= 0 && pj < S) bulk_s2g(out + (int64_t)pj * row_bytes + off, src, bytes);
+        }
+        bulk_commit();
+        if (n >= 1) {
+            bulk_wait_read<1>();  // this lane's stores of chunk n-1 have read their stage
+            __syncwarp();
+            if (lane == 0 && issued < mine) load(issued);
+            issued = __shfl_sync(0xffffffffu, issued < mine ? issued + 1 : issued, 0);
         }
     }
+    if (failed) {
+        if (lane == 0) atomicExch(&g_dispatch_error, 1u);
+        // let every load still in flight land before the block releases its
+        // shared memory (again bounded)
+        for (int64_t m = n; m < issued; ++m)
+            mbar_wait(&bar[m % kBulkStages], (uint32_t)((m / kBulkStages) & 1), kMaxPolls);
+    }
+    bulk_wait_all();
 }
 
 __global__ void __launch_bounds__(kCopyThreads)
@@ -157,10 +219,11 @@ __global__ void __launch_bounds__(kFp8Threads)
 
 cudaError_t run_dispatch_scatter(const void *x, int64_t T, int64_t row_bytes, int k,
                                  const int32_t *out_perm, void *out, cudaStream_t stream) {
-    const int64_t nvec = row_bytes / 16;
-    const int64_t grid = persistent_grid(dispatch_scatter_kernel, kCopyThreads, 0, T);
-    return launch(dispatch_scatter_kernel, grid, kCopyThreads, 0, stream, (const uint4 *)x, T,
-                  nvec, k, out_perm, (uint4 *)out);
+    const size_t smem = (size_t)kBulkStages * kBulkChunk;
+    const int64_t units = T * ((row_bytes + kBulkChunk - 1) / kBulkChunk);
+    const int64_t grid = persistent_grid(dispatch_bulk_kernel, 32, smem, units);
+    return launch(dispatch_bulk_kernel, grid, 32, smem, stream, (const char *)x, T, row_bytes, k,
+                  out_perm, (char *)out);
 }
 
 cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int k,

@@ -22,9 +22,12 @@ constexpr int kWarpChunk = 32 * kPrepRounds;       // slots per warp per tile
 constexpr int kPrepTile = kPrepThreads * kPrepRounds;  // slots per tile
 constexpr int kSingleBlockSlots = kPrepTile;
 constexpr int kMaxExperts = 1024;
+// Up to this many slots the sort runs in one thread-block cluster.
+constexpr int64_t kClusterMaxSlots = 1 << 20;
 constexpr int kFusedMaxSlots = 4096;
 
 size_t prepare_workspace_bytes(int64_t S, int E);
+bool prepare_uses_cluster(int64_t S, int E);
 
 cudaError_t run_prepare(const int32_t *ids, int64_t S, int E, int A, int32_t *counts,
                         int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,

@@ -31,21 +31,37 @@ inline int sm_count() {
     return n;
 }
 
+// Raises `kernel`'s dynamic shared-memory limit on the current device to at
+// least `smem` (needed above the 48 KB default).  The limit is per kernel, so
+// it is only ever raised: lowering it for a smaller launch would make a later
+// larger one invalid.
+template <typename Kernel>
+cudaError_t ensure_smem(Kernel kernel, size_t smem) {
+    if (smem <= 48 * 1024) return cudaSuccess;
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, size_t> limit;
+    const auto key = std::make_pair((const void *)kernel, current_device());
+    std::lock_guard<std::mutex> g(mu);
+    auto it = limit.find(key);
+    if (it != limit.end() && it->second >= smem) return cudaSuccess;
+    cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) limit[key] = smem;
+    return e;
+}
+
 // Resident blocks per SM of `kernel` at this block size and dynamic shared
-// memory, memoised per (kernel, block size, smem, device).  Also raises the
-// kernel's dynamic shared-memory limit when the request is above the 48 KB
-// default.
+// memory, memoised per (kernel, block size, smem, device).
 template <typename Kernel>
 int blocks_per_sm(Kernel kernel, int threads, size_t smem) {
     static std::mutex mu;
     static std::map<std::tuple<const void *, int, size_t, int>, int> cache;
     const int dev = current_device();
     const auto key = std::make_tuple((const void *)kernel, threads, smem, dev);
+    ensure_smem(kernel, smem);
     std::lock_guard<std::mutex> g(mu);
     auto it = cache.find(key);
     if (it != cache.end()) return it->second;
-    if (smem > 48 * 1024)
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int n = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess ||
         n <= 0) {
@@ -68,7 +84,8 @@ int64_t persistent_grid(Kernel kernel, int threads, size_t smem, int64_t units) 
 template <typename... KArgs, typename... Args>
 cudaError_t launch(void (*kernel)(KArgs...), int64_t grid, int threads, size_t smem,
                    cudaStream_t stream, Args &&...args) {
-    if (smem > 48 * 1024) blocks_per_sm(kernel, threads, smem);  // sets the smem limit once
+    cudaError_t se = ensure_smem(kernel, smem);
+    if (se != cudaSuccess) return se;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
     cfg.blockDim = dim3((unsigned)threads, 1, 1);

@@ -3,7 +3,12 @@
 // per expert, prefix-sum expert offsets, optional FP8 block-scale offsets,
 // input / output permutations).
 //
-// Large problems run as tiles of kPrepTile slots in two kernels:
+// Three paths by problem size:
+//  * up to kSingleBlockSlots slots: one block (prep_single_kernel);
+//  * up to kClusterMaxSlots: one thread-block cluster that exchanges its
+//    blocks' histograms through distributed shared memory
+//    (prep_cluster_kernel, described where it is defined);
+//  * above that, tiles of kPrepTile slots in two kernels:
 //   prep_count_kernel    per-tile shared-memory histogram (warp-aggregated
 //                        with __match_any_sync), then a decoupled look-back
 //                        across tiles, one column per expert (plus one for
@@ -21,8 +26,9 @@
 // diag[1] instead of hanging.  The ticket counter wraps to zero and the
 // scatter kernel clears the look-back words, leaving the workspace zeroed.
 //
-// Small problems (<= kSingleBlockSlots slots) run in one block and need no
-// workspace.
+// Only the tiled path uses the workspace.
+#include <cooperative_groups.h>
+
 #include "kernels.h"
 #include "launch.h"
 #include "moe_device.cuh"
@@ -300,6 +306,7 @@ __global__ void __launch_bounds__(kPrepThreads)
 
     for (int e = tid; e < E; e += nt) {
         int run = __ldg(offsets + e) + ws.prefix[(size_t)tile * C + e];
+        ws.prefix[(size_t)tile * C + e] = 0;  // the workspace is all-zero between calls
         for (int w = 0; w < kPrepWarps; ++w) {
             const int c = wcnt[w * E + e];
             wcnt[w * E + e] = run;
@@ -328,12 +335,229 @@ __global__ void __launch_bounds__(kPrepThreads)
     const int64_t hi = base + kPrepTile < S ? base + kPrepTile : S;
     for (int64_t p = lo + tid; p < hi; p += nt) in_perm[p] = -1;
 
-    // leave the workspace zeroed for the next call
+    // leave the workspace zeroed for the next call (its layout depends on the
+    // problem size, so every byte this call used must return to zero)
     for (int c = tid; c < C; c += nt) ws.state[(size_t)tile * C + c] = 0ull;
+    if (tid == 0) ws.prefix[(size_t)tile * C + E] = 0;
     if (tile == 0 && tid == 0) {
         if (diag) diag[1] = *ws.timeout ? 1 : 0;
         *ws.timeout = 0u;
     }
+}
+
+// ---------------------------------------------------------------------------
+// Mid-size batches: the whole sort in ONE thread-block cluster (up to 16
+// blocks, one per SM).  Every warp owns a contiguous run of slots.
+//   pass 1  each warp counts its run per expert (warp-private shared-memory
+//           row, ballot-based match); the block folds its warps into a
+//           per-expert histogram.
+//   cluster barrier; every block reads all blocks' histograms through
+//           distributed shared memory: totals and the prefix of earlier
+//           blocks, then a block-wide scan gives the expert offsets.
+//   pass 2  each warp re-reads its run (now in L2) and ranks every slot:
+//           offset + earlier blocks + earlier warps + earlier lanes.
+// One launch, no global workspace, and the only waits are hardware cluster
+// barriers.
+// ---------------------------------------------------------------------------
+constexpr int kClusterThreads = 1024;
+constexpr int kClusterWarps = kClusterThreads / 32;
+constexpr int kClusterBatch = 8;  // rounds of 32 slots whose loads are in flight together
+
+// Lanes holding the same key (keys < 2^nbits): a match built from nbits
+// ballots.
+__device__ __forceinline__ unsigned match_by_ballot(unsigned key, int nbits) {
+    unsigned m = 0xffffffffu;
+    for (int b = 0; b < nbits; ++b) {
+        const unsigned bit = (key >> b) & 1u;
+        const unsigned vote = __ballot_sync(0xffffffffu, bit);
+        m &= bit ? vote : ~vote;
+    }
+    return m;
+}
+
+// Threads per expert when folding the per-warp counts: a power of two that
+// divides the warp count and keeps every thread busy for small E.
+__device__ __forceinline__ int fold_parts(int E) {
+    int parts = 1;
+    while (parts < kClusterWarps && parts * 2 * E <= kClusterThreads) parts *= 2;
+    return parts;
+}
+
+__global__ void __launch_bounds__(kClusterThreads, 1)
+    prep_cluster_kernel(const int32_t *__restrict__ ids, int64_t S, int E, int A, int nbits,
+                        int64_t wch, int32_t *counts, int32_t *offsets, int32_t *bso,
+                        int32_t *in_perm, int32_t *out_perm, int32_t *diag) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int nc = (int)cluster.num_blocks();
+    const int c = (int)cluster.block_rank();
+    extern __shared__ int smem[];
+    __shared__ int warp_tmp[33];
+    __shared__ int s_invalid;
+    int *wcnt = smem;                          // [kClusterWarps][E]
+    int *hist = wcnt + kClusterWarps * E;      // [E+1]: per expert, then invalid ids
+    int *tot = hist + (E + 1);                 // [E+1]
+    int *pre = tot + (E + 1);                  // [E]
+    int *pad = pre + E;                        // [E]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const unsigned lt = lanemask_lt();
+    const unsigned key_invalid = (unsigned)E;
+
+    for (int x = tid; x < kClusterWarps * E; x += kClusterThreads) wcnt[x] = 0;
+    if (tid == 0) s_invalid = 0;
+    pdl_wait();
+    pdl_launch_dependents();
+    __syncthreads();
+
+    const int64_t beg = ((int64_t)c * kClusterWarps + warp) * wch;
+    const int64_t end = min(S, beg + wch);
+    int *row = wcnt + warp * E;
+
+    // pass 1: per-warp counts
+    int bad = 0;
+    for (int64_t r0 = beg; r0 < end; r0 += 32 * kClusterBatch) {
+        int key[kClusterBatch];
+#pragma unroll
+        for (int b = 0; b < kClusterBatch; ++b) {
+            const int64_t i = r0 + b * 32 + lane;
+            int k2 = -2;  // past the run
+            if (i < end) {
+                const int id = __ldg(ids + i);
+                k2 = (id >= 0 && id < E) ? id : -1;
+            }
+            key[b] = k2;
+        }
+#pragma unroll
+        for (int b = 0; b < kClusterBatch; ++b) {
+            if (r0 + b * 32 >= end) break;  // warp-uniform
+            const bool valid = key[b] >= 0;
+            bad += key[b] == -1;
+            const unsigned grp = match_by_ballot(valid ? (unsigned)key[b] : key_invalid, nbits);
+            if (valid && (grp & lt) == 0) row[key[b]] += __popc(grp);
+            __syncwarp();
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
+    if (lane == 0 && bad) atomicAdd(&s_invalid, bad);
+    __syncthreads();
+
+    // block histogram; per-warp counts become exclusive prefixes over warps.
+    // `parts` threads share one expert (consecutive lanes), each folding a
+    // contiguous group of warps, then combine with shuffles.
+    {
+        const int parts = fold_parts(E);
+        const int per = kClusterWarps / parts;
+        const int q = tid % parts;
+        const int stride = kClusterThreads / parts;
+        const int iters = (E + stride - 1) / stride;  // the same for every thread
+        for (int it = 0; it < iters; ++it) {
+            const int e = it * stride + tid / parts;
+            const bool live = e < E;
+            int sum = 0;
+            if (live)
+                for (int w = q * per; w < q * per + per; ++w) sum += wcnt[w * E + e];
+            int incl = sum;  // inclusive scan of the part sums within the expert's lanes
+            for (int o = 1; o < parts; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, incl, o, parts);
+                if (q >= o) incl += u;
+            }
+            if (live) {
+                int run = incl - sum;
+                for (int w = q * per; w < q * per + per; ++w) {
+                    const int v = wcnt[w * E + e];
+                    wcnt[w * E + e] = run;
+                    run += v;
+                }
+                if (q == parts - 1) hist[e] = run;
+            }
+        }
+    }
+    if (tid == 0) hist[E] = s_invalid;
+    cluster.sync();
+
+    // totals and the prefix of earlier blocks, read from every block's
+    // shared memory (all loads in flight together)
+    for (int e = tid; e <= E; e += kClusterThreads) {
+        int v[16];
+#pragma unroll
+        for (int b = 0; b < 16; ++b) v[b] = b < nc ? cluster.map_shared_rank(hist, b)[e] : 0;
+        int t = 0, p = 0;
+#pragma unroll
+        for (int b = 0; b < 16; ++b) {
+            t += v[b];
+            p += b < c ? v[b] : 0;
+        }
+        tot[e] = t;
+        if (e < E) {
+            pre[e] = p;
+            pad[e] = (t + A - 1) / A * A;
+        }
+    }
+    __syncthreads();
+    const int n_invalid = tot[E];
+    const int total = block_exclusive_scan(tot, E, warp_tmp);  // tot[e] = expert offset
+    int pad_total = 0;
+    if (bso) pad_total = block_exclusive_scan(pad, E, warp_tmp);
+    if (c == 0) {
+        for (int e = tid; e < E; e += kClusterThreads) {
+            counts[e] = (e + 1 < E ? tot[e + 1] : total) - tot[e];
+            offsets[e] = tot[e];
+            if (bso) bso[e] = pad[e];
+        }
+        if (tid == 0) {
+            offsets[E] = total;
+            if (bso) bso[E] = pad_total;
+            if (diag) {
+                diag[0] = n_invalid;
+                diag[1] = 0;
+            }
+        }
+    }
+    for (int x = tid; x < kClusterWarps * E; x += kClusterThreads) {
+        const int e = x % E;
+        wcnt[x] += tot[e] + pre[e];
+    }
+    __syncthreads();
+
+    // pass 2: ranks and both permutations
+    for (int64_t r0 = beg; r0 < end; r0 += 32 * kClusterBatch) {
+        int key[kClusterBatch];
+#pragma unroll
+        for (int b = 0; b < kClusterBatch; ++b) {
+            const int64_t i = r0 + b * 32 + lane;
+            int k2 = -2;
+            if (i < end) {
+                const int id = __ldg(ids + i);
+                k2 = (id >= 0 && id < E) ? id : -1;
+            }
+            key[b] = k2;
+        }
+#pragma unroll
+        for (int b = 0; b < kClusterBatch; ++b) {
+            if (r0 + b * 32 >= end) break;
+            const int64_t i = r0 + b * 32 + lane;
+            const bool valid = key[b] >= 0;
+            const unsigned grp = match_by_ballot(valid ? (unsigned)key[b] : key_invalid, nbits);
+            int p = -1;
+            if (valid) {
+                const int basev = row[key[b]];
+                p = basev + __popc(grp & lt);
+                __syncwarp(grp);
+                if ((grp & lt) == 0) row[key[b]] = basev + __popc(grp);
+            }
+            __syncwarp();
+            if (i < end) {
+                out_perm[i] = p;
+                if (p >= 0 && p < S) in_perm[p] = (int)i;
+            }
+        }
+    }
+    // input_permutation past the valid rows
+    for (int64_t p = total + (int64_t)c * kClusterThreads + tid; p < S;
+         p += (int64_t)nc * kClusterThreads)
+        in_perm[p] = -1;
+    cluster.sync();  // no block leaves while another may still read its histogram
 }
 
 // Tiny batches: every block recomputes the metadata in shared memory (the
@@ -375,12 +599,90 @@ size_t prepare_workspace_bytes(int64_t S, int E) {
     return 256 + align256((size_t)G * C * 8) + align256((size_t)G * C * 4);
 }
 
+namespace {
+
+// Largest cluster of prep_cluster_kernel blocks this device can co-schedule
+// (16 with the non-portable size, else 8), cached per device; 0 if none.
+int cluster_blocks(size_t smem) {
+    static std::mutex mu;
+    static std::map<std::pair<int, size_t>, int> cache;
+    const int dev = current_device();
+    std::lock_guard<std::mutex> g(mu);
+    auto key = std::make_pair(dev, smem);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    int best = 0;
+    ensure_smem(prep_cluster_kernel, smem);
+    cudaFuncSetAttribute(prep_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    for (int nc : {16, 8}) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(nc, 1, 1);
+        cfg.blockDim = dim3(kClusterThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = nc;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, prep_cluster_kernel, &cfg) == cudaSuccess && n > 0) {
+            best = nc;
+            break;
+        }
+        cudaGetLastError();
+    }
+    cache[key] = best;
+    return best;
+}
+
+size_t cluster_smem(int E) {
+    return (size_t)(kClusterWarps * E + 2 * (E + 1) + 2 * E) * sizeof(int);
+}
+
+}  // namespace
+
+bool prepare_uses_cluster(int64_t S, int E) {
+    return S > kSingleBlockSlots && S <= kClusterMaxSlots && cluster_blocks(cluster_smem(E)) > 0;
+}
+
 cudaError_t run_prepare(const int32_t *ids, int64_t S, int E, int A, int32_t *counts,
                         int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,
                         int32_t *diag, void *workspace, cudaStream_t stream) {
     if (S <= kSingleBlockSlots)
         return launch(prep_single_kernel, 1, kPrepThreads, single_block_smem(E), stream, ids, S,
                       E, A, counts, offsets, bso, in_perm, out_perm, diag);
+    if (S <= kClusterMaxSlots) {
+        const size_t smem = cluster_smem(E);
+        const int nc = cluster_blocks(smem);
+        if (nc > 0) {
+            const int64_t warps = (int64_t)nc * kClusterWarps;
+            const int64_t wch = ((S + warps - 1) / warps + 31) / 32 * 32;
+            int nbits = 1;
+            while ((1 << nbits) <= E) ++nbits;  // keys 0..E (E marks an invalid id)
+            cudaError_t se = ensure_smem(prep_cluster_kernel, smem);
+            if (se != cudaSuccess) return se;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(nc, 1, 1);
+            cfg.blockDim = dim3(kClusterThreads, 1, 1);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[2];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = nc;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            attr[1].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 2;
+            cudaError_t e = cudaLaunchKernelEx(&cfg, prep_cluster_kernel, ids, S, E, A, nbits, wch,
+                                               counts, offsets, bso, in_perm, out_perm, diag);
+            if (e != cudaSuccess) return e;
+            return cudaGetLastError();
+        }
+    }
     const int G = (int)((S + kPrepTile - 1) / kPrepTile);
     const size_t smem1 = (size_t)3 * (E + 1) * sizeof(int);
     cudaError_t e = launch(prep_count_kernel, G, kPrepThreads, smem1, stream, ids, S, E, A, G,

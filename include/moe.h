@@ -76,6 +76,11 @@ const char *moe_status_string(moe_status_t status);
 /* Library version as major*10000 + minor*100 + patch. */
 int32_t moe_version(void);
 
+/* Name and description of the CUDA error behind the calling thread's most
+ * recent MOE_ERR_CUDA ("no CUDA error" if there was none).  The string is
+ * thread-local and valid until the thread's next failing call. */
+const char *moe_last_cuda_error(void);
+
 /*
  * Bytes of scratch workspace moe_prepare needs for this problem size (0 when
  * the problem is small enough for the single-block path).  The workspace
@@ -119,10 +124,15 @@ size_t moe_prepare_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t nu
  *                                      (see above); may be NULL when that
  *                                      size is 0.
  *
+ * Batches of up to 4096 slots run in one block, up to 2^20 slots in one
+ * thread-block cluster, larger ones as tiles in two kernels (the only case
+ * that touches the workspace).
+ *
  * Dispatched order: by expert ascending, and within an expert by expanded
  * index ascending (token, then slot): a stable counting sort, so the result
  * is deterministic.  Ids outside [0, E) are not counted and get no row; the
- * call still succeeds (check diag[0]).  T = 0 writes zero counts/offsets.
+ * call still succeeds (check diag[0]).  T = 0 writes zero counts/offsets;
+ * topk_ids and the permutations may then be NULL.
  */
 moe_status_t moe_prepare(const int32_t *topk_ids, int64_t num_tokens, int32_t top_k,
                          int32_t num_experts, int32_t *expert_counts, int32_t *expert_offsets,

@@ -86,6 +86,9 @@ def test_prepare_validation(lib):
     assert _prepare(lib, offsets=None) == INVALID
     assert _prepare(lib, inp=None) == INVALID
     assert _prepare(lib, outp=None) == INVALID
+    # an empty batch needs neither ids nor permutations (torch gives NULL for
+    # empty tensors); it still launches, so only the argument check is tested
+    assert _prepare(lib, T=0, ids=None, inp=None, outp=None, E=0) == INVALID
     assert _prepare(lib, bso=P, A=0) == INVALID
     assert _prepare(lib, T=1 << 28, k=8) == UNSUPPORTED              # T*k = 2^31
     # above one tile the workspace is required, large enough and aligned

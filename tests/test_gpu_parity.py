@@ -66,6 +66,8 @@ def test_prepare_tiny_vs_oracle(trial):
     (513, 8, 256), (1024, 8, 7), (3001, 6, 64),          # two or more tiles, ragged tails
     (4095, 1, 1), (20000, 8, 1024), (9216, 8, 256),
     (40000, 3, 5), (70000, 8, 288),
+    (131072, 8, 1024),                                    # the largest single-cluster batches
+    (140000, 8, 64), (262144, 6, 256),                    # past 2^20 slots: the tiled path
 ])
 def test_prepare_sizes_vs_oracle(T, k, E):
     rng = np.random.default_rng(T * 31 + k * 7 + E)
@@ -94,8 +96,9 @@ def test_prepare_full_workloads(name):
     _check_prepare(ids, w.E, A=w.block_align if w.block_align > 1 else 128)
 
 
-def test_prepare_deterministic_and_workspace_left_zero():
-    w = CONFIGS["zipf_fp16_t131072_h2048_e64_k6"]
+@pytest.mark.parametrize("T", [131072, 200000])   # single-cluster path; tiled path (> 2^20 slots)
+def test_prepare_deterministic_and_workspace_left_zero(T):
+    w = CONFIGS["zipf_fp16_t131072_h2048_e64_k6"].scaled(T)
     ids_np, _, _, _ = make_workload(w, with_x=False, with_y=False)
     ids = torch.from_numpy(ids_np).to(DEV)
     nbytes = moe.moe_prepare_workspace_bytes(w.T, w.k, w.E)
@@ -147,9 +150,10 @@ def test_dispatch_full_workloads_sampled(name):
     rows = np.unique(np.concatenate([rng.integers(0, w.S, 2000), [0, w.S - 1]]))
     ref = oracle.dispatch(bits(x), w.k, ref_meta["input_perm"][rows])
     np.testing.assert_array_equal(bits(out[torch.from_numpy(rows).to(DEV)]), ref)
-    # any-size property: every token row appears exactly k times (row sums as a fingerprint)
-    fp_x = x.float().sum(dim=1).double()
-    fp_out = out.float().sum(dim=1).double()
+    # any-size property: every dispatched row equals its token row (exact
+    # integer fingerprint of the raw bits)
+    fp_x = x.view(torch.int16).to(torch.int32).sum(dim=1)
+    fp_out = out.view(torch.int16).to(torch.int32).sum(dim=1)
     counts = torch.bincount(meta.input_permutation.long() // w.k, minlength=w.T)
     assert bool((counts == w.k).all())
     assert torch.equal(fp_out, fp_x[meta.input_permutation.long() // w.k])
