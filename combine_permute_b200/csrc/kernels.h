@@ -14,20 +14,16 @@ inline int dtype_bytes(DType d) {
 }
 
 // Prepare: a problem with at most kSingleBlockSlots slots runs as one block;
-// larger ones as tiles of kPrepTile slots in two kernels.
-constexpr int kPrepThreads = 512;
-constexpr int kPrepWarps = kPrepThreads / 32;
-constexpr int kPrepRounds = 8;
-constexpr int kWarpChunk = 32 * kPrepRounds;       // slots per warp per tile
-constexpr int kPrepTile = kPrepThreads * kPrepRounds;  // slots per tile
-constexpr int kSingleBlockSlots = kPrepTile;
+// larger ones as tiles of kTileSlots slots over the whole GPU.
+constexpr int kSingleBlockSlots = 4096;
+constexpr int kTileThreads = 256;
+constexpr int kTileWarps = kTileThreads / 32;
+constexpr int kTileRounds = 8;  // rounds of 32 slots per warp
+constexpr int kTileSlots = kTileThreads * kTileRounds;
 constexpr int kMaxExperts = 1024;
-// Up to this many slots the sort runs in one thread-block cluster.
-constexpr int64_t kClusterMaxSlots = 1 << 20;
 constexpr int kFusedMaxSlots = 4096;
 
 size_t prepare_workspace_bytes(int64_t S, int E);
-bool prepare_uses_cluster(int64_t S, int E);
 
 cudaError_t run_prepare(const int32_t *ids, int64_t S, int E, int A, int32_t *counts,
                         int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,

@@ -125,6 +125,60 @@ __device__ __forceinline__ int block_exclusive_scan(int *data, int n, int *warp_
     return total;
 }
 
+// Two exclusive scans in one pass over n <= 32 * blockDim.x counts held in
+// shared memory: a[] in place, and pad[] <- exclusive scan of a[] each
+// rounded up to a multiple of A.  Returns the total of a; *pad_total gets
+// the total of the rounded counts.  Needs blockDim.x a multiple of 32 and
+// at most 1024; warp_tmp needs 66 ints.  All threads must call it.
+__device__ __forceinline__ int block_exclusive_scan2(int *a, int *pad, int n, int A, int *warp_tmp,
+                                                     int *pad_total) {
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+    const int nw = nt >> 5;
+    const int per = (n + nt - 1) / nt;
+    const int beg = min(n, tid * per), end = min(n, beg + per);
+    int la = 0, lp = 0;
+    for (int i = beg; i < end; ++i) {
+        la += a[i];
+        lp += (a[i] + A - 1) / A * A;
+    }
+    int va = la, vp = lp;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int ua = __shfl_up_sync(0xffffffffu, va, o);
+        const int up = __shfl_up_sync(0xffffffffu, vp, o);
+        if (lane >= o) {
+            va += ua;
+            vp += up;
+        }
+    }
+    if (lane == 31) {
+        warp_tmp[warp] = va;
+        warp_tmp[33 + warp] = vp;
+    }
+    __syncthreads();
+    int ba = 0, bp = 0, ta = 0, tp = 0;
+    for (int w = 0; w < nw; ++w) {  // warp totals: a short broadcast read
+        const int xa = warp_tmp[w], xp = warp_tmp[33 + w];
+        if (w < warp) {
+            ba += xa;
+            bp += xp;
+        }
+        ta += xa;
+        tp += xp;
+    }
+    int ra = va - la + ba, rp = vp - lp + bp;
+    for (int i = beg; i < end; ++i) {
+        const int c = a[i];
+        a[i] = ra;
+        pad[i] = rp;
+        ra += c;
+        rp += (c + A - 1) / A * A;
+    }
+    __syncthreads();
+    *pad_total = tp;
+    return ta;
+}
+
 }  // namespace moe
 
 namespace moe {

@@ -82,8 +82,8 @@ int32_t moe_version(void);
 const char *moe_last_cuda_error(void);
 
 /*
- * Bytes of scratch workspace moe_prepare needs for this problem size (0 when
- * the problem is small enough for the single-block path).  The workspace
+ * Bytes of scratch workspace moe_prepare needs for this problem size: 0 up
+ * to 4096 slots (T*k), which run in one block without one.  The workspace
  * must be all-zero before its first use (e.g. one cudaMemsetAsync); every
  * completed call leaves it all-zero again, so one workspace serves any
  * number of consecutive calls on one stream.  Calls that may run
@@ -124,9 +124,8 @@ size_t moe_prepare_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t nu
  *                                      (see above); may be NULL when that
  *                                      size is 0.
  *
- * Batches of up to 4096 slots run in one block, up to 2^20 slots in one
- * thread-block cluster, larger ones as tiles in two kernels (the only case
- * that touches the workspace).
+ * Batches of up to 4096 slots run in one block; larger ones as tiles over
+ * the whole GPU in two kernels (the only case that touches the workspace).
  *
  * Dispatched order: by expert ascending, and within an expert by expanded
  * index ascending (token, then slot): a stable counting sort, so the result

@@ -63,9 +63,9 @@ def test_status_strings_and_version(lib):
 
 def test_workspace_bytes(lib):
     assert lib.moe_prepare_workspace_bytes(32, 8, 256) == 0          # single-block path
-    assert lib.moe_prepare_workspace_bytes(512, 8, 256) == 0         # exactly one tile
-    a = lib.moe_prepare_workspace_bytes(513, 8, 256)
-    b = lib.moe_prepare_workspace_bytes(131072, 6, 64)
+    assert lib.moe_prepare_workspace_bytes(512, 8, 256) == 0         # 4096 slots: still one block
+    a = lib.moe_prepare_workspace_bytes(513, 8, 256)                 # tiled path
+    b = lib.moe_prepare_workspace_bytes(1 << 20, 6, 256)
     assert a > 0 and b > a and a % 256 == 0 and b % 256 == 0
     assert lib.moe_prepare_workspace_bytes(-1, 8, 256) == 0
 
@@ -92,10 +92,11 @@ def test_prepare_validation(lib):
     assert _prepare(lib, bso=P, A=0) == INVALID
     assert _prepare(lib, T=1 << 28, k=8) == UNSUPPORTED              # T*k = 2^31
     # above one tile the workspace is required, large enough and aligned
-    need = lib.moe_prepare_workspace_bytes(1000, 8, 8)
-    assert _prepare(lib, T=1000, k=8, ws=None) == WORKSPACE
-    assert _prepare(lib, T=1000, k=8, ws=P, ws_bytes=need - 1) == WORKSPACE
-    assert _prepare(lib, T=1000, k=8, ws=P + 16, ws_bytes=need) == WORKSPACE
+    need = lib.moe_prepare_workspace_bytes(140000, 8, 8)
+    assert need > 0
+    assert _prepare(lib, T=140000, k=8, ws=None) == WORKSPACE
+    assert _prepare(lib, T=140000, k=8, ws=P, ws_bytes=need - 1) == WORKSPACE
+    assert _prepare(lib, T=140000, k=8, ws=P + 16, ws_bytes=need) == WORKSPACE
 
 
 def test_dispatch_validation(lib):

@@ -66,8 +66,7 @@ def test_prepare_tiny_vs_oracle(trial):
     (513, 8, 256), (1024, 8, 7), (3001, 6, 64),          # two or more tiles, ragged tails
     (4095, 1, 1), (20000, 8, 1024), (9216, 8, 256),
     (40000, 3, 5), (70000, 8, 288),
-    (131072, 8, 1024),                                    # the largest single-cluster batches
-    (140000, 8, 64), (262144, 6, 256),                    # past 2^20 slots: the tiled path
+    (131072, 8, 1024), (140000, 8, 64), (262144, 6, 256),
 ])
 def test_prepare_sizes_vs_oracle(T, k, E):
     rng = np.random.default_rng(T * 31 + k * 7 + E)
@@ -96,7 +95,7 @@ def test_prepare_full_workloads(name):
     _check_prepare(ids, w.E, A=w.block_align if w.block_align > 1 else 128)
 
 
-@pytest.mark.parametrize("T", [131072, 200000])   # single-cluster path; tiled path (> 2^20 slots)
+@pytest.mark.parametrize("T", [131072, 200000])
 def test_prepare_deterministic_and_workspace_left_zero(T):
     w = CONFIGS["zipf_fp16_t131072_h2048_e64_k6"].scaled(T)
     ids_np, _, _, _ = make_workload(w, with_x=False, with_y=False)
