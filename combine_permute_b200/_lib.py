@@ -31,6 +31,7 @@ EXPORTED = (
     "moe_dispatch_rows_fp8",
     "moe_combine",
     "moe_prepare_dispatch",
+    "moe_prepare_no_alloc",
 )
 
 _vp = ctypes.c_void_p
@@ -51,6 +52,8 @@ _SIGNATURES = {
     "moe_combine": (_int, [_vp, _int, _i64, _i64, _i32, _vp, _vp, _vp, _int, _vp]),
     "moe_prepare_dispatch": (_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp,
                                     _vp, _int, _i64, _vp, _vp]),
+    "moe_prepare_no_alloc": (_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp,
+                                    _vp]),
 }
 
 _lib = None

@@ -38,6 +38,11 @@ inline moe_status_t check_tk(int64_t T, int32_t k) {
 
 }  // namespace
 
+namespace moe {
+// Status of a CUDA result, recording the error text like every entry point.
+moe_status_t status_from_cuda(cudaError_t e) { return from_cuda(e); }
+}  // namespace moe
+
 extern "C" {
 
 const char *moe_status_string(moe_status_t s) {

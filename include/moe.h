@@ -215,6 +215,42 @@ moe_status_t moe_combine(const void *y, moe_dtype_t y_dtype, int64_t num_tokens,
                          int32_t top_k, const int32_t *output_permutation, const float *weights,
                          void *out, moe_dtype_t out_dtype, moe_stream_t stream);
 
+/* Size of the device array that moe_prepare_no_alloc uses as scratch. */
+#define MOE_PREPARE_NO_ALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+
+/*
+ * moe_prepare without a workspace argument, for callers that cannot
+ * allocate device memory: work being recorded into a CUDA graph (cudaMalloc
+ * may not run while a stream is captured), serving loops in which a
+ * cudaMalloc would synchronise the device and stall every other stream, and
+ * processes whose GPU memory is handed to a pool allocator up front.  This
+ * call has no counterpart in the paper.
+ *
+ * Arguments, results and errors are those of moe_prepare.  In place of a
+ * workspace the call uses one fixed device array of
+ * MOE_PREPARE_NO_ALLOC_SCRATCH_BYTES (4 MiB), which every GPU that loads the
+ * library holds until the process exits.  A problem that needs more scratch
+ * than that (moe_prepare_workspace_bytes() above 4 MiB: T*k beyond about 4.1
+ * million slots with 256 experts, about 1 million with 1024) is rejected
+ * with MOE_ERR_UNSUPPORTED before anything is launched.  The call allocates
+ * nothing: it clears the part of the array it needs with cudaMemsetAsync on
+ * `stream`, then launches the same kernels as moe_prepare.
+ *
+ * All calls on one device share the array and it keeps the last call's
+ * contents, so two calls whose work overlaps on the GPU (different streams
+ * with no ordering between them) race and produce wrong results: order them
+ * on one stream, or use moe_prepare with separate workspaces.  The first
+ * call on a device that needs the scratch (T*k above 4096) looks up the
+ * array's device address, once per device; make that first call before any
+ * stream capture begins.
+ */
+moe_status_t moe_prepare_no_alloc(const int32_t *topk_ids, int64_t num_tokens, int32_t top_k,
+                                  int32_t num_experts, int32_t *expert_counts,
+                                  int32_t *expert_offsets, int32_t *blockscale_offsets,
+                                  int32_t blockscale_align, int32_t *input_permutation,
+                                  int32_t *output_permutation, int32_t *diag,
+                                  moe_stream_t stream);
+
 /* Largest T*k that moe_prepare_dispatch accepts. */
 #define MOE_FUSED_MAX_SLOTS 4096
 
