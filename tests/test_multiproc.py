@@ -1,0 +1,84 @@
+"""Multi-process host logic of the benchmark, on CPU with gloo.
+
+The path has no exchange step: a run on N GPUs is N independent replicas,
+timed as the maximum over ranks, the value being the tokens of every rank
+over that time.  These tests run that bookkeeping with world size 2 over
+gloo, and the reference arm (the CPU oracle) under torchrun, where rank 0
+alone works and prints.
+"""
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    r = bench.Ranks("gloo", device=None, timeout_s=60)
+    r.barrier()
+    elapsed = 10.0 * (rank + 1)             # rank 1 is the slower one
+    worst = r.max_over_ranks(elapsed)
+    value = bench.whole_job_tokens_per_s(4096, 50, r.world, worst)
+    r.close()
+    with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+        json.dump({"rank": r.rank, "world": r.world, "worst": worst, "value": value}, f)
+
+
+def test_replicas_time_is_max_over_ranks_gloo(tmp_path):
+    world, port = 2, _free_port()
+    mp.start_processes(_worker, args=(world, port, str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    assert [x["rank"] for x in res] == [0, 1] and all(x["world"] == 2 for x in res)
+    assert all(x["worst"] == 20.0 for x in res)
+    # 2 ranks x 50 steps x 4096 tokens over the slower rank's 20 ms
+    assert res[0]["value"] == pytest.approx(2 * 50 * 4096 / 0.020)
+
+
+def _json_lines(text):
+    return [json.loads(l) for l in text.splitlines() if l.startswith("{")]
+
+
+@pytest.mark.slow
+def test_reference_arm_single_process():
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "2",
+                          "--warmup", "3", "--ref-budget", "2"], cwd=ROOT, capture_output=True,
+                         text=True, timeout=600)
+    assert out.returncode == 0, out.stderr
+    lines = _json_lines(out.stdout)
+    assert len(lines) == 1
+    d = lines[0]
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["config"]["workload"] == "uniform_t4096_h7168_e256_k8"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+@pytest.mark.slow
+def test_reference_arm_under_torchrun_prints_once():
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl",
+           "reference", "--gpus", "2", "--steps", "1", "--warmup", "3", "--ref-budget", "1",
+           "--workload", "tiny_t32_h4096_e256_k8"]
+    out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr
+    lines = _json_lines(out.stdout)
+    assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
