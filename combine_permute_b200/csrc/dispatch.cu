@@ -22,71 +22,73 @@ constexpr int kCopyUnroll = 8;  // 16-byte vectors in flight per thread
 
 // ---------------------------------------------------------------------------
 // Scatter-form dispatch on the TMA engine.  One warp per block drives a ring
-// of kBulkStages shared-memory stages: lane 0 bulk-loads a row chunk of x
+// of shared-memory stages: lane 0 bulk-loads a chunk of an x row
 // (cp.async.bulk global -> shared, completing on an mbarrier), then lane j
 // bulk-stores the staged chunk to dispatched row output_permutation[t*k+j]
 // (cp.async.bulk shared -> global).  A stage is refilled once the stores of
 // its previous chunk have finished reading it (bulk async-group wait).  The
 // row is read from HBM once and written k times with one instruction per
-// copy, so the load/store unit queues never throttle.
+// copy, so the load/store unit queues never throttle.  The host splits rows
+// into `nch` chunks so that the (token, chunk) units spread evenly over the
+// persistent grid.
 // ---------------------------------------------------------------------------
-constexpr int kBulkStages = 4;
-constexpr uint32_t kBulkChunk = 16384;      // bytes per stage (row chunk)
+constexpr int kBulkMaxStages = 16;
+constexpr uint32_t kBulkSmem = 64 * 1024;   // stage ring per block
 constexpr uint32_t kMaxPolls = 1u << 24;    // bounded mbarrier wait (each poll suspends briefly)
 
 __device__ unsigned g_dispatch_error;  // set when a bounded wait gave up
 
 __global__ void __launch_bounds__(32)
     dispatch_bulk_kernel(const char *__restrict__ x, int64_t T, int64_t row_bytes, int k,
-                         const int32_t *__restrict__ out_perm, char *__restrict__ out) {
-    extern __shared__ __align__(128) unsigned char stage[];  // kBulkStages * kBulkChunk
-    __shared__ __align__(8) uint64_t bar[kBulkStages];
+                         const int32_t *__restrict__ out_perm, char *__restrict__ out,
+                         int64_t nch, uint32_t chunk, int stages) {
+    extern __shared__ __align__(128) unsigned char stage[];  // stages * chunk
+    __shared__ __align__(8) uint64_t bar[kBulkMaxStages];
     const int lane = threadIdx.x;
-    const int64_t nch = (row_bytes + kBulkChunk - 1) / kBulkChunk;
     const int64_t units = T * nch;
     const int64_t S = T * k;
     const int64_t mine =
         units > (int64_t)blockIdx.x ? (units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     if (lane == 0) {
-        for (int s = 0; s < kBulkStages; ++s) mbar_init(&bar[s], 1);
+        for (int s = 0; s < stages; ++s) mbar_init(&bar[s], 1);
         fence_mbar_init();
     }
     __syncwarp();
     pdl_wait();
     pdl_launch_dependents();
 
-    auto load = [&](int64_t n) {  // lane 0: chunk n of this block into stage n % kBulkStages
+    auto load = [&](int64_t n) {  // lane 0: this block's unit n into stage n % stages
         const int64_t u = blockIdx.x + n * (int64_t)gridDim.x;
-        const int64_t t = u / nch, off = (u - t * nch) * kBulkChunk;
-        const uint32_t bytes = (uint32_t)min((int64_t)kBulkChunk, row_bytes - off);
-        const int s = (int)(n % kBulkStages);
+        const int64_t t = u / nch, off = (u - t * nch) * (int64_t)chunk;
+        const uint32_t bytes = (uint32_t)min((int64_t)chunk, row_bytes - off);
+        const int s = (int)(n % stages);
         mbar_expect_tx(&bar[s], bytes);
-        bulk_g2s(stage + (size_t)s * kBulkChunk, x + t * row_bytes + off, bytes, &bar[s]);
+        bulk_g2s(stage + (size_t)s * chunk, x + t * row_bytes + off, bytes, &bar[s]);
     };
     int64_t issued = 0;
     if (lane == 0)
-        for (; issued < kBulkStages && issued < mine; ++issued) load(issued);
+        for (; issued < stages && issued < mine; ++issued) load(issued);
     issued = __shfl_sync(0xffffffffu, issued, 0);
 
     bool failed = false;
     int64_t n = 0;
     for (; n < mine; ++n) {
         const int64_t u = blockIdx.x + n * (int64_t)gridDim.x;
-        const int64_t t = u / nch, off = (u - t * nch) * kBulkChunk;
-        const uint32_t bytes = (uint32_t)min((int64_t)kBulkChunk, row_bytes - off);
-        const int s = (int)(n % kBulkStages);
+        const int64_t t = u / nch, off = (u - t * nch) * (int64_t)chunk;
+        const uint32_t bytes = (uint32_t)min((int64_t)chunk, row_bytes - off);
+        const int s = (int)(n % stages);
         int p[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int j = lane + 32 * h;
             p[h] = j < k ? __ldg(out_perm + t * k + j) : -1;
         }
-        const bool ok = mbar_wait(&bar[s], (uint32_t)((n / kBulkStages) & 1), kMaxPolls);
+        const bool ok = mbar_wait(&bar[s], (uint32_t)((n / stages) & 1), kMaxPolls);
         if (!__all_sync(0xffffffffu, ok)) {
             failed = true;
             break;
         }
-        const unsigned char *src = stage + (size_t)s * kBulkChunk;
+        const unsigned char *src = stage + (size_t)s * chunk;
 #pragma unroll
         for (int h = 0; h < 2; ++h)
             if (p[h] >= 0 && p[h] < S) bulk_s2g(out + (int64_t)p[h] * row_bytes + off, src, bytes);
@@ -96,7 +98,7 @@ __global__ void __launch_bounds__(32)
         }
         bulk_commit();
         if (n >= 1) {
-            bulk_wait_read<1>();  // this lane's stores of chunk n-1 have read their stage
+            bulk_wait_read<1>();  // this lane's stores of unit n-1 have read their stage
             __syncwarp();
             if (lane == 0 && issued < mine) load(issued);
             issued = __shfl_sync(0xffffffffu, issued < mine ? issued + 1 : issued, 0);
@@ -107,7 +109,7 @@ __global__ void __launch_bounds__(32)
         // let every load still in flight land before the block releases its
         // shared memory (again bounded)
         for (int64_t m = n; m < issued; ++m)
-            mbar_wait(&bar[m % kBulkStages], (uint32_t)((m / kBulkStages) & 1), kMaxPolls);
+            mbar_wait(&bar[m % stages], (uint32_t)((m / stages) & 1), kMaxPolls);
     }
     bulk_wait_all();
 }
@@ -217,13 +219,47 @@ __global__ void __launch_bounds__(kFp8Threads)
 
 }  // namespace
 
+// Row split for the bulk dispatch: the number of chunks per row that
+// minimises (units per block) x (bytes per unit + a per-unit overhead), the
+// makespan of a persistent grid of `grid_max` blocks.
+static int64_t bulk_split(int64_t T, int64_t row_bytes, int64_t grid_max) {
+    constexpr int64_t kUnitOverheadBytes = 1024;
+    int64_t best_n = 1, best_cost = -1;
+    for (int64_t n = 1; n <= 16; ++n) {
+        const int64_t chunk = ((row_bytes + n - 1) / n + 15) / 16 * 16;
+        if (chunk > kBulkSmem / 2) continue;  // at least two stages
+        const int64_t nch = (row_bytes + chunk - 1) / chunk;
+        const int64_t units = T * nch;
+        const int64_t grid = units < grid_max ? units : grid_max;
+        const int64_t per = (units + grid - 1) / grid;
+        const int64_t cost = per * (chunk + kUnitOverheadBytes);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best_n = n;
+        }
+        if (chunk <= 16) break;
+    }
+    return best_n;
+}
+
+cudaError_t run_dispatch_scatter_split(const void *x, int64_t T, int64_t row_bytes, int k,
+                                       const int32_t *out_perm, void *out, int64_t nsplit,
+                                       cudaStream_t stream) {
+    const uint32_t chunk = (uint32_t)(((row_bytes + nsplit - 1) / nsplit + 15) / 16 * 16);
+    const int64_t nch = (row_bytes + chunk - 1) / chunk;
+    int stages = (int)(kBulkSmem / chunk);
+    if (stages > kBulkMaxStages) stages = kBulkMaxStages;
+    const size_t smem = (size_t)stages * chunk;
+    const int64_t grid = persistent_grid(dispatch_bulk_kernel, 32, smem, T * nch);
+    return launch(dispatch_bulk_kernel, grid, 32, smem, stream, (const char *)x, T, row_bytes, k,
+                  out_perm, (char *)out, nch, chunk, stages);
+}
+
 cudaError_t run_dispatch_scatter(const void *x, int64_t T, int64_t row_bytes, int k,
                                  const int32_t *out_perm, void *out, cudaStream_t stream) {
-    const size_t smem = (size_t)kBulkStages * kBulkChunk;
-    const int64_t units = T * ((row_bytes + kBulkChunk - 1) / kBulkChunk);
-    const int64_t grid = persistent_grid(dispatch_bulk_kernel, 32, smem, units);
-    return launch(dispatch_bulk_kernel, grid, 32, smem, stream, (const char *)x, T, row_bytes, k,
-                  out_perm, (char *)out);
+    const int64_t grid_max = (int64_t)sm_count() * blocks_per_sm(dispatch_bulk_kernel, 32, kBulkSmem);
+    return run_dispatch_scatter_split(x, T, row_bytes, k, out_perm, out,
+                                      bulk_split(T, row_bytes, grid_max), stream);
 }
 
 cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int k,

@@ -38,12 +38,22 @@ cudaError_t run_prepare_dispatch(const int32_t *ids, int64_t T, int k, int E, in
 cudaError_t run_dispatch_scatter(const void *x, int64_t T, int64_t row_bytes, int k,
                                  const int32_t *out_perm, void *out, cudaStream_t stream);
 
+// The same with an explicit number of chunks per row (for tuning).
+cudaError_t run_dispatch_scatter_split(const void *x, int64_t T, int64_t row_bytes, int k,
+                                       const int32_t *out_perm, void *out, int64_t nsplit,
+                                       cudaStream_t stream);
+
 cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int k,
                                 const int32_t *in_perm, void *out, cudaStream_t stream);
 
 cudaError_t run_dispatch_fp8(const void *x, DType x_dtype, int64_t T, int64_t H, int k, int E,
                              const int32_t *ids, const int32_t *out_perm, const int32_t *offsets,
                              const int32_t *bso, uint8_t *q, float *scales, cudaStream_t stream);
+
+// The same with an explicit column split per row (0 = chosen for balance).
+cudaError_t run_combine_split(const void *y, DType y_dtype, int64_t T, int64_t H, int k,
+                              const int32_t *out_perm, const float *w, void *out,
+                              DType out_dtype, int64_t nsplit, cudaStream_t stream);
 
 cudaError_t run_combine(const void *y, DType y_dtype, int64_t T, int64_t H, int k,
                         const int32_t *out_perm, const float *w, void *out, DType out_dtype,

@@ -32,12 +32,14 @@ inline int sm_count() {
 }
 
 // Raises `kernel`'s dynamic shared-memory limit on the current device to at
-// least `smem` (needed above the 48 KB default).  The limit is per kernel, so
+// least `smem` (needed when dynamic plus static use passes 48 KB).  The limit is per kernel, so
 // it is only ever raised: lowering it for a smaller launch would make a later
 // larger one invalid.
 template <typename Kernel>
 cudaError_t ensure_smem(Kernel kernel, size_t smem) {
-    if (smem <= 48 * 1024) return cudaSuccess;
+    // 48 KB is the default limit for dynamic plus static shared memory; a
+    // dynamic request near it needs the attribute once static use is added
+    if (smem <= 32 * 1024) return cudaSuccess;
     static std::mutex mu;
     static std::map<std::pair<const void *, int>, size_t> limit;
     const auto key = std::make_pair((const void *)kernel, current_device());
