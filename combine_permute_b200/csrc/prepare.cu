@@ -29,8 +29,8 @@ namespace moe {
 
 namespace {
 
-constexpr unsigned long long kFlagAgg = 1ull << 32;
-constexpr unsigned long long kFlagIncl = 2ull << 32;
+constexpr unsigned long long kFlagAgg = 1ull << 32;   // word holds this tile's aggregate
+constexpr unsigned long long kFlagIncl = 2ull << 32;  // word holds the inclusive prefix
 constexpr int kMaxSpins = 1 << 20;  // x ~256 ns sleep: a wait gives up after ~0.3-1 s
 constexpr int kLookbackWindow = 8;  // predecessor tiles read together
 
@@ -140,19 +140,43 @@ __device__ __forceinline__ int offsets_from_totals(int *tot, int *pad, int E, in
 
 __host__ __device__ inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
+// Workspace of the tiled path: a 256-byte header, then one 64-bit look-back
+// word per (tile, expert column).  A word holds epoch << 34 | flag << 32 |
+// value; it counts as published by this call only when its epoch field is
+// this call's epoch, so words left by earlier calls need no clearing.  The
+// epoch advances once per call (by the call's last block); the ticket and
+// done counters wrap back to zero.
 struct PrepWs {
-    unsigned *ticket;
-    unsigned *timeout;
-    unsigned long long *state;  // [G][E+1] look-back words: flag << 32 | value
+    unsigned *ticket;   // tile tickets, wraps at G
+    unsigned *done;     // blocks finished, wraps at G
+    unsigned *epoch;    // this call's epoch
+    unsigned *ready;    // one-pass path: epoch + 1 once the offsets are out
+    unsigned *timeout;  // set when a bounded wait gave up
+    unsigned long long *state;  // [G][E+1] look-back words
 };
 
 __host__ __device__ inline PrepWs carve(void *ws) {
     char *b = (char *)ws;
     PrepWs w;
     w.ticket = (unsigned *)b;
-    w.timeout = (unsigned *)(b + 4);
+    w.done = (unsigned *)(b + 4);
+    w.epoch = (unsigned *)(b + 8);
+    w.ready = (unsigned *)(b + 12);
+    w.timeout = (unsigned *)(b + 16);
     w.state = (unsigned long long *)(b + 256);
     return w;
+}
+
+constexpr unsigned kEpochMask = 0x3fffffffu;
+
+__device__ __forceinline__ unsigned long long lb_word(unsigned epoch, unsigned long long flag,
+                                                      int value) {
+    return ((unsigned long long)(epoch & kEpochMask) << 34) | flag | (unsigned)value;
+}
+
+// Flag bits of a look-back word if it was published in `epoch`, else 0.
+__device__ __forceinline__ unsigned long long lb_flag(unsigned long long w, unsigned epoch) {
+    return (unsigned)(w >> 34) == (epoch & kEpochMask) ? (w & (3ull << 32)) : 0ull;
 }
 
 // ---------------------------------------------------------------------------
@@ -236,46 +260,46 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
 size_t single_block_smem(int E) { return (size_t)(kSingleWarps * (E + 1) + 2 * E) * sizeof(int); }
 
 // ---------------------------------------------------------------------------
-// Tiled path, kernel A: rank every slot of a tile, look back across tiles,
-// store rank(i) in output_permutation (-1 for an invalid id).  The last tile
-// writes counts, offsets and block-scale offsets.
+// Tiled path.  tile_rank_lookback() is the part both variants share: take a
+// tile ticket, rank the tile's slots within each warp's run, fold the warps
+// into the tile histogram, publish it and look back over the earlier tiles.
+// On return (after a block barrier) excl[c] holds the slots of column c in
+// earlier tiles, hist[c] this tile's, wcnt the per-warp exclusive prefixes,
+// and key/rank each thread's slots.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kTileThreads, 2)
-    prep_rank_kernel(const int32_t *__restrict__ ids, int64_t S, int E, int A, int G,
-                     void *workspace, int32_t *counts, int32_t *offsets, int32_t *bso,
-                     int32_t *out_perm, int32_t *diag) {
-    extern __shared__ int smem[];
-    __shared__ int warp_tmp[66];
-    __shared__ unsigned s_ticket;
-    __shared__ int s_invalid;
-    const int C = E + 1;                  // one column per expert plus one for invalid ids
-    int *wcnt = smem;                     // [kTileWarps][E+1]
-    int *hist = wcnt + kTileWarps * C;    // [C] this tile's counts
-    int *excl = hist + C;                 // [C] slots of earlier tiles, then totals
-    int *pad = excl + C;                  // [E]
+struct TileCtx {
+    int tile;
+    unsigned epoch;
+    int64_t wbase;  // first slot of this warp's run
+};
+
+__device__ __forceinline__ TileCtx tile_rank_lookback(
+    const int32_t *__restrict__ ids, int64_t S, int E, int G, const PrepWs &ws, int *wcnt,
+    int *hist, int *excl, unsigned *s_misc, int *s_invalid, int (&key)[kTileRounds],
+    int (&rank)[kTileRounds]) {
+    const int C = E + 1;  // one column per expert plus one for invalid ids
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned lt = lanemask_lt();
     const int nbits = key_bits(E);
-    PrepWs ws = carve(workspace);
 
     for (int x = tid; x < kTileWarps * C; x += kTileThreads) wcnt[x] = 0;
-    if (tid == 0) s_invalid = 0;
-    pdl_wait();
-    pdl_launch_dependents();
     if (tid == 0) {
+        *s_invalid = 0;
         const unsigned t = atomicInc(ws.ticket, (unsigned)(G - 1));
         // a counter left non-zero by an aborted call: stay in bounds; the
-        // bounded waits below then report the failure through diag[1]
-        s_ticket = t < (unsigned)G ? t : t % (unsigned)G;
+        // bounded waits then report the failure through diag[1]
+        s_misc[0] = t < (unsigned)G ? t : t % (unsigned)G;
+        s_misc[1] = *(volatile unsigned *)ws.epoch;
     }
     __syncthreads();
-    const int tile = (int)s_ticket;
-    const int64_t wbase = (int64_t)tile * kTileSlots + (int64_t)warp * 32 * kTileRounds;
+    TileCtx ctx;
+    ctx.tile = (int)s_misc[0];
+    ctx.epoch = s_misc[1];
+    ctx.wbase = (int64_t)ctx.tile * kTileSlots + (int64_t)warp * 32 * kTileRounds;
 
-    // 1. ranks within each warp's run, per-warp counts
-    int key[kTileRounds], rank[kTileRounds];
+    // ranks within each warp's run, per-warp counts
 #pragma unroll
-    for (int r = 0; r < kTileRounds; ++r) key[r] = load_key(ids, wbase + r * 32 + lane, S, E);
+    for (int r = 0; r < kTileRounds; ++r) key[r] = load_key(ids, ctx.wbase + r * 32 + lane, S, E);
     int *row = wcnt + warp * C;
     int bad = 0;
 #pragma unroll
@@ -285,34 +309,34 @@ __global__ void __launch_bounds__(kTileThreads, 2)
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
-    if (lane == 0 && bad) atomicAdd(&s_invalid, bad);
+    if (lane == 0 && bad) atomicAdd(s_invalid, bad);
     __syncthreads();
     fold_warp_counts<kTileThreads, kTileWarps>(wcnt, E, hist);
-    if (tid == 0) hist[E] = s_invalid;
+    if (tid == 0) hist[E] = *s_invalid;
     __syncthreads();
 
-    // 2. publish this tile's aggregates
-    unsigned long long *mine = ws.state + (size_t)tile * C;
-    for (int c = tid; c < C; c += kTileThreads) st_relaxed_u64(mine + c, kFlagAgg | (unsigned)hist[c]);
+    // publish this tile's aggregates
+    unsigned long long *mine = ws.state + (size_t)ctx.tile * C;
+    for (int c = tid; c < C; c += kTileThreads)
+        st_relaxed_u64(mine + c, lb_word(ctx.epoch, kFlagAgg, hist[c]));
 
-    // 3. decoupled look-back, one column per thread, kLookbackWindow
-    //    predecessors read together
+    // decoupled look-back, one column per thread, kLookbackWindow
+    // predecessors read together
     bool gave_up = false;
     for (int c = tid; c < C; c += kTileThreads) {
         int sum = 0;
         bool done = false;
-        for (int pred = tile - 1; pred >= 0 && !done && !gave_up; pred -= kLookbackWindow) {
+        for (int pred = ctx.tile - 1; pred >= 0 && !done && !gave_up; pred -= kLookbackWindow) {
             unsigned long long v[kLookbackWindow];
 #pragma unroll
             for (int q = 0; q < kLookbackWindow; ++q)
-                v[q] = pred - q >= 0 ? ld_relaxed_u64(ws.state + (size_t)(pred - q) * C + c)
-                                     : kFlagIncl;
+                v[q] = pred - q >= 0 ? ld_relaxed_u64(ws.state + (size_t)(pred - q) * C + c) : 0ull;
 #pragma unroll
             for (int q = 0; q < kLookbackWindow; ++q) {
                 if (done || gave_up || pred - q < 0) continue;
                 const unsigned long long *wp = ws.state + (size_t)(pred - q) * C + c;
                 int spins = 0;
-                while ((v[q] >> 32) == 0) {  // not published yet
+                while (lb_flag(v[q], ctx.epoch) == 0) {  // not published by this call yet
                     if (++spins > kMaxSpins) {
                         gave_up = true;
                         break;
@@ -321,42 +345,155 @@ __global__ void __launch_bounds__(kTileThreads, 2)
                     v[q] = ld_relaxed_u64(wp);
                 }
                 sum += (int)(unsigned)(v[q] & 0xffffffffu);
-                if ((v[q] & kFlagIncl) != 0) done = true;
+                if (lb_flag(v[q], ctx.epoch) == kFlagIncl) done = true;
             }
         }
         // publish even after giving up, so that no later tile waits on us
-        st_relaxed_u64(mine + c, kFlagIncl | (unsigned)(sum + hist[c]));
+        st_relaxed_u64(mine + c, lb_word(ctx.epoch, kFlagIncl, sum + hist[c]));
         excl[c] = sum;
     }
     if (gave_up) atomicExch(ws.timeout, 1u);
     __syncthreads();
+    return ctx;
+}
 
-    // 4. rank(i) = earlier tiles + earlier warps + earlier lanes of the run
+// The block's exit: the last block of the call to finish reports a wait
+// that gave up, clears that flag and advances the epoch for the next call.
+__device__ __forceinline__ void tile_finish(const PrepWs &ws, int G, unsigned epoch,
+                                            int32_t *diag) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicInc(ws.done, (unsigned)(G - 1)) == (unsigned)(G - 1)) {
+            const unsigned to = atomicExch(ws.timeout, 0u);
+            if (diag) diag[1] = to ? 1 : 0;
+            *(volatile unsigned *)ws.epoch = epoch + 1;
+        }
+    }
+}
+
+// Shared memory of the tiled kernels: per-warp rows, then hist, excl, off,
+// pad (one column per expert plus one for invalid ids each).
+size_t tile_smem(int E) { return (size_t)(kTileWarps + 4) * (E + 1) * sizeof(int); }
+
+// One-pass variant (all tiles resident together: cooperative launch).  The
+// last tile turns the totals into offsets, writes them and raises `ready`;
+// every tile waits for it (bounded), then writes its slots' final rows into
+// both permutations.
+__global__ void __launch_bounds__(kTileThreads, 2)
+    prep_onepass_kernel(const int32_t *__restrict__ ids, int64_t S, int E, int A, int G,
+                        void *workspace, int32_t *counts, int32_t *offsets, int32_t *bso,
+                        int32_t *in_perm, int32_t *out_perm, int32_t *diag) {
+    extern __shared__ int smem[];
+    __shared__ int warp_tmp[66];
+    __shared__ unsigned s_misc[2];
+    __shared__ int s_invalid, s_total;
+    const int C = E + 1;
+    int *wcnt = smem;                   // [kTileWarps][C]
+    int *hist = wcnt + kTileWarps * C;  // [C]
+    int *excl = hist + C;               // [C]
+    int *off = excl + C;                // [C] expert offsets
+    int *pad = off + C;                 // [C] scan scratch
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    PrepWs ws = carve(workspace);
+    pdl_wait();
+    pdl_launch_dependents();
+    int key[kTileRounds], rank[kTileRounds];
+    const TileCtx ctx =
+        tile_rank_lookback(ids, S, E, G, ws, wcnt, hist, excl, s_misc, &s_invalid, key, rank);
+    if (ctx.tile == G - 1) {
+        // totals = earlier tiles + this one; offsets out, then release the others
+        for (int c = tid; c < C; c += kTileThreads) off[c] = excl[c] + hist[c];
+        __syncthreads();
+        if (tid == 0 && diag) diag[0] = off[E];
+        const int total = offsets_from_totals(off, pad, E, A, true, counts, offsets, bso, warp_tmp);
+        if (tid == 0) {
+            s_total = total;
+            __threadfence();
+            st_release_u32(ws.ready, ctx.epoch + 1);
+        }
+    } else {
+        if (tid == 0) {
+            int spins = 0;
+            while (ld_acquire_u32(ws.ready) != ctx.epoch + 1) {
+                if (++spins > kMaxSpins) {
+                    atomicExch(ws.timeout, 1u);
+                    break;
+                }
+                __nanosleep(128);
+            }
+        }
+        __syncthreads();
+        for (int c = tid; c <= E; c += kTileThreads) off[c] = __ldcg(offsets + c);
+        if (tid == 0) s_total = __ldcg(offsets + E);
+    }
+    __syncthreads();
+    const int total = s_total;
+    const int *row = wcnt + warp * C;
 #pragma unroll
     for (int r = 0; r < kTileRounds; ++r) {
-        const int64_t i = wbase + r * 32 + lane;
+        const int64_t i = ctx.wbase + r * 32 + lane;
+        if (i < S) {
+            const int e = key[r];
+            const int p = e >= 0 ? off[e] + excl[e] + row[e] + rank[r] : -1;
+            out_perm[i] = p;
+            if (p >= 0 && p < S) in_perm[p] = (int)i;
+        }
+    }
+    const int64_t base = (int64_t)ctx.tile * kTileSlots;
+    const int64_t lo = base > total ? base : (int64_t)total;
+    const int64_t hi = base + kTileSlots < S ? base + kTileSlots : S;
+    for (int64_t p = lo + tid; p < hi; p += kTileThreads) in_perm[p] = -1;
+    tile_finish(ws, G, ctx.epoch, diag);
+}
+
+// Two-kernel variant, kernel 1 (any number of tiles): store rank(i) in
+// output_permutation (-1 for an invalid id); the last tile writes counts,
+// offsets and block-scale offsets.
+__global__ void __launch_bounds__(kTileThreads, 2)
+    prep_rank_kernel(const int32_t *__restrict__ ids, int64_t S, int E, int A, int G,
+                     void *workspace, int32_t *counts, int32_t *offsets, int32_t *bso,
+                     int32_t *out_perm, int32_t *diag) {
+    extern __shared__ int smem[];
+    __shared__ int warp_tmp[66];
+    __shared__ unsigned s_misc[2];
+    __shared__ int s_invalid;
+    const int C = E + 1;
+    int *wcnt = smem;
+    int *hist = wcnt + kTileWarps * C;
+    int *excl = hist + C;
+    int *off = excl + C;
+    int *pad = off + C;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    PrepWs ws = carve(workspace);
+    pdl_wait();
+    pdl_launch_dependents();
+    int key[kTileRounds], rank[kTileRounds];
+    const TileCtx ctx =
+        tile_rank_lookback(ids, S, E, G, ws, wcnt, hist, excl, s_misc, &s_invalid, key, rank);
+    const int *row = wcnt + warp * C;
+#pragma unroll
+    for (int r = 0; r < kTileRounds; ++r) {
+        const int64_t i = ctx.wbase + r * 32 + lane;
         if (i < S) {
             const int e = key[r];
             out_perm[i] = e >= 0 ? excl[e] + row[e] + rank[r] : -1;
         }
     }
-
-    // 5. the last tile holds the totals
-    if (tile != G - 1) return;
-    __syncthreads();  // every rank above has read excl
-    for (int c = tid; c < C; c += kTileThreads) excl[c] += hist[c];
-    __syncthreads();
-    if (tid == 0 && diag) diag[0] = excl[E];
-    offsets_from_totals(excl, pad, E, A, true, counts, offsets, bso, warp_tmp);
+    if (ctx.tile == G - 1) {
+        for (int c = threadIdx.x; c < C; c += kTileThreads) off[c] = excl[c] + hist[c];
+        __syncthreads();
+        if (threadIdx.x == 0 && diag) diag[0] = off[E];
+        offsets_from_totals(off, pad, E, A, true, counts, offsets, bso, warp_tmp);
+    }
+    tile_finish(ws, G, ctx.epoch, diag);
 }
 
-// Tiled path, kernel B (element-wise): row = expert offset + rank; both
-// permutations; clear the look-back words.
+// Two-kernel variant, kernel 2 (element-wise): row = expert offset + rank;
+// both permutations.
 __global__ void __launch_bounds__(256)
-    prep_finish_kernel(const int32_t *__restrict__ ids, int64_t S, int E, int64_t ws_words,
-                       void *workspace, const int32_t *__restrict__ offsets, int32_t *in_perm,
-                       int32_t *out_perm, int32_t *diag) {
-    PrepWs ws = carve(workspace);
+    prep_finish_kernel(const int32_t *__restrict__ ids, int64_t S, int E,
+                       const int32_t *__restrict__ offsets, int32_t *in_perm, int32_t *out_perm) {
     pdl_wait();
     pdl_launch_dependents();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -370,11 +507,6 @@ __global__ void __launch_bounds__(256)
         }
     }
     for (int64_t p = __ldg(offsets + E) + g; p < S; p += stride) in_perm[p] = -1;
-    for (int64_t w = g; w < ws_words; w += stride) ws.state[w] = 0ull;
-    if (g == 0) {
-        if (diag) diag[1] = *ws.timeout ? 1 : 0;
-        *ws.timeout = 0u;
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -415,6 +547,42 @@ size_t prepare_workspace_bytes(int64_t S, int E) {
     return 256 + align256((size_t)G * ((size_t)E + 1) * 8);
 }
 
+namespace {
+
+// One cooperative launch of prep_onepass_kernel when every tile fits on the
+// GPU at once; returns cudaErrorCooperativeLaunchTooLarge (nothing launched)
+// when the tiles do not fit or the launch form is refused.
+cudaError_t launch_onepass(const int32_t *ids, int64_t S, int E, int A, int G, void *workspace,
+                           int32_t *counts, int32_t *offsets, int32_t *bso, int32_t *in_perm,
+                           int32_t *out_perm, int32_t *diag, cudaStream_t stream) {
+    const size_t smem = tile_smem(E);
+    const int64_t resident = (int64_t)sm_count() * blocks_per_sm(prep_onepass_kernel, kTileThreads, smem);
+    if (G > resident) return cudaErrorCooperativeLaunchTooLarge;
+    cudaError_t se = ensure_smem(prep_onepass_kernel, smem);
+    if (se != cudaSuccess) return se;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)G, 1, 1);
+    cfg.blockDim = dim3(kTileThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    for (int n : {2, 1}) {  // with programmatic serialization if allowed, else without
+        cfg.numAttrs = n;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, prep_onepass_kernel, ids, S, E, A, G, workspace,
+                                           counts, offsets, bso, in_perm, out_perm, diag);
+        if (e == cudaSuccess) return cudaGetLastError();
+        cudaGetLastError();
+    }
+    return cudaErrorCooperativeLaunchTooLarge;
+}
+
+}  // namespace
+
 cudaError_t run_prepare(const int32_t *ids, int64_t S, int E, int A, int32_t *counts,
                         int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,
                         int32_t *diag, void *workspace, cudaStream_t stream) {
@@ -422,14 +590,15 @@ cudaError_t run_prepare(const int32_t *ids, int64_t S, int E, int A, int32_t *co
         return launch(prep_single_kernel, 1, kSingleThreads, single_block_smem(E), stream, ids, S,
                       E, A, counts, offsets, bso, in_perm, out_perm, diag);
     const int G = (int)((S + kTileSlots - 1) / kTileSlots);
-    const size_t smem = (size_t)(kTileWarps * (E + 1) + 2 * (E + 1) + E) * sizeof(int);
-    cudaError_t e = launch(prep_rank_kernel, G, kTileThreads, smem, stream, ids, S, E, A, G,
-                           workspace, counts, offsets, bso, out_perm, diag);
+    cudaError_t e = launch_onepass(ids, S, E, A, G, workspace, counts, offsets, bso, in_perm,
+                                   out_perm, diag, stream);
+    if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+    e = launch(prep_rank_kernel, G, kTileThreads, tile_smem(E), stream, ids, S, E, A, G,
+               workspace, counts, offsets, bso, out_perm, diag);
     if (e != cudaSuccess) return e;
-    const int64_t words = (int64_t)G * (E + 1);
     const int64_t grid = persistent_grid(prep_finish_kernel, 256, 0, (S + 1023) / 1024);
-    return launch(prep_finish_kernel, grid, 256, 0, stream, ids, S, E, words, workspace,
-                  (const int32_t *)offsets, in_perm, out_perm, diag);
+    return launch(prep_finish_kernel, grid, 256, 0, stream, ids, S, E, (const int32_t *)offsets,
+                  in_perm, out_perm);
 }
 
 cudaError_t run_prepare_dispatch(const int32_t *ids, int64_t T, int k, int E, int A,

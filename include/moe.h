@@ -84,11 +84,12 @@ const char *moe_last_cuda_error(void);
 /*
  * Bytes of scratch workspace moe_prepare needs for this problem size: 0 up
  * to 4096 slots (T*k), which run in one block without one.  The workspace
- * must be all-zero before its first use (e.g. one cudaMemsetAsync); every
- * completed call leaves it all-zero again, so one workspace serves any
- * number of consecutive calls on one stream.  Calls that may run
- * concurrently need separate workspaces.  After a call that reported a
- * CUDA error, zero it again.
+ * must be all-zero before its first use (e.g. one cudaMemsetAsync); the
+ * library maintains it from then on (it holds a call counter and look-back
+ * words tagged with it, so it is not all-zero between calls), and one
+ * workspace serves any number of consecutive calls of any size on one
+ * stream.  Zero it again only as a whole, and after a call that reported a
+ * CUDA error.  Calls that may run concurrently need separate workspaces.
  */
 size_t moe_prepare_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t num_experts);
 
@@ -125,7 +126,8 @@ size_t moe_prepare_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t nu
  *                                      size is 0.
  *
  * Batches of up to 4096 slots run in one block; larger ones as tiles over
- * the whole GPU in two kernels (the only case that touches the workspace).
+ * the whole GPU (the only case that touches the workspace): one cooperative
+ * launch when every tile fits on the GPU at once, else two kernels.
  *
  * Dispatched order: by expert ascending, and within an expert by expanded
  * index ascending (token, then slot): a stable counting sort, so the result

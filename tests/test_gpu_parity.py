@@ -96,18 +96,29 @@ def test_prepare_full_workloads(name):
 
 
 @pytest.mark.parametrize("T", [131072, 200000])
-def test_prepare_deterministic_and_workspace_left_zero(T):
+def test_prepare_deterministic_and_workspace_reusable(T):
+    """Repeated calls give identical results, and one workspace serves calls
+    of different sizes in any order (look-back words left by an earlier call
+    never count for a later one)."""
     w = CONFIGS["zipf_fp16_t131072_h2048_e64_k6"].scaled(T)
     ids_np, _, _, _ = make_workload(w, with_x=False, with_y=False)
     ids = torch.from_numpy(ids_np).to(DEV)
     nbytes = moe.moe_prepare_workspace_bytes(w.T, w.k, w.E)
     ws = torch.zeros(nbytes, dtype=torch.uint8, device=DEV)
     runs = [moe.moe_prepare(ids, w.E, blockscale_align=16, workspace=ws) for _ in range(3)]
+    small = CONFIGS["uniform_t4096_h7168_e256_k8"].scaled(3000)
+    sids_np, _, _, _ = make_workload(small, with_x=False, with_y=False)
+    smeta = moe.moe_prepare(torch.from_numpy(sids_np).to(DEV), small.E, workspace=ws)
+    runs.append(moe.moe_prepare(ids, w.E, blockscale_align=16, workspace=ws))
     torch.cuda.synchronize()
-    assert int(ws.count_nonzero()) == 0
     for r in runs[1:]:
         for a, b in zip(runs[0], r):
             assert torch.equal(a, b)
+    ref = oracle.prepare(ids_np, w.E, 16)
+    np.testing.assert_array_equal(runs[-1].output_permutation.cpu().numpy(), ref["output_perm"])
+    sref = oracle.prepare(sids_np, small.E)
+    np.testing.assert_array_equal(smeta.input_permutation.cpu().numpy(), sref["input_perm"])
+    assert runs[-1].diag.cpu().tolist() == [0, 0]
 
 
 # ---------------------------------------------------------------------------
