@@ -33,7 +33,7 @@ from .build import build_oracle, oracle_lib_path
 
 __all__ = [
     "F32", "F16", "BF16", "lib", "prepare", "dispatch", "dispatch_fp8",
-    "combine", "brute_prepare", "f32_to_bf16", "f32_to_f16", "f16_to_f32",
+    "combine", "brute_prepare", "problem_sizes", "tile_layout", "f32_to_bf16", "f32_to_f16", "f16_to_f32",
     "bf16_to_f32", "f32_to_e4m3", "e4m3_to_f32",
 ]
 
@@ -65,6 +65,11 @@ def lib():
         L.oracle_combine.restype = None
         L.oracle_combine.argtypes = [_vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
                                      ctypes.c_int32, _vp, _vp, _vp, ctypes.c_int]
+        L.oracle_problem_sizes.restype = None
+        L.oracle_problem_sizes.argtypes = [_vp, ctypes.c_int32] + [ctypes.c_int32] * 4 + [_vp, _vp]
+        L.oracle_tile_layout.restype = ctypes.c_int
+        L.oracle_tile_layout.argtypes = [_vp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
+                                         ctypes.c_int32, _vp, _vp, _vp, ctypes.c_int32] + [_vp] * 7
         for name in ["oracle_f32_to_e4m3_n", "oracle_f32_to_bf16_n", "oracle_f32_to_f16_n",
                      "oracle_f16_to_f32_n", "oracle_bf16_to_f32_n", "oracle_e4m3_to_f32_n"]:
             fn = getattr(L, name)
@@ -151,6 +156,36 @@ def combine(y_bits: np.ndarray, y_dtype: str, output_perm: np.ndarray, w: np.nda
     out = np.zeros((T, H), np.float32 if out_dtype == "fp32" else np.uint16)
     lib().oracle_combine(_ptr(y_bits), _DT[y_dtype], T, H, k, _ptr(output_perm), _ptr(w),
                          _ptr(out), _DT[out_dtype])
+    return out
+
+
+def problem_sizes(counts: np.ndarray, n1: int, k1: int, n2: int, k2: int):
+    """(M, N, K) of the two grouped GEMMs per expert: [E,3] int32 each."""
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    E = counts.size
+    ps1 = np.zeros((E, 3), np.int32)
+    ps2 = np.zeros((E, 3), np.int32)
+    lib().oracle_problem_sizes(_ptr(counts), E, n1, k1, n2, k2, _ptr(ps1), _ptr(ps2))
+    return ps1, ps2
+
+
+def tile_layout(ids: np.ndarray, meta: dict, E: int, tile: int, max_tiles: int):
+    """Tile-padded grouped-GEMM layout (see moe_oracle.c).  Returns a dict,
+    or None when max_tiles * tile cannot hold the padded rows."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, k = ids.shape
+    out = dict(padded_offsets=np.zeros(E + 1, np.int32), tile_group=np.zeros(max_tiles, np.int32),
+               tile_mn_limit=np.zeros(max_tiles, np.int32), exp2perm=np.zeros(T * k, np.int32),
+               perm2exp=np.zeros(max_tiles * tile, np.int32), num_tiles=np.zeros(1, np.int32),
+               total_padded=np.zeros(1, np.int32))
+    rc = lib().oracle_tile_layout(_ptr(ids), T, k, E, tile, _ptr(meta["counts"]), _ptr(meta["offsets"]),
+                                  _ptr(meta["output_perm"]), max_tiles, _ptr(out["padded_offsets"]),
+                                  _ptr(out["tile_group"]), _ptr(out["tile_mn_limit"]), _ptr(out["exp2perm"]),
+                                  _ptr(out["perm2exp"]), _ptr(out["num_tiles"]), _ptr(out["total_padded"]))
+    if rc != 0:
+        return None
+    out["num_tiles"] = int(out["num_tiles"][0])
+    out["total_padded"] = int(out["total_padded"][0])
     return out
 
 

@@ -379,3 +379,87 @@ void oracle_e4m3_to_f32_n(const uint8_t *in, int64_t n, float *out)
     for (int64_t i = 0; i < n; ++i)
         out[i] = oracle_e4m3_to_f32(in[i]);
 }
+
+/* ------------------------------------------------------------------ */
+/* Grouped-GEMM metadata (the step after prepare).                     */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Problem sizes of the two grouped GEMMs that follow dispatch (sglang PR
+ * #19058, item 1: compute_problem_sizes_kernel fills problem_sizes1 /
+ * problem_sizes2): for every expert e, ps1[e] = {counts[e], n1, k1} and
+ * ps2[e] = {counts[e], n2, k2} as (M, N, K).
+ */
+void oracle_problem_sizes(const int32_t *counts, int32_t E, int32_t n1, int32_t k1, int32_t n2,
+                          int32_t k2, int32_t *ps1, int32_t *ps2)
+{
+    for (int32_t e = 0; e < E; ++e) {
+        ps1[3 * e + 0] = counts[e];
+        ps1[3 * e + 1] = n1;
+        ps1[3 * e + 2] = k1;
+        ps2[3 * e + 0] = counts[e];
+        ps2[3 * e + 1] = n2;
+        ps2[3 * e + 2] = k2;
+    }
+}
+
+/*
+ * Tile-padded layout for a tiled grouped GEMM (the moe_sort outputs of
+ * TensorRT-LLM PR #9592: tile_idx_to_group_idx, tile_idx_to_mn_limit,
+ * expanded_idx_to_permuted_idx, permuted_idx_to_expanded_idx,
+ * total_num_padded_tokens, num_non_exiting_tiles).  Every expert's rows are
+ * padded up to a multiple of the tile size:
+ *   padded_offsets[e]  = sum over e' < e of roundup(counts[e'], tile)
+ *   tile t (of the first padded_offsets[E] / tile) belongs to the expert e
+ *     whose padded range holds row t*tile; its row limit is
+ *     padded_offsets[e] + counts[e]; tiles past the last are -1 / -1;
+ *   a valid slot i of expert e with dispatched row p lands on padded row
+ *     padded_offsets[e] + (p - offsets[e]);
+ *   permuted_idx_to_expanded_idx is the inverse, -1 on padding rows and on
+ *     every row past the padded total (up to max_tiles * tile).
+ * Returns 0, or -1 when max_tiles * tile is too small for the padded total
+ * (then nothing is written).
+ */
+int oracle_tile_layout(const int32_t *ids, int64_t T, int32_t k, int32_t E, int32_t tile,
+                       const int32_t *counts, const int32_t *offsets, const int32_t *output_perm,
+                       int32_t max_tiles, int32_t *padded_offsets, int32_t *tile_group,
+                       int32_t *tile_mn_limit, int32_t *exp2perm, int32_t *perm2exp,
+                       int32_t *num_tiles, int32_t *total_padded)
+{
+    int64_t S = T * (int64_t)k;
+    int64_t acc = 0;
+    for (int32_t e = 0; e < E; ++e)
+        acc += (counts[e] + tile - 1) / tile * (int64_t)tile;
+    if (acc > (int64_t)max_tiles * tile)
+        return -1;
+    padded_offsets[0] = 0;
+    for (int32_t e = 0; e < E; ++e)
+        padded_offsets[e + 1] = padded_offsets[e] + (counts[e] + tile - 1) / tile * tile;
+    *total_padded = padded_offsets[E];
+    *num_tiles = padded_offsets[E] / tile;
+    for (int32_t t = 0; t < max_tiles; ++t) {
+        tile_group[t] = -1;
+        tile_mn_limit[t] = -1;
+    }
+    int32_t t = 0;
+    for (int32_t e = 0; e < E; ++e) {
+        for (int32_t r = padded_offsets[e]; r < padded_offsets[e + 1]; r += tile) {
+            tile_group[t] = e;
+            tile_mn_limit[t] = padded_offsets[e] + counts[e];
+            ++t;
+        }
+    }
+    for (int64_t q = 0; q < (int64_t)max_tiles * tile; ++q)
+        perm2exp[q] = -1;
+    for (int64_t i = 0; i < S; ++i) {
+        int32_t e = ids[i];
+        if (e < 0 || e >= E) {
+            exp2perm[i] = -1;
+            continue;
+        }
+        int32_t pp = padded_offsets[e] + (output_perm[i] - offsets[e]);
+        exp2perm[i] = pp;
+        perm2exp[pp] = (int32_t)i;
+    }
+    return 0;
+}

@@ -372,3 +372,62 @@ def test_combine_skips_invalid_slots():
     w = np.array([[0.5, 100.0], [2.0, 100.0]], np.float32)
     got = oracle.combine(y.numpy(), "fp32", out_perm, w, "fp32")
     np.testing.assert_array_equal(got, [[1.5, 2.0], [2.0, 4.0]])
+
+
+# ---------------------------------------------------------------------------
+# grouped-GEMM metadata (problem sizes, tile-padded layout)
+# ---------------------------------------------------------------------------
+
+def test_problem_sizes_closed_form():
+    counts = np.array([0, 5, 3, 9], np.int32)
+    ps1, ps2 = oracle.problem_sizes(counts, 14336, 7168, 7168, 7168)
+    np.testing.assert_array_equal(ps1, np.stack([counts, np.full(4, 14336), np.full(4, 7168)], 1))
+    np.testing.assert_array_equal(ps2, np.stack([counts, np.full(4, 7168), np.full(4, 7168)], 1))
+
+
+def test_tile_layout_hand_worked_example():
+    # ids [[2,0],[1,2],[2,1]], E=3, tile 2: counts [1,2,3] pad to [2,2,4]
+    # rows: expert 0 -> 0 (1 padding), expert 1 -> 2,3, expert 2 -> 4,5,6 (7 padding)
+    ids = np.array([[2, 0], [1, 2], [2, 1]], np.int32)
+    m = oracle.prepare(ids, 3)
+    L = oracle.tile_layout(ids, m, 3, 2, 6)
+    assert L["padded_offsets"].tolist() == [0, 2, 4, 8]
+    assert L["num_tiles"] == 4 and L["total_padded"] == 8
+    assert L["tile_group"].tolist() == [0, 1, 2, 2, -1, -1]
+    assert L["tile_mn_limit"].tolist() == [1, 4, 7, 7, -1, -1]
+    assert L["exp2perm"].tolist() == [4, 0, 2, 5, 6, 3]
+    assert L["perm2exp"].tolist() == [1, -1, 2, 5, 0, 3, 4, -1, -1, -1, -1, -1]
+    assert oracle.tile_layout(ids, m, 3, 2, 3) is None   # 6 rows cannot hold 8
+
+
+@pytest.mark.parametrize("tile", [1, 7, 128])
+@pytest.mark.parametrize("name", ["uniform_t4096_h7168_e256_k8", "zipf_fp8_t16384_h4096_e288_k8"])
+def test_tile_layout_invariants(name, tile):
+    w = CONFIGS[name].scaled(3000)
+    ids, _, _, _ = make_workload(w, with_x=False, with_y=False)
+    ids = ids.copy()
+    ids[::53, 1] = -1
+    m = oracle.prepare(ids, w.E)
+    max_tiles = -(-w.S // tile) + w.E
+    L = oracle.tile_layout(ids, m, w.E, tile, max_tiles)
+    per_expert = -(-m["counts"] // tile)
+    # library special case: the tile owners are each expert repeated once per tile
+    np.testing.assert_array_equal(L["tile_group"][:L["num_tiles"]],
+                                  np.repeat(np.arange(w.E), per_expert))
+    assert (L["tile_group"][L["num_tiles"]:] == -1).all()
+    np.testing.assert_array_equal(L["padded_offsets"][1:], np.cumsum(per_expert * tile))
+    g = L["tile_group"][:L["num_tiles"]]
+    np.testing.assert_array_equal(L["tile_mn_limit"][:L["num_tiles"]],
+                                  L["padded_offsets"][g] + m["counts"][g])
+    # the padded rows hold exactly the valid slots, each expert's in its own range, in order
+    flat = ids.ravel()
+    valid = (flat >= 0) & (flat < w.E)
+    e2p = L["exp2perm"]
+    assert (e2p[~valid] == -1).all()
+    rows = e2p[valid]
+    assert np.unique(rows).size == rows.size
+    np.testing.assert_array_equal(L["perm2exp"][rows], np.nonzero(valid)[0])
+    assert (np.delete(L["perm2exp"], rows) == -1).all()
+    e = flat[valid]
+    assert (rows >= L["padded_offsets"][e]).all() and (rows < L["padded_offsets"][e] + m["counts"][e]).all()
+    np.testing.assert_array_equal(rows - L["padded_offsets"][e], m["output_perm"][valid] - m["offsets"][e])
