@@ -458,6 +458,7 @@ def run_gpu(args, w):
 
     # ---- end to end through the public API from pinned host buffers
     e2e = run_e2e(step, w, dev, K, W, barrier, max_over_ranks)
+    next_rows = time_next_rows(step, w, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -511,6 +512,7 @@ def run_gpu(args, w):
         "gpu_launches": step.launches_per_step * K,
         "clocks": clocks.summary(),
         "breakdown": breakdown,
+        "next_rows": next_rows,
         "expert_load": {"max_tokens_per_expert": int(counts.max()),
                         "min_tokens_per_expert": int(counts.min()),
                         "mean_tokens_per_expert": float(counts.mean()),
@@ -518,6 +520,46 @@ def run_gpu(args, w):
         "diag": diag,
     }
     print(json.dumps(line), flush=True)
+
+
+def time_next_rows(step, w, dev, reps=20):
+    """The grouped-GEMM metadata steps that follow prepare (tile-padded
+    layout with 128-row tiles, and the per-expert problem sizes), timed on
+    this workload's metadata as a CUDA graph of `reps` calls each."""
+    import torch
+    moe = step.moe
+    meta = step.prepare()
+    tile = 128
+    S, E = w.S, w.E
+    max_tiles = max(1, -(-S // tile) + min(E, S))
+    out = {}
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for _ in range(reps):
+                    fn()
+        torch.cuda.synchronize(dev)
+        g.replay()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        g.replay()
+        e.record()
+        torch.cuda.synchronize(dev)
+        return s.elapsed_time(e) / reps * 1e3
+
+    us = timed(lambda: moe.moe_tile_layout(step.ids, meta, tile, max_tiles))
+    b = 8 * S + 8 * E + 4 * (E + 1) + 8 * max_tiles + 4 * S + 4 * max_tiles * tile + 8
+    out["tile_layout_t128"] = {"us": us, "algorithmic_bytes": b, "effective_gbs": b / us / 1e3}
+    us = timed(lambda: moe.moe_problem_sizes(meta.expert_counts, 2 * w.H, w.H, w.H, w.H))
+    b = 4 * E + 24 * E
+    out["problem_sizes"] = {"us": us, "algorithmic_bytes": b}
+    return out
 
 
 def run_e2e(step, w, dev, K, W, barrier, max_over_ranks):

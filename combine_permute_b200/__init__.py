@@ -31,6 +31,9 @@ __all__ = [
     "moe_combine",
     "moe_prepare_dispatch",
     "moe_version",
+    "moe_problem_sizes",
+    "moe_tile_layout",
+    "TileLayout",
     "library_path",
 ]
 
@@ -39,6 +42,16 @@ _DTYPES = {
     torch.float16: _lib.MOE_F16,
     torch.bfloat16: _lib.MOE_BF16,
 }
+
+
+class TileLayout(NamedTuple):
+    padded_offsets: torch.Tensor                # [E+1]
+    tile_idx_to_group_idx: torch.Tensor         # [max_tiles]
+    tile_idx_to_mn_limit: torch.Tensor          # [max_tiles]
+    expanded_idx_to_permuted_idx: torch.Tensor  # [T*k]
+    permuted_idx_to_expanded_idx: torch.Tensor  # [max_tiles * tile_size]
+    num_non_exiting_tiles: torch.Tensor         # [1] (-1: max_tiles too small)
+    total_num_padded_tokens: torch.Tensor       # [1]
 
 
 class PrepareResult(NamedTuple):
@@ -86,8 +99,8 @@ def _dtype_code(dt: torch.dtype) -> int:
     return _DTYPES[dt]
 
 
-# One zero-initialised prepare workspace per (device, stream); the library
-# leaves it zeroed after every call.
+# One prepare workspace per (device, stream), zeroed once when allocated;
+# the library maintains it between calls.
 _WORKSPACES: dict = {}
 
 
@@ -278,3 +291,43 @@ def moe_prepare_dispatch(topk_ids: torch.Tensor, num_experts: int, x: torch.Tens
             _stream(dev))
     _lib.check("moe_prepare_dispatch", st)
     return meta, out
+
+
+def moe_problem_sizes(expert_counts: torch.Tensor, n1: int, k1: int, n2: int, k2: int):
+    """(M, N, K) per expert of the two grouped GEMMs: two [E, 3] int32 tensors."""
+    _need(expert_counts, "expert_counts", torch.int32)
+    E = expert_counts.numel()
+    dev = expert_counts.device
+    ps1 = torch.empty((E, 3), dtype=torch.int32, device=dev)
+    ps2 = torch.empty((E, 3), dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_problem_sizes(expert_counts.data_ptr(), E, n1, k1, n2, k2,
+                                           ps1.data_ptr(), ps2.data_ptr(), _stream(dev))
+    _lib.check("moe_problem_sizes", st)
+    return ps1, ps2
+
+
+def moe_tile_layout(topk_ids: torch.Tensor, meta: PrepareResult, tile_size: int,
+                    max_tiles: Optional[int] = None) -> TileLayout:
+    """Tile-padded grouped-GEMM layout from moe_prepare's results (see
+    include/moe.h).  Without ``max_tiles`` the always-sufficient bound
+    ceil(T*k / tile) + min(E, T*k) is used."""
+    _need(topk_ids, "topk_ids", torch.int32)
+    T, k = topk_ids.shape
+    E = meta.expert_counts.numel()
+    S = T * k
+    dev = topk_ids.device
+    if max_tiles is None:
+        max_tiles = max(1, -(-S // tile_size) + min(E, S))
+    i32 = dict(dtype=torch.int32, device=dev)
+    out = TileLayout(torch.empty(E + 1, **i32), torch.empty(max_tiles, **i32),
+                     torch.empty(max_tiles, **i32), torch.empty(S, **i32),
+                     torch.empty(max_tiles * tile_size, **i32), torch.empty(1, **i32),
+                     torch.empty(1, **i32))
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_tile_layout(
+            topk_ids.data_ptr(), T, k, E, tile_size, meta.expert_counts.data_ptr(),
+            meta.expert_offsets.data_ptr(), _ptr(meta.output_permutation) if S else None,
+            max_tiles, *[_ptr(t) if t.numel() else None for t in out], _stream(dev))
+    _lib.check("moe_tile_layout", st)
+    return out

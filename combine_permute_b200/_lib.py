@@ -32,6 +32,8 @@ EXPORTED = (
     "moe_combine",
     "moe_prepare_dispatch",
     "moe_prepare_no_alloc",
+    "moe_problem_sizes",
+    "moe_tile_layout",
 )
 
 _vp = ctypes.c_void_p
@@ -54,6 +56,9 @@ _SIGNATURES = {
                                     _vp, _int, _i64, _vp, _vp]),
     "moe_prepare_no_alloc": (_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp,
                                     _vp]),
+    "moe_problem_sizes": (_int, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moe_tile_layout": (_int, [_vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp,
+                               _vp, _vp, _vp, _vp, _vp]),
 }
 
 _lib = None

@@ -173,4 +173,40 @@ moe_status_t moe_prepare_dispatch(const int32_t *topk_ids, int64_t num_tokens, i
         diag, x, row_bytes, out, (cudaStream_t)stream));
 }
 
+moe_status_t moe_problem_sizes(const int32_t *expert_counts, int32_t num_experts, int32_t n1,
+                               int32_t k1, int32_t n2, int32_t k2, int32_t *problem_sizes1,
+                               int32_t *problem_sizes2, moe_stream_t stream) {
+    if (num_experts < 1 || !expert_counts || !problem_sizes1) return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_problem_sizes(expert_counts, num_experts, n1, k1, n2, k2,
+                                            problem_sizes1, problem_sizes2, (cudaStream_t)stream));
+}
+
+moe_status_t moe_tile_layout(const int32_t *topk_ids, int64_t num_tokens, int32_t top_k,
+                             int32_t num_experts, int32_t tile_size, const int32_t *expert_counts,
+                             const int32_t *expert_offsets, const int32_t *output_permutation,
+                             int32_t max_tiles, int32_t *padded_offsets,
+                             int32_t *tile_idx_to_group_idx, int32_t *tile_idx_to_mn_limit,
+                             int32_t *expanded_idx_to_permuted_idx,
+                             int32_t *permuted_idx_to_expanded_idx,
+                             int32_t *num_non_exiting_tiles, int32_t *total_num_padded_tokens,
+                             moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (num_experts < 1 || tile_size < 1 || max_tiles < 1) return MOE_ERR_INVALID_ARG;
+    if (num_experts > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    if ((int64_t)max_tiles * tile_size >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
+    const int64_t S = num_tokens * (int64_t)top_k;
+    if (!expert_counts || !expert_offsets || !padded_offsets || !tile_idx_to_group_idx ||
+        !tile_idx_to_mn_limit || !permuted_idx_to_expanded_idx || !num_non_exiting_tiles ||
+        !total_num_padded_tokens)
+        return MOE_ERR_INVALID_ARG;
+    if (S > 0 && (!topk_ids || !output_permutation || !expanded_idx_to_permuted_idx))
+        return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_tile_layout(
+        topk_ids, S, num_experts, tile_size, expert_counts, expert_offsets, output_permutation,
+        max_tiles, padded_offsets, tile_idx_to_group_idx, tile_idx_to_mn_limit,
+        expanded_idx_to_permuted_idx, permuted_idx_to_expanded_idx, num_non_exiting_tiles,
+        total_num_padded_tokens, (cudaStream_t)stream));
+}
+
 }  // extern "C"

@@ -59,4 +59,13 @@ cudaError_t run_combine(const void *y, DType y_dtype, int64_t T, int64_t H, int 
                         const int32_t *out_perm, const float *w, void *out, DType out_dtype,
                         cudaStream_t stream);
 
+cudaError_t run_problem_sizes(const int32_t *counts, int E, int n1, int k1, int n2, int k2,
+                              int32_t *ps1, int32_t *ps2, cudaStream_t stream);
+
+cudaError_t run_tile_layout(const int32_t *ids, int64_t S, int E, int tile, const int32_t *counts,
+                            const int32_t *offsets, const int32_t *out_perm, int max_tiles,
+                            int32_t *padded_offsets, int32_t *tile_group, int32_t *tile_limit,
+                            int32_t *exp2perm, int32_t *perm2exp, int32_t *num_tiles,
+                            int32_t *total_padded, cudaStream_t stream);
+
 }  // namespace moe

@@ -217,6 +217,65 @@ moe_status_t moe_combine(const void *y, moe_dtype_t y_dtype, int64_t num_tokens,
                          int32_t top_k, const int32_t *output_permutation, const float *weights,
                          void *out, moe_dtype_t out_dtype, moe_stream_t stream);
 
+/*
+ * Problem sizes of the two grouped GEMMs that follow dispatch (sglang PR
+ * #19058, "Changes", item 1: compute_problem_sizes_kernel fills
+ * problem_sizes1 / problem_sizes2): for every expert e,
+ *
+ *   problem_sizes1[e] = {expert_counts[e], n1, k1}
+ *   problem_sizes2[e] = {expert_counts[e], n2, k2}      (M, N, K)
+ *
+ * e.g. n1 = 2 * intermediate, k1 = hidden for the gate/up projection and
+ * n2 = hidden, k2 = intermediate for the down projection.
+ *
+ *   expert_counts    [E]    int32 (from moe_prepare)
+ *   problem_sizes1   [E, 3] int32 out; problem_sizes2 [E, 3] int32 out or NULL
+ */
+moe_status_t moe_problem_sizes(const int32_t *expert_counts, int32_t num_experts, int32_t n1,
+                               int32_t k1, int32_t n2, int32_t k2, int32_t *problem_sizes1,
+                               int32_t *problem_sizes2, moe_stream_t stream);
+
+/*
+ * Tile-padded layout for a tiled grouped GEMM (TensorRT-LLM PR #9592, the
+ * moe_sort outputs tile_idx_to_group_idx, tile_idx_to_mn_limit,
+ * expanded_idx_to_permuted_idx, permuted_idx_to_expanded_idx,
+ * total_num_padded_tokens, num_non_exiting_tiles).  Every expert's rows are
+ * padded up to a multiple of tile_size:
+ *
+ *   padded_offsets[e]  = sum over e' < e of roundup(expert_counts[e'], tile)
+ *   tile t < num_non_exiting_tiles belongs to the expert e whose padded
+ *     range holds row t*tile_size: tile_idx_to_group_idx[t] = e and
+ *     tile_idx_to_mn_limit[t] = padded_offsets[e] + expert_counts[e] (the
+ *     end of that expert's real rows); later tiles up to max_tiles get -1
+ *     in both;
+ *   a valid slot i of expert e with dispatched row p is on padded row
+ *     expanded_idx_to_permuted_idx[i] = padded_offsets[e] + p - expert_offsets[e]
+ *     (-1 for slots whose id was invalid);
+ *   permuted_idx_to_expanded_idx is its inverse over all max_tiles *
+ *     tile_size rows, -1 on padding rows and past the padded total.
+ *
+ *   topk_ids [T, k], expert_counts [E], expert_offsets [E+1],
+ *   output_permutation [T*k]           int32, from moe_prepare
+ *   padded_offsets [E+1], tile_idx_to_group_idx [max_tiles],
+ *   tile_idx_to_mn_limit [max_tiles], expanded_idx_to_permuted_idx [T*k],
+ *   permuted_idx_to_expanded_idx [max_tiles * tile_size],
+ *   num_non_exiting_tiles [1], total_num_padded_tokens [1]   int32 out
+ *
+ * max_tiles = ceil(T*k / tile_size) + min(E, T*k) always suffices.  When
+ * max_tiles * tile_size is smaller than the padded total (known only on the
+ * device), num_non_exiting_tiles is set to -1, total_num_padded_tokens and
+ * padded_offsets hold the needed sizes and nothing else is written.
+ */
+moe_status_t moe_tile_layout(const int32_t *topk_ids, int64_t num_tokens, int32_t top_k,
+                             int32_t num_experts, int32_t tile_size, const int32_t *expert_counts,
+                             const int32_t *expert_offsets, const int32_t *output_permutation,
+                             int32_t max_tiles, int32_t *padded_offsets,
+                             int32_t *tile_idx_to_group_idx, int32_t *tile_idx_to_mn_limit,
+                             int32_t *expanded_idx_to_permuted_idx,
+                             int32_t *permuted_idx_to_expanded_idx,
+                             int32_t *num_non_exiting_tiles, int32_t *total_num_padded_tokens,
+                             moe_stream_t stream);
+
 /* Size of the device array that moe_prepare_no_alloc uses as scratch. */
 #define MOE_PREPARE_NO_ALLOC_SCRATCH_BYTES ((size_t)4 << 20)
 
