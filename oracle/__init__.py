@@ -33,7 +33,8 @@ from .build import build_oracle, oracle_lib_path
 
 __all__ = [
     "F32", "F16", "BF16", "lib", "prepare", "dispatch", "dispatch_fp8",
-    "combine", "brute_prepare", "problem_sizes", "tile_layout", "f32_to_bf16", "f32_to_f16", "f16_to_f32",
+    "combine", "brute_prepare", "problem_sizes", "tile_layout", "prepare_local",
+    "output_memset", "f32_to_bf16", "f32_to_f16", "f16_to_f32",
     "bf16_to_f32", "f32_to_e4m3", "e4m3_to_f32",
 ]
 
@@ -65,6 +66,11 @@ def lib():
         L.oracle_combine.restype = None
         L.oracle_combine.argtypes = [_vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
                                      ctypes.c_int32, _vp, _vp, _vp, ctypes.c_int]
+        L.oracle_prepare_local_i64.restype = ctypes.c_int64
+        L.oracle_prepare_local_i64.argtypes = [_vp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int64,
+                                               ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp]
+        L.oracle_output_memset.restype = None
+        L.oracle_output_memset.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _vp]
         L.oracle_problem_sizes.restype = None
         L.oracle_problem_sizes.argtypes = [_vp, ctypes.c_int32] + [ctypes.c_int32] * 4 + [_vp, _vp]
         L.oracle_tile_layout.restype = ctypes.c_int
@@ -156,6 +162,32 @@ def combine(y_bits: np.ndarray, y_dtype: str, output_perm: np.ndarray, w: np.nda
     out = np.zeros((T, H), np.float32 if out_dtype == "fp32" else np.uint16)
     lib().oracle_combine(_ptr(y_bits), _DT[y_dtype], T, H, k, _ptr(output_perm), _ptr(w),
                          _ptr(out), _DT[out_dtype])
+    return out
+
+
+def prepare_local(ids: np.ndarray, base: int, E: int, block_align: int = 1):
+    """Routing metadata of the experts [base, base + E) from int64 ids [T,k];
+    slots outside the window are excluded like invalid ids."""
+    ids = np.ascontiguousarray(ids, dtype=np.int64)
+    T, k = ids.shape
+    S = T * k
+    counts = np.zeros(E, np.int32)
+    offsets = np.zeros(E + 1, np.int32)
+    bso = np.zeros(E + 1, np.int32)
+    inp = np.zeros(S, np.int32)
+    outp = np.zeros(S, np.int32)
+    n_bad = lib().oracle_prepare_local_i64(_ptr(ids), T, k, base, E, block_align, _ptr(counts),
+                                           _ptr(offsets), _ptr(bso), _ptr(inp), _ptr(outp))
+    return dict(counts=counts, offsets=offsets, bso=bso, input_perm=inp, output_perm=outp,
+                n_invalid=int(n_bad))
+
+
+def output_memset(out: np.ndarray, output_perm: np.ndarray, k: int):
+    """Zero (in place) the rows of tokens with at least one routed slot."""
+    assert out.flags["C_CONTIGUOUS"]
+    output_perm = np.ascontiguousarray(output_perm, dtype=np.int32)
+    T = out.shape[0]
+    lib().oracle_output_memset(_ptr(out), out.nbytes // max(T, 1), T, k, _ptr(output_perm))
     return out
 
 

@@ -463,3 +463,66 @@ int oracle_tile_layout(const int32_t *ids, int64_t T, int32_t k, int32_t E, int3
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* One rank's window of experts, int64 ids, output memset.             */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Routing metadata for the experts [base, base + E) of one rank, from int64
+ * ids (Mooncake's top-k index type): slot i belongs to local expert
+ * ids[i] - base when that lies in [0, E); every other slot is excluded
+ * exactly as an invalid id is.  Written out directly, without calling
+ * oracle_prepare: the same per-expert scan over the slots.
+ */
+int64_t oracle_prepare_local_i64(const int64_t *ids, int64_t T, int32_t k, int64_t base, int32_t E,
+                                 int32_t A, int32_t *counts, int32_t *offsets, int32_t *bso,
+                                 int32_t *input_perm, int32_t *output_perm)
+{
+    int64_t S = T * (int64_t)k;
+    for (int64_t i = 0; i < S; ++i) {
+        output_perm[i] = -1;
+        input_perm[i] = -1;
+    }
+    int64_t p = 0;
+    for (int32_t e = 0; e < E; ++e) {
+        int32_t c = 0;
+        for (int64_t i = 0; i < S; ++i) {
+            if (ids[i] - base == (int64_t)e) {
+                input_perm[p] = (int32_t)i;
+                output_perm[i] = (int32_t)p;
+                ++p;
+                ++c;
+            }
+        }
+        counts[e] = c;
+    }
+    offsets[0] = 0;
+    for (int32_t e = 0; e < E; ++e)
+        offsets[e + 1] = offsets[e] + counts[e];
+    if (bso) {
+        bso[0] = 0;
+        for (int32_t e = 0; e < E; ++e)
+            bso[e + 1] = bso[e] + (counts[e] + A - 1) / A * A;
+    }
+    return S - p;
+}
+
+/*
+ * Output memset (TensorRT-LLM PR #9592, moe_output_memset_inplace): zero the
+ * output row of every token that has at least one slot with a dispatched
+ * row (output_perm >= 0); every other row is left unchanged.
+ */
+void oracle_output_memset(void *out, int64_t row_bytes, int64_t T, int32_t k,
+                          const int32_t *output_perm)
+{
+    unsigned char *o = (unsigned char *)out;
+    for (int64_t t = 0; t < T; ++t) {
+        int routed = 0;
+        for (int32_t j = 0; j < k; ++j)
+            if (output_perm[t * k + j] >= 0)
+                routed = 1;
+        if (routed)
+            memset(o + t * row_bytes, 0, (size_t)row_bytes);
+    }
+}

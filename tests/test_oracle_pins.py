@@ -431,3 +431,47 @@ def test_tile_layout_invariants(name, tile):
     e = flat[valid]
     assert (rows >= L["padded_offsets"][e]).all() and (rows < L["padded_offsets"][e] + m["counts"][e]).all()
     np.testing.assert_array_equal(rows - L["padded_offsets"][e], m["output_perm"][valid] - m["offsets"][e])
+
+
+# ---------------------------------------------------------------------------
+# one rank's expert window, int64 ids, output memset
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("base,E", [(0, 256), (64, 32), (250, 16), (2**33, 40)])
+def test_prepare_local_equals_prepare_of_shifted_ids(base, E):
+    """The window [base, base+E) over int64 ids is prepare of ids - base with
+    every id outside the window made invalid (a different code path)."""
+    w = CONFIGS["uniform_t4096_h7168_e256_k8"].scaled(700)
+    ids32, _, _, _ = make_workload(w, with_x=False, with_y=False)
+    ids = ids32.astype(np.int64) + (base - 64 if base >= 64 else 0)
+    m = oracle.prepare_local(ids, base, E, 8)
+    shifted = ids - base
+    shifted[(shifted < 0) | (shifted >= E)] = -1
+    r = oracle.prepare(shifted.astype(np.int32), E, 8)
+    for key in ("counts", "offsets", "bso", "input_perm", "output_perm", "n_invalid"):
+        np.testing.assert_array_equal(m[key], r[key])
+
+
+def test_prepare_local_hand_worked_example():
+    # window [10, 13): ids 10, 12 local (experts 0 and 2); 9, 13, -1 not local
+    ids = np.array([[12, 9], [10, 13], [12, -1]], np.int64)
+    m = oracle.prepare_local(ids, 10, 3)
+    assert m["counts"].tolist() == [1, 0, 2]
+    assert m["offsets"].tolist() == [0, 1, 1, 3]
+    assert m["input_perm"].tolist() == [2, 0, 4, -1, -1, -1]
+    assert m["output_perm"].tolist() == [1, -1, 0, -1, 2, -1]
+    assert m["n_invalid"] == 3
+
+
+def test_output_memset_zeroes_exactly_the_routed_tokens():
+    rng = np.random.default_rng(4)
+    T, k, H = 50, 4, 24
+    out_perm = rng.integers(0, 10, size=T * k).astype(np.int32)
+    out_perm[rng.random(T * k) < 0.6] = -1
+    out = rng.standard_normal((T, H)).astype(np.float32)
+    before = out.copy()
+    oracle.output_memset(out, out_perm, k)
+    routed = (out_perm.reshape(T, k) >= 0).any(axis=1)
+    assert (out[routed] == 0).all()
+    np.testing.assert_array_equal(out[~routed], before[~routed])
+    assert routed.any() and (~routed).any()
