@@ -299,7 +299,7 @@ class Step:
 
     def dispatch(self, meta):
         if self.fp8:
-            self.moe.moe_dispatch_rows_fp8(self.x, self.ids, meta.output_permutation,
+            self.moe.moe_dispatch_rows_fp8(self.x, self.w.k, meta.output_permutation,
                                            meta.expert_offsets, meta.blockscale_offsets,
                                            blockscale_align=self.A, out_q=self.xq,
                                            out_scales=self.scales)
@@ -553,7 +553,7 @@ def time_next_rows(step, w, dev, reps=20):
         torch.cuda.synchronize(dev)
         return s.elapsed_time(e) / reps * 1e3
 
-    us = timed(lambda: moe.moe_tile_layout(step.ids, meta, tile, max_tiles))
+    us = timed(lambda: moe.moe_tile_layout(meta, w.k, tile, max_tiles))
     b = 8 * S + 8 * E + 4 * (E + 1) + 8 * max_tiles + 4 * S + 4 * max_tiles * tile + 8
     out["tile_layout_t128"] = {"us": us, "algorithmic_bytes": b, "effective_gbs": b / us / 1e3}
     us = timed(lambda: moe.moe_problem_sizes(meta.expert_counts, 2 * w.H, w.H, w.H, w.H))

@@ -33,6 +33,8 @@ __all__ = [
     "moe_version",
     "moe_problem_sizes",
     "moe_tile_layout",
+    "moe_prepare_local",
+    "moe_output_memset",
     "TileLayout",
     "library_path",
 ]
@@ -198,7 +200,7 @@ def moe_dispatch_rows(x: torch.Tensor, top_k: int, input_permutation: Optional[t
     return out
 
 
-def moe_dispatch_rows_fp8(x: torch.Tensor, topk_ids: torch.Tensor, output_permutation: torch.Tensor,
+def moe_dispatch_rows_fp8(x: torch.Tensor, top_k: int, output_permutation: torch.Tensor,
                           expert_offsets: torch.Tensor, blockscale_offsets: torch.Tensor, *,
                           blockscale_align: int = 1, out_q: Optional[torch.Tensor] = None,
                           out_scales: Optional[torch.Tensor] = None):
@@ -209,13 +211,11 @@ def moe_dispatch_rows_fp8(x: torch.Tensor, topk_ids: torch.Tensor, output_permut
     T*k + E*(blockscale_align - 1) rows (no device-to-host read).
     """
     _need(x, "x")
-    _need(topk_ids, "topk_ids", torch.int32)
     T, H = x.shape
-    k = topk_ids.shape[1]
+    k = top_k
     E = expert_offsets.numel() - 1
     S = T * k
     dev = x.device
-    _need(topk_ids, "topk_ids", torch.int32, (T, k), dev)
     _need(output_permutation, "output_permutation", torch.int32, (S,), dev)
     _need(expert_offsets, "expert_offsets", torch.int32, (E + 1,), dev)
     _need(blockscale_offsets, "blockscale_offsets", torch.int32, (E + 1,), dev)
@@ -232,9 +232,9 @@ def moe_dispatch_rows_fp8(x: torch.Tensor, topk_ids: torch.Tensor, output_permut
     _need(out_scales, "out_scales", torch.float32, None, dev)
     with torch.cuda.device(dev):
         st = _lib.load().moe_dispatch_rows_fp8(
-            x.data_ptr(), _dtype_code(x.dtype), T, H, k, E, topk_ids.data_ptr(),
-            output_permutation.data_ptr(), expert_offsets.data_ptr(),
-            blockscale_offsets.data_ptr(), out_q.data_ptr(), out_scales.data_ptr(), _stream(dev))
+            x.data_ptr(), _dtype_code(x.dtype), T, H, k, E, output_permutation.data_ptr(),
+            expert_offsets.data_ptr(), blockscale_offsets.data_ptr(), out_q.data_ptr(),
+            out_scales.data_ptr(), _stream(dev))
     _lib.check("moe_dispatch_rows_fp8", st)
     return out_q, out_scales
 
@@ -307,16 +307,15 @@ def moe_problem_sizes(expert_counts: torch.Tensor, n1: int, k1: int, n2: int, k2
     return ps1, ps2
 
 
-def moe_tile_layout(topk_ids: torch.Tensor, meta: PrepareResult, tile_size: int,
+def moe_tile_layout(meta: PrepareResult, top_k: int, tile_size: int,
                     max_tiles: Optional[int] = None) -> TileLayout:
     """Tile-padded grouped-GEMM layout from moe_prepare's results (see
     include/moe.h).  Without ``max_tiles`` the always-sufficient bound
     ceil(T*k / tile) + min(E, T*k) is used."""
-    _need(topk_ids, "topk_ids", torch.int32)
-    T, k = topk_ids.shape
     E = meta.expert_counts.numel()
-    S = T * k
-    dev = topk_ids.device
+    S = meta.output_permutation.numel()
+    T = S // top_k
+    dev = meta.expert_counts.device
     if max_tiles is None:
         max_tiles = max(1, -(-S // tile_size) + min(E, S))
     i32 = dict(dtype=torch.int32, device=dev)
@@ -326,8 +325,50 @@ def moe_tile_layout(topk_ids: torch.Tensor, meta: PrepareResult, tile_size: int,
                      torch.empty(1, **i32))
     with torch.cuda.device(dev):
         st = _lib.load().moe_tile_layout(
-            topk_ids.data_ptr(), T, k, E, tile_size, meta.expert_counts.data_ptr(),
-            meta.expert_offsets.data_ptr(), _ptr(meta.output_permutation) if S else None,
-            max_tiles, *[_ptr(t) if t.numel() else None for t in out], _stream(dev))
+            T, top_k, E, tile_size, meta.expert_counts.data_ptr(), meta.expert_offsets.data_ptr(),
+            _ptr(meta.output_permutation) if S else None, max_tiles,
+            *[_ptr(t) if t.numel() else None for t in out], _stream(dev))
     _lib.check("moe_tile_layout", st)
+    return out
+
+
+def moe_prepare_local(topk_ids: torch.Tensor, local_expert_offset: int, num_local_experts: int, *,
+                      blockscale_align: Optional[int] = None,
+                      workspace: Optional[torch.Tensor] = None) -> PrepareResult:
+    """Routing metadata of one rank's experts [offset, offset + n) from int32
+    or int64 ids [T, k]; other slots are excluded (see include/moe.h)."""
+    if topk_ids.dtype not in (torch.int32, torch.int64):
+        raise ValueError("topk_ids must be int32 or int64")
+    _need(topk_ids, "topk_ids")
+    T, k = topk_ids.shape
+    E = num_local_experts
+    dev = topk_ids.device
+    with torch.cuda.device(dev):
+        meta = _alloc_meta(dev, T * k, E, blockscale_align is not None, None, None, None, None,
+                           None, None)
+        need = moe_prepare_workspace_bytes(T, k, E) if T * k > 0 else 0
+        if workspace is None:
+            workspace = _workspace(dev, need)
+        ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        id_type = _lib.MOE_I64 if topk_ids.dtype == torch.int64 else _lib.MOE_I32
+        st = _lib.load().moe_prepare_local(
+            _ptr(topk_ids) if T * k else None, id_type, T, k, local_expert_offset, E,
+            meta.expert_counts.data_ptr(), meta.expert_offsets.data_ptr(),
+            _ptr(meta.blockscale_offsets), blockscale_align or 1,
+            _ptr(meta.input_permutation) if T * k else None,
+            _ptr(meta.output_permutation) if T * k else None, meta.diag.data_ptr(),
+            _ptr(workspace), ws_bytes, _stream(dev))
+    _lib.check("moe_prepare_local", st)
+    return meta
+
+
+def moe_output_memset(out: torch.Tensor, output_permutation: torch.Tensor, top_k: int) -> torch.Tensor:
+    """Zero (in place) the rows of tokens with at least one routed slot."""
+    _need(out, "out")
+    T, H = out.shape
+    _need(output_permutation, "output_permutation", torch.int32, (T * top_k,), out.device)
+    with torch.cuda.device(out.device):
+        st = _lib.load().moe_output_memset(out.data_ptr(), _dtype_code(out.dtype), T, H, top_k,
+                                           output_permutation.data_ptr(), _stream(out.device))
+    _lib.check("moe_output_memset", st)
     return out

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(PKG, "libmoe.so")
 MOE_OK = 0
 MOE_ERR_CUDA = 4
 MOE_F32, MOE_F16, MOE_BF16, MOE_FP8_E4M3 = 0, 1, 2, 3
+MOE_I32, MOE_I64 = 0, 1
 MAX_EXPERTS = 1024
 FUSED_MAX_SLOTS = 4096
 
@@ -34,6 +35,8 @@ EXPORTED = (
     "moe_prepare_no_alloc",
     "moe_problem_sizes",
     "moe_tile_layout",
+    "moe_prepare_local",
+    "moe_output_memset",
 )
 
 _vp = ctypes.c_void_p
@@ -49,7 +52,7 @@ _SIGNATURES = {
     "moe_prepare": (_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp,
                            ctypes.c_size_t, _vp]),
     "moe_dispatch_rows": (_int, [_vp, _int, _i64, _i64, _i32, _vp, _vp, _vp, _vp]),
-    "moe_dispatch_rows_fp8": (_int, [_vp, _int, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp, _vp,
+    "moe_dispatch_rows_fp8": (_int, [_vp, _int, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp,
                                      _vp, _vp]),
     "moe_combine": (_int, [_vp, _int, _i64, _i64, _i32, _vp, _vp, _vp, _int, _vp]),
     "moe_prepare_dispatch": (_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp,
@@ -57,8 +60,11 @@ _SIGNATURES = {
     "moe_prepare_no_alloc": (_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp,
                                     _vp]),
     "moe_problem_sizes": (_int, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
-    "moe_tile_layout": (_int, [_vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp,
+    "moe_tile_layout": (_int, [_i64, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp,
                                _vp, _vp, _vp, _vp, _vp]),
+    "moe_prepare_local": (_int, [_vp, _int, _i64, _i32, _i64, _i32, _vp, _vp, _vp, _i32, _vp,
+                                 _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "moe_output_memset": (_int, [_vp, _int, _i64, _i64, _i32, _vp, _vp]),
 }
 
 _lib = None

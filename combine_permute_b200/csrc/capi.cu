@@ -82,11 +82,52 @@ moe_status_t moe_prepare(const int32_t *topk_ids, int64_t num_tokens, int32_t to
     const size_t need = moe::prepare_workspace_bytes(S, num_experts);
     if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
         return MOE_ERR_WORKSPACE;
-    return from_cuda(moe::run_prepare(topk_ids, S, num_experts,
+    return from_cuda(moe::run_prepare(topk_ids, false, 0, S, num_experts,
                                       blockscale_offsets ? blockscale_align : 1, expert_counts,
                                       expert_offsets, blockscale_offsets, input_permutation,
                                       output_permutation, diag, workspace,
                                       (cudaStream_t)stream));
+}
+
+moe_status_t moe_prepare_local(const void *topk_ids, moe_index_t id_type, int64_t num_tokens,
+                               int32_t top_k, int64_t local_expert_offset,
+                               int32_t num_local_experts, int32_t *expert_counts,
+                               int32_t *expert_offsets, int32_t *blockscale_offsets,
+                               int32_t blockscale_align, int32_t *input_permutation,
+                               int32_t *output_permutation, int32_t *diag, void *workspace,
+                               size_t workspace_bytes, moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (id_type != MOE_I32 && id_type != MOE_I64) return MOE_ERR_INVALID_ARG;
+    if (num_local_experts < 1) return MOE_ERR_INVALID_ARG;
+    if (num_local_experts > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    const int64_t S = num_tokens * (int64_t)top_k;
+    if (!expert_counts || !expert_offsets) return MOE_ERR_INVALID_ARG;
+    if (S > 0 && (!topk_ids || !input_permutation || !output_permutation))
+        return MOE_ERR_INVALID_ARG;
+    if (blockscale_offsets && blockscale_align < 1) return MOE_ERR_INVALID_ARG;
+    const size_t need = moe::prepare_workspace_bytes(S, num_local_experts);
+    if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)))
+        return MOE_ERR_WORKSPACE;
+    return from_cuda(moe::run_prepare(topk_ids, id_type == MOE_I64, local_expert_offset, S,
+                                      num_local_experts, blockscale_offsets ? blockscale_align : 1,
+                                      expert_counts, expert_offsets, blockscale_offsets,
+                                      input_permutation, output_permutation, diag, workspace,
+                                      (cudaStream_t)stream));
+}
+
+moe_status_t moe_output_memset(void *out, moe_dtype_t dtype, int64_t num_tokens, int64_t hidden,
+                               int32_t top_k, const int32_t *output_permutation,
+                               moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (!io_dtype(dtype) || hidden < 1) return MOE_ERR_INVALID_ARG;
+    const int64_t row_bytes = hidden * moe::dtype_bytes(dt(dtype));
+    if (row_bytes % 16 != 0) return MOE_ERR_INVALID_ARG;
+    if (num_tokens == 0) return MOE_OK;
+    if (!out || !output_permutation || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_output_memset(out, num_tokens, row_bytes, top_k, output_permutation,
+                                            (cudaStream_t)stream));
 }
 
 moe_status_t moe_dispatch_rows(const void *x, moe_dtype_t dtype, int64_t num_tokens,
@@ -110,7 +151,7 @@ moe_status_t moe_dispatch_rows(const void *x, moe_dtype_t dtype, int64_t num_tok
 
 moe_status_t moe_dispatch_rows_fp8(const void *x, moe_dtype_t x_dtype, int64_t num_tokens,
                                    int64_t hidden, int32_t top_k, int32_t num_experts,
-                                   const int32_t *topk_ids, const int32_t *output_permutation,
+                                   const int32_t *output_permutation,
                                    const int32_t *expert_offsets,
                                    const int32_t *blockscale_offsets, uint8_t *out_q,
                                    float *out_scales, moe_stream_t stream) {
@@ -118,16 +159,16 @@ moe_status_t moe_dispatch_rows_fp8(const void *x, moe_dtype_t x_dtype, int64_t n
     if (st != MOE_OK) return st;
     if (x_dtype != MOE_BF16 && x_dtype != MOE_F16) return MOE_ERR_UNSUPPORTED;
     if (hidden < 1 || hidden % 128 != 0 || num_experts < 1) return MOE_ERR_INVALID_ARG;
+    if (num_experts > 4 * moe::kMaxExperts || top_k > 4096) return MOE_ERR_UNSUPPORTED;
     if (num_tokens == 0) return MOE_OK;
-    if (!x || !topk_ids || !output_permutation || !expert_offsets || !blockscale_offsets ||
-        !out_q || !out_scales)
+    if (!x || !output_permutation || !expert_offsets || !blockscale_offsets || !out_q ||
+        !out_scales)
         return MOE_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(out_q) || ((uintptr_t)out_scales & 3u))
         return MOE_ERR_INVALID_ARG;
-    return from_cuda(moe::run_dispatch_fp8(x, dt(x_dtype), num_tokens, hidden, top_k, num_experts, topk_ids,
-                                           output_permutation, expert_offsets,
-                                           blockscale_offsets, out_q, out_scales,
-                                           (cudaStream_t)stream));
+    return from_cuda(moe::run_dispatch_fp8(x, dt(x_dtype), num_tokens, hidden, top_k, num_experts,
+                                           output_permutation, expert_offsets, blockscale_offsets,
+                                           out_q, out_scales, (cudaStream_t)stream));
 }
 
 moe_status_t moe_combine(const void *y, moe_dtype_t y_dtype, int64_t num_tokens, int64_t hidden,
@@ -181,8 +222,8 @@ moe_status_t moe_problem_sizes(const int32_t *expert_counts, int32_t num_experts
                                             problem_sizes1, problem_sizes2, (cudaStream_t)stream));
 }
 
-moe_status_t moe_tile_layout(const int32_t *topk_ids, int64_t num_tokens, int32_t top_k,
-                             int32_t num_experts, int32_t tile_size, const int32_t *expert_counts,
+moe_status_t moe_tile_layout(int64_t num_tokens, int32_t top_k, int32_t num_experts,
+                             int32_t tile_size, const int32_t *expert_counts,
                              const int32_t *expert_offsets, const int32_t *output_permutation,
                              int32_t max_tiles, int32_t *padded_offsets,
                              int32_t *tile_idx_to_group_idx, int32_t *tile_idx_to_mn_limit,
@@ -200,13 +241,12 @@ moe_status_t moe_tile_layout(const int32_t *topk_ids, int64_t num_tokens, int32_
         !tile_idx_to_mn_limit || !permuted_idx_to_expanded_idx || !num_non_exiting_tiles ||
         !total_num_padded_tokens)
         return MOE_ERR_INVALID_ARG;
-    if (S > 0 && (!topk_ids || !output_permutation || !expanded_idx_to_permuted_idx))
-        return MOE_ERR_INVALID_ARG;
+    if (S > 0 && (!output_permutation || !expanded_idx_to_permuted_idx)) return MOE_ERR_INVALID_ARG;
     return from_cuda(moe::run_tile_layout(
-        topk_ids, S, num_experts, tile_size, expert_counts, expert_offsets, output_permutation,
-        max_tiles, padded_offsets, tile_idx_to_group_idx, tile_idx_to_mn_limit,
-        expanded_idx_to_permuted_idx, permuted_idx_to_expanded_idx, num_non_exiting_tiles,
-        total_num_padded_tokens, (cudaStream_t)stream));
+        S, num_experts, tile_size, expert_counts, expert_offsets, output_permutation, max_tiles,
+        padded_offsets, tile_idx_to_group_idx, tile_idx_to_mn_limit, expanded_idx_to_permuted_idx,
+        permuted_idx_to_expanded_idx, num_non_exiting_tiles, total_num_padded_tokens,
+        (cudaStream_t)stream));
 }
 
 }  // extern "C"

@@ -140,13 +140,31 @@ __global__ void __launch_bounds__(kCopyThreads)
     }
 }
 
+// Output memset (TensorRT-LLM PR #9592, moe_output_memset_inplace): zero the
+// row of every token with at least one routed slot (output_permutation >= 0);
+// other rows stay as they are.  One block per token at a time.
+__global__ void __launch_bounds__(kCopyThreads)
+    output_memset_kernel(uint4 *__restrict__ out, int64_t T, int64_t nvec, int k,
+                         const int32_t *__restrict__ out_perm) {
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        bool routed = false;
+        for (int j = 0; j < k; ++j) routed |= __ldg(out_perm + t * k + j) >= 0;
+        if (!routed) continue;
+        uint4 *row = out + t * nvec;
+        for (int64_t c = threadIdx.x; c < nvec; c += kCopyThreads) st_v4(row + c, make_uint4(0, 0, 0, 0));
+    }
+}
+
 // ---------------------------------------------------------------------------
 // FP8 dispatch.  Each thread owns 16 consecutive elements of a token row (two
 // 16-byte loads); the 8 threads of one 128-column block reduce amax with
 // shuffles, divide by s = amax / 448 in IEEE fp32 and convert pairs with
 // cvt.rn.satfinite.e4m3x2.  The quantised row is computed once per token
 // and stored to its k dispatched rows; the first thread of each block also
-// stores s into the expert's scale segment.
+// stores s into the scale segment of the row's expert (found from the expert
+// offsets, so the kernel needs no ids).
 // ---------------------------------------------------------------------------
 constexpr int kFp8Threads = 256;
 
@@ -160,15 +178,43 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
 template <typename XT>
 __global__ void __launch_bounds__(kFp8Threads)
     dispatch_fp8_kernel(const XT *__restrict__ x, int64_t T, int64_t H, int k, int E,
-                        const int32_t *__restrict__ ids, const int32_t *__restrict__ out_perm,
-                        const int32_t *__restrict__ offsets, const int32_t *__restrict__ bso,
-                        uint8_t *__restrict__ q, float *__restrict__ scales) {
+                        const int32_t *__restrict__ out_perm, const int32_t *__restrict__ offsets,
+                        const int32_t *__restrict__ bso, uint8_t *__restrict__ q,
+                        float *__restrict__ scales) {
+    extern __shared__ int smem[];
+    int *s_off = smem;             // [E+1] expert offsets
+    int *s_delta = s_off + E + 1;  // [E] scale row - dispatched row, per expert
+    int *s_p = s_delta + E;        // [k] this token's dispatched rows
+    int *s_srow = s_p + k;         // [k] and their scale rows
     pdl_wait();
     pdl_launch_dependents();
+    for (int e = threadIdx.x; e <= E; e += kFp8Threads) {
+        s_off[e] = __ldg(offsets + e);
+        if (e < E) s_delta[e] = __ldg(bso + e) - __ldg(offsets + e);
+    }
     const int64_t n16 = H / 16;  // 16-element groups per row
     const int64_t nb = H / 128;
     const int64_t S = T * k;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        __syncthreads();  // offsets staged; the previous token's rows consumed
+        for (int j = threadIdx.x; j < k; j += kFp8Threads) {
+            int p = __ldg(out_perm + t * k + j);
+            int srow = -1;
+            if (p >= 0 && p < S && p < s_off[E]) {
+                int lo = 0, hi = E;  // the expert whose rows hold p
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (s_off[mid] <= p) lo = mid;
+                    else hi = mid;
+                }
+                srow = p + s_delta[lo];
+            } else {
+                p = -1;
+            }
+            s_p[j] = p;
+            s_srow[j] = srow;
+        }
+        __syncthreads();
         for (int64_t g = threadIdx.x; g < n16; g += kFp8Threads) {
             const XT *src = x + t * H + g * 16;
             float f[16];
@@ -202,16 +248,10 @@ __global__ void __launch_bounds__(kFp8Threads)
             const bool block_lead = (g & 7) == 0;
             const int64_t b = g >> 3;
             for (int j = 0; j < k; ++j) {
-                const int64_t i = t * k + j;
-                const int p = __ldg(out_perm + i);
-                if (p < 0 || p >= S) continue;
-                const int e = __ldg(ids + i);
-                if (e < 0 || e >= E) continue;
+                const int p = s_p[j];
+                if (p < 0) continue;
                 st_v4(q + (int64_t)p * H + g * 16, packed);
-                if (block_lead) {
-                    const int64_t srow = (int64_t)__ldg(bso + e) + (p - __ldg(offsets + e));
-                    scales[srow * nb + b] = s;
-                }
+                if (block_lead) scales[(int64_t)s_srow[j] * nb + b] = s;
             }
         }
     }
@@ -272,18 +312,26 @@ cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int
 }
 
 cudaError_t run_dispatch_fp8(const void *x, DType x_dtype, int64_t T, int64_t H, int k, int E,
-                             const int32_t *ids, const int32_t *out_perm, const int32_t *offsets,
-                             const int32_t *bso, uint8_t *q, float *scales, cudaStream_t stream) {
+                             const int32_t *out_perm, const int32_t *offsets, const int32_t *bso,
+                             uint8_t *q, float *scales, cudaStream_t stream) {
+    const size_t smem = (size_t)(2 * E + 1 + 2 * k) * sizeof(int);
     if (x_dtype == DType::BF16) {
         auto kern = dispatch_fp8_kernel<__nv_bfloat16>;
-        const int64_t grid = persistent_grid(kern, kFp8Threads, 0, T);
-        return launch(kern, grid, kFp8Threads, 0, stream, (const __nv_bfloat16 *)x, T, H, k, E, ids,
+        const int64_t grid = persistent_grid(kern, kFp8Threads, smem, T);
+        return launch(kern, grid, kFp8Threads, smem, stream, (const __nv_bfloat16 *)x, T, H, k, E,
                       out_perm, offsets, bso, q, scales);
     }
     auto kern = dispatch_fp8_kernel<__half>;
-    const int64_t grid = persistent_grid(kern, kFp8Threads, 0, T);
-    return launch(kern, grid, kFp8Threads, 0, stream, (const __half *)x, T, H, k, E, ids, out_perm,
+    const int64_t grid = persistent_grid(kern, kFp8Threads, smem, T);
+    return launch(kern, grid, kFp8Threads, smem, stream, (const __half *)x, T, H, k, E, out_perm,
                   offsets, bso, q, scales);
+}
+
+cudaError_t run_output_memset(void *out, int64_t T, int64_t row_bytes, int k,
+                              const int32_t *out_perm, cudaStream_t stream) {
+    const int64_t grid = persistent_grid(output_memset_kernel, kCopyThreads, 0, T);
+    return launch(output_memset_kernel, grid, kCopyThreads, 0, stream, (uint4 *)out, T,
+                  row_bytes / 16, k, out_perm);
 }
 
 }  // namespace moe

@@ -25,9 +25,11 @@ constexpr int kFusedMaxSlots = 4096;
 
 size_t prepare_workspace_bytes(int64_t S, int E);
 
-cudaError_t run_prepare(const int32_t *ids, int64_t S, int E, int A, int32_t *counts,
-                        int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,
-                        int32_t *diag, void *workspace, cudaStream_t stream);
+// ids are int32 (ids64 false) or int64; slot i's expert is ids[i] - base when
+// that lies in [0, E), else the slot is excluded like an invalid id.
+cudaError_t run_prepare(const void *ids, bool ids64, int64_t base, int64_t S, int E, int A,
+                        int32_t *counts, int32_t *offsets, int32_t *bso, int32_t *in_perm,
+                        int32_t *out_perm, int32_t *diag, void *workspace, cudaStream_t stream);
 
 cudaError_t run_prepare_dispatch(const int32_t *ids, int64_t T, int k, int E, int A,
                                  int32_t *counts, int32_t *offsets, int32_t *bso,
@@ -47,13 +49,11 @@ cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int
                                 const int32_t *in_perm, void *out, cudaStream_t stream);
 
 cudaError_t run_dispatch_fp8(const void *x, DType x_dtype, int64_t T, int64_t H, int k, int E,
-                             const int32_t *ids, const int32_t *out_perm, const int32_t *offsets,
-                             const int32_t *bso, uint8_t *q, float *scales, cudaStream_t stream);
+                             const int32_t *out_perm, const int32_t *offsets, const int32_t *bso,
+                             uint8_t *q, float *scales, cudaStream_t stream);
 
-// The same with an explicit column split per row (0 = chosen for balance).
-cudaError_t run_combine_split(const void *y, DType y_dtype, int64_t T, int64_t H, int k,
-                              const int32_t *out_perm, const float *w, void *out,
-                              DType out_dtype, int64_t nsplit, cudaStream_t stream);
+cudaError_t run_output_memset(void *out, int64_t T, int64_t row_bytes, int k,
+                              const int32_t *out_perm, cudaStream_t stream);
 
 cudaError_t run_combine(const void *y, DType y_dtype, int64_t T, int64_t H, int k,
                         const int32_t *out_perm, const float *w, void *out, DType out_dtype,
@@ -62,7 +62,7 @@ cudaError_t run_combine(const void *y, DType y_dtype, int64_t T, int64_t H, int 
 cudaError_t run_problem_sizes(const int32_t *counts, int E, int n1, int k1, int n2, int k2,
                               int32_t *ps1, int32_t *ps2, cudaStream_t stream);
 
-cudaError_t run_tile_layout(const int32_t *ids, int64_t S, int E, int tile, const int32_t *counts,
+cudaError_t run_tile_layout(int64_t S, int E, int tile, const int32_t *counts,
                             const int32_t *offsets, const int32_t *out_perm, int max_tiles,
                             int32_t *padded_offsets, int32_t *tile_group, int32_t *tile_limit,
                             int32_t *exp2perm, int32_t *perm2exp, int32_t *num_tiles,

@@ -9,8 +9,9 @@
 // tile_layout_kernel is one grid-stride pass: every block turns the E counts
 // into padded offsets in shared memory (a block-wide scan of the counts
 // rounded up to the tile), then the grid writes the tile owners and row
-// limits, the padded row of every valid slot and its inverse, and -1 on
-// padding rows.  The valid rows and the padding rows are disjoint, so the
+// limits, the padded row of every valid slot (its expert found from the
+// expert offsets, so any id type or expert window works) and its inverse,
+// and -1 on padding rows.  The valid rows and the padding rows are disjoint, so the
 // writes never race.
 #include "kernels.h"
 #include "launch.h"
@@ -52,8 +53,19 @@ __device__ __forceinline__ int owner_of(const int *poff, int E, int64_t row) {
     return lo;
 }
 
+// The same search over the unpadded offsets (off[e] <= p < off[e] + cnt[e]).
+__device__ __forceinline__ int owner_of_rows(const int *off, int E, int p) {
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (off[mid] <= p) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
 __global__ void __launch_bounds__(kLayoutThreads)
-    tile_layout_kernel(const int32_t *__restrict__ ids, int64_t S, int E, int tile,
+    tile_layout_kernel(int64_t S, int E, int tile,
                        const int32_t *__restrict__ counts, const int32_t *__restrict__ offsets,
                        const int32_t *__restrict__ out_perm, int max_tiles,
                        int32_t *padded_offsets, int32_t *tile_group, int32_t *tile_limit,
@@ -101,11 +113,13 @@ __global__ void __launch_bounds__(kLayoutThreads)
             tile_limit[t] = -1;
         }
     }
+    const int nvalid = E > 0 ? off[E - 1] + cnt[E - 1] : 0;
     for (int64_t i = g; i < S; i += stride) {
-        const int id = __ldg(ids + i);
+        const int p = __ldg(out_perm + i);
         int pp = -1;
-        if (id >= 0 && id < E) {
-            pp = poff[id] + (__ldg(out_perm + i) - off[id]);
+        if (p >= 0 && p < nvalid) {  // the slot's expert owns dispatched row p
+            const int e = owner_of_rows(off, E, p);
+            pp = poff[e] + (p - off[e]);
             if (pp >= 0 && pp < capacity) perm2exp[pp] = (int)i;
         }
         exp2perm[i] = pp;
@@ -129,7 +143,7 @@ cudaError_t run_problem_sizes(const int32_t *counts, int E, int n1, int k1, int 
                   ps1, ps2);
 }
 
-cudaError_t run_tile_layout(const int32_t *ids, int64_t S, int E, int tile, const int32_t *counts,
+cudaError_t run_tile_layout(int64_t S, int E, int tile, const int32_t *counts,
                             const int32_t *offsets, const int32_t *out_perm, int max_tiles,
                             int32_t *padded_offsets, int32_t *tile_group, int32_t *tile_limit,
                             int32_t *exp2perm, int32_t *perm2exp, int32_t *num_tiles,
@@ -139,7 +153,7 @@ cudaError_t run_tile_layout(const int32_t *ids, int64_t S, int E, int tile, cons
     if (S > work) work = S;
     const int64_t grid =
         persistent_grid(tile_layout_kernel, kLayoutThreads, smem, (work + kLayoutThreads - 1) / kLayoutThreads);
-    return launch(tile_layout_kernel, grid, kLayoutThreads, smem, stream, ids, S, E, tile, counts,
+    return launch(tile_layout_kernel, grid, kLayoutThreads, smem, stream, S, E, tile, counts,
                   offsets, out_perm, max_tiles, padded_offsets, tile_group, tile_limit, exp2perm,
                   perm2exp, num_tiles, total_padded);
 }

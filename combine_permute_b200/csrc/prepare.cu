@@ -78,12 +78,14 @@ __device__ __forceinline__ int rank_round(int e, int E, int nbits, int *row, uns
     return e >= 0 ? base + __popc(grp & lt) : -1;
 }
 
-// Expert of slot i, -1 for an id outside [0, E), -2 past `end`.
-__device__ __forceinline__ int load_key(const int32_t *__restrict__ ids, int64_t i, int64_t end,
-                                        int E) {
+// Expert of slot i (its id minus `base`), -1 for an id outside the window
+// [base, base + E), -2 past `end`.  Ids are int32 or int64.
+template <typename IdT>
+__device__ __forceinline__ int load_key(const IdT *__restrict__ ids, int64_t i, int64_t end,
+                                        int64_t base, int E) {
     if (i >= end) return -2;
-    const int id = __ldg(ids + i);
-    return (id >= 0 && id < E) ? id : -1;
+    const int64_t id = (int64_t)__ldg(ids + i) - base;
+    return (id >= 0 && id < E) ? (int)id : -1;
 }
 
 // Per-warp counts wcnt[w][e] (NW warps, row stride E+1 so that the lanes
@@ -185,8 +187,9 @@ __device__ __forceinline__ unsigned long long lb_flag(unsigned long long w, unsi
 // (shared memory, S entries); global outputs are written when `write` is
 // set.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void single_block_prepare(const int32_t *__restrict__ ids, int64_t S,
-                                                     int E, int A, int *smem, int *pos,
+template <typename IdT>
+__device__ __forceinline__ void single_block_prepare(const IdT *__restrict__ ids, int64_t base,
+                                                     int64_t S, int E, int A, int *smem, int *pos,
                                                      bool write, int32_t *counts,
                                                      int32_t *offsets, int32_t *bso,
                                                      int32_t *in_perm, int32_t *out_perm,
@@ -205,7 +208,8 @@ __device__ __forceinline__ void single_block_prepare(const int32_t *__restrict__
     int key[kSingleRounds];
     const int64_t wbase = (int64_t)warp * 32 * kSingleRounds;
 #pragma unroll
-    for (int r = 0; r < kSingleRounds; ++r) key[r] = load_key(ids, wbase + r * 32 + lane, S, E);
+    for (int r = 0; r < kSingleRounds; ++r)
+        key[r] = load_key(ids, wbase + r * 32 + lane, S, base, E);
     __syncthreads();
 
     int rank[kSingleRounds];
@@ -246,14 +250,16 @@ __device__ __forceinline__ void single_block_prepare(const int32_t *__restrict__
         for (int64_t p = total + tid; p < S; p += kSingleThreads) in_perm[p] = -1;
 }
 
+template <typename IdT>
 __global__ void __launch_bounds__(kSingleThreads, 1)
-    prep_single_kernel(const int32_t *__restrict__ ids, int64_t S, int E, int A, int32_t *counts,
+    prep_single_kernel(const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int A,
+                       int32_t *counts,
                        int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,
                        int32_t *diag) {
     extern __shared__ int smem[];
     pdl_wait();
     pdl_launch_dependents();
-    single_block_prepare(ids, S, E, A, smem, nullptr, true, counts, offsets, bso, in_perm,
+    single_block_prepare(ids, base, S, E, A, smem, nullptr, true, counts, offsets, bso, in_perm,
                          out_perm, diag);
 }
 
@@ -273,8 +279,9 @@ struct TileCtx {
     int64_t wbase;  // first slot of this warp's run
 };
 
+template <typename IdT>
 __device__ __forceinline__ TileCtx tile_rank_lookback(
-    const int32_t *__restrict__ ids, int64_t S, int E, int G, const PrepWs &ws, int *wcnt,
+    const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int G, const PrepWs &ws, int *wcnt,
     int *hist, int *excl, unsigned *s_misc, int *s_invalid, int (&key)[kTileRounds],
     int (&rank)[kTileRounds]) {
     const int C = E + 1;  // one column per expert plus one for invalid ids
@@ -299,7 +306,8 @@ __device__ __forceinline__ TileCtx tile_rank_lookback(
 
     // ranks within each warp's run, per-warp counts
 #pragma unroll
-    for (int r = 0; r < kTileRounds; ++r) key[r] = load_key(ids, ctx.wbase + r * 32 + lane, S, E);
+    for (int r = 0; r < kTileRounds; ++r)
+        key[r] = load_key(ids, ctx.wbase + r * 32 + lane, S, base, E);
     int *row = wcnt + warp * C;
     int bad = 0;
 #pragma unroll
@@ -380,8 +388,9 @@ size_t tile_smem(int E) { return (size_t)(kTileWarps + 4) * (E + 1) * sizeof(int
 // last tile turns the totals into offsets, writes them and raises `ready`;
 // every tile waits for it (bounded), then writes its slots' final rows into
 // both permutations.
+template <typename IdT>
 __global__ void __launch_bounds__(kTileThreads, 2)
-    prep_onepass_kernel(const int32_t *__restrict__ ids, int64_t S, int E, int A, int G,
+    prep_onepass_kernel(const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int A, int G,
                         void *workspace, int32_t *counts, int32_t *offsets, int32_t *bso,
                         int32_t *in_perm, int32_t *out_perm, int32_t *diag) {
     extern __shared__ int smem[];
@@ -400,7 +409,7 @@ __global__ void __launch_bounds__(kTileThreads, 2)
     pdl_launch_dependents();
     int key[kTileRounds], rank[kTileRounds];
     const TileCtx ctx =
-        tile_rank_lookback(ids, S, E, G, ws, wcnt, hist, excl, s_misc, &s_invalid, key, rank);
+        tile_rank_lookback(ids, base, S, E, G, ws, wcnt, hist, excl, s_misc, &s_invalid, key, rank);
     if (ctx.tile == G - 1) {
         // totals = earlier tiles + this one; offsets out, then release the others
         for (int c = tid; c < C; c += kTileThreads) off[c] = excl[c] + hist[c];
@@ -440,9 +449,9 @@ __global__ void __launch_bounds__(kTileThreads, 2)
             if (p >= 0 && p < S) in_perm[p] = (int)i;
         }
     }
-    const int64_t base = (int64_t)ctx.tile * kTileSlots;
-    const int64_t lo = base > total ? base : (int64_t)total;
-    const int64_t hi = base + kTileSlots < S ? base + kTileSlots : S;
+    const int64_t first = (int64_t)ctx.tile * kTileSlots;
+    const int64_t lo = first > total ? first : (int64_t)total;
+    const int64_t hi = first + kTileSlots < S ? first + kTileSlots : S;
     for (int64_t p = lo + tid; p < hi; p += kTileThreads) in_perm[p] = -1;
     tile_finish(ws, G, ctx.epoch, diag);
 }
@@ -450,8 +459,9 @@ __global__ void __launch_bounds__(kTileThreads, 2)
 // Two-kernel variant, kernel 1 (any number of tiles): store rank(i) in
 // output_permutation (-1 for an invalid id); the last tile writes counts,
 // offsets and block-scale offsets.
+template <typename IdT>
 __global__ void __launch_bounds__(kTileThreads, 2)
-    prep_rank_kernel(const int32_t *__restrict__ ids, int64_t S, int E, int A, int G,
+    prep_rank_kernel(const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int A, int G,
                      void *workspace, int32_t *counts, int32_t *offsets, int32_t *bso,
                      int32_t *out_perm, int32_t *diag) {
     extern __shared__ int smem[];
@@ -470,7 +480,7 @@ __global__ void __launch_bounds__(kTileThreads, 2)
     pdl_launch_dependents();
     int key[kTileRounds], rank[kTileRounds];
     const TileCtx ctx =
-        tile_rank_lookback(ids, S, E, G, ws, wcnt, hist, excl, s_misc, &s_invalid, key, rank);
+        tile_rank_lookback(ids, base, S, E, G, ws, wcnt, hist, excl, s_misc, &s_invalid, key, rank);
     const int *row = wcnt + warp * C;
 #pragma unroll
     for (int r = 0; r < kTileRounds; ++r) {
@@ -491,17 +501,18 @@ __global__ void __launch_bounds__(kTileThreads, 2)
 
 // Two-kernel variant, kernel 2 (element-wise): row = expert offset + rank;
 // both permutations.
+template <typename IdT>
 __global__ void __launch_bounds__(256)
-    prep_finish_kernel(const int32_t *__restrict__ ids, int64_t S, int E,
+    prep_finish_kernel(const IdT *__restrict__ ids, int64_t base, int64_t S, int E,
                        const int32_t *__restrict__ offsets, int32_t *in_perm, int32_t *out_perm) {
     pdl_wait();
     pdl_launch_dependents();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     for (int64_t i = g; i < S; i += stride) {
-        const int id = __ldg(ids + i);
-        if (id >= 0 && id < E) {
-            const int p = __ldg(offsets + id) + out_perm[i];
+        const int e = load_key(ids, i, S, base, E);
+        if (e >= 0) {
+            const int p = __ldg(offsets + e) + out_perm[i];
             out_perm[i] = p;
             if (p >= 0 && p < S) in_perm[p] = (int)i;
         }
@@ -524,8 +535,8 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
     int *pos = smem + kSingleWarps * (E + 1) + 2 * E;  // [S]
     pdl_wait();
     pdl_launch_dependents();
-    single_block_prepare(ids, S, E, A, smem, pos, blockIdx.x == 0, counts, offsets, bso, in_perm,
-                         out_perm, diag);
+    single_block_prepare(ids, (int64_t)0, S, E, A, smem, pos, blockIdx.x == 0, counts, offsets,
+                         bso, in_perm, out_perm, diag);
     __syncthreads();
     const int64_t total = T * nvec;
     for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
@@ -552,13 +563,16 @@ namespace {
 // One cooperative launch of prep_onepass_kernel when every tile fits on the
 // GPU at once; returns cudaErrorCooperativeLaunchTooLarge (nothing launched)
 // when the tiles do not fit or the launch form is refused.
-cudaError_t launch_onepass(const int32_t *ids, int64_t S, int E, int A, int G, void *workspace,
-                           int32_t *counts, int32_t *offsets, int32_t *bso, int32_t *in_perm,
-                           int32_t *out_perm, int32_t *diag, cudaStream_t stream) {
+template <typename IdT>
+cudaError_t launch_onepass(const IdT *ids, int64_t base, int64_t S, int E, int A, int G,
+                           void *workspace, int32_t *counts, int32_t *offsets, int32_t *bso,
+                           int32_t *in_perm, int32_t *out_perm, int32_t *diag,
+                           cudaStream_t stream) {
+    auto kern = prep_onepass_kernel<IdT>;
     const size_t smem = tile_smem(E);
-    const int64_t resident = (int64_t)sm_count() * blocks_per_sm(prep_onepass_kernel, kTileThreads, smem);
+    const int64_t resident = (int64_t)sm_count() * blocks_per_sm(kern, kTileThreads, smem);
     if (G > resident) return cudaErrorCooperativeLaunchTooLarge;
-    cudaError_t se = ensure_smem(prep_onepass_kernel, smem);
+    cudaError_t se = ensure_smem(kern, smem);
     if (se != cudaSuccess) return se;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)G, 1, 1);
@@ -573,32 +587,43 @@ cudaError_t launch_onepass(const int32_t *ids, int64_t S, int E, int A, int G, v
     cfg.attrs = attr;
     for (int n : {2, 1}) {  // with programmatic serialization if allowed, else without
         cfg.numAttrs = n;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, prep_onepass_kernel, ids, S, E, A, G, workspace,
-                                           counts, offsets, bso, in_perm, out_perm, diag);
+        cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ids, base, S, E, A, G, workspace, counts,
+                                           offsets, bso, in_perm, out_perm, diag);
         if (e == cudaSuccess) return cudaGetLastError();
         cudaGetLastError();
     }
     return cudaErrorCooperativeLaunchTooLarge;
 }
 
+template <typename IdT>
+cudaError_t run_prepare_t(const IdT *ids, int64_t base, int64_t S, int E, int A, int32_t *counts,
+                          int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,
+                          int32_t *diag, void *workspace, cudaStream_t stream) {
+    if (S <= kSingleBlockSlots)
+        return launch(prep_single_kernel<IdT>, 1, kSingleThreads, single_block_smem(E), stream, ids,
+                      base, S, E, A, counts, offsets, bso, in_perm, out_perm, diag);
+    const int G = (int)((S + kTileSlots - 1) / kTileSlots);
+    cudaError_t e = launch_onepass(ids, base, S, E, A, G, workspace, counts, offsets, bso,
+                                   in_perm, out_perm, diag, stream);
+    if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+    e = launch(prep_rank_kernel<IdT>, G, kTileThreads, tile_smem(E), stream, ids, base, S, E, A,
+               G, workspace, counts, offsets, bso, out_perm, diag);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = persistent_grid(prep_finish_kernel<IdT>, 256, 0, (S + 1023) / 1024);
+    return launch(prep_finish_kernel<IdT>, grid, 256, 0, stream, ids, base, S, E,
+                  (const int32_t *)offsets, in_perm, out_perm);
+}
+
 }  // namespace
 
-cudaError_t run_prepare(const int32_t *ids, int64_t S, int E, int A, int32_t *counts,
-                        int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,
-                        int32_t *diag, void *workspace, cudaStream_t stream) {
-    if (S <= kSingleBlockSlots)
-        return launch(prep_single_kernel, 1, kSingleThreads, single_block_smem(E), stream, ids, S,
-                      E, A, counts, offsets, bso, in_perm, out_perm, diag);
-    const int G = (int)((S + kTileSlots - 1) / kTileSlots);
-    cudaError_t e = launch_onepass(ids, S, E, A, G, workspace, counts, offsets, bso, in_perm,
-                                   out_perm, diag, stream);
-    if (e != cudaErrorCooperativeLaunchTooLarge) return e;
-    e = launch(prep_rank_kernel, G, kTileThreads, tile_smem(E), stream, ids, S, E, A, G,
-               workspace, counts, offsets, bso, out_perm, diag);
-    if (e != cudaSuccess) return e;
-    const int64_t grid = persistent_grid(prep_finish_kernel, 256, 0, (S + 1023) / 1024);
-    return launch(prep_finish_kernel, grid, 256, 0, stream, ids, S, E, (const int32_t *)offsets,
-                  in_perm, out_perm);
+cudaError_t run_prepare(const void *ids, bool ids64, int64_t base, int64_t S, int E, int A,
+                        int32_t *counts, int32_t *offsets, int32_t *bso, int32_t *in_perm,
+                        int32_t *out_perm, int32_t *diag, void *workspace, cudaStream_t stream) {
+    if (ids64)
+        return run_prepare_t((const int64_t *)ids, base, S, E, A, counts, offsets, bso, in_perm,
+                             out_perm, diag, workspace, stream);
+    return run_prepare_t((const int32_t *)ids, base, S, E, A, counts, offsets, bso, in_perm,
+                         out_perm, diag, workspace, stream);
 }
 
 cudaError_t run_prepare_dispatch(const int32_t *ids, int64_t T, int k, int E, int A,

@@ -75,7 +75,7 @@ extern "C" moe_status_t moe_prepare_no_alloc(const int32_t *topk_ids, int64_t nu
         if (e != cudaSuccess) return moe::status_from_cuda(e);
     }
     return moe::status_from_cuda(moe::run_prepare(
-        topk_ids, S, num_experts, blockscale_offsets ? blockscale_align : 1, expert_counts,
+        topk_ids, false, 0, S, num_experts, blockscale_offsets ? blockscale_align : 1, expert_counts,
         expert_offsets, blockscale_offsets, input_permutation, output_permutation, diag, scratch,
         (cudaStream_t)stream));
 }

@@ -67,6 +67,11 @@ typedef enum {
     MOE_FP8_E4M3 = 3 /* OCP E4M3 "FN": no infinities, max finite 448 */
 } moe_dtype_t;
 
+typedef enum {
+    MOE_I32 = 0, /* int32 expert ids                                   */
+    MOE_I64 = 1  /* int64 expert ids (the Mooncake top-k index type)   */
+} moe_index_t;
+
 /* Largest expert count the prepare kernels accept. */
 #define MOE_MAX_EXPERTS 1024
 
@@ -170,8 +175,9 @@ moe_status_t moe_dispatch_rows(const void *x, moe_dtype_t dtype, int64_t num_tok
  * Dispatch with FP8 E4M3 1x128 block-scale quantisation (TensorRT-LLM PR
  * #9592, FP8 block-scale MoE path, "run_moe_fp8_block_scales"; the optional
  * FP8 block-scale offsets of sglang PR #19058 place the scales).  For every
- * valid slot i = t*k + j with p = output_permutation[i] and e = topk_ids[i],
- * and every 128-column block b:
+ * valid slot i = t*k + j with p = output_permutation[i] >= 0, e the expert
+ * whose rows [expert_offsets[e], expert_offsets[e+1]) hold p, and every
+ * 128-column block b:
  *
  *   amax = max |x[t, 128b .. 128b+127]|      (in fp32)
  *   s    = amax / 448                         (fp32, round to nearest)
@@ -180,17 +186,18 @@ moe_status_t moe_dispatch_rows(const void *x, moe_dtype_t dtype, int64_t num_tok
  *
  * A block with amax = 0 gets s = 0 and zero bytes.  Rows of out_q and
  * scale rows that no valid slot maps to (including the padding rows of each
- * expert's scale segment) are not written.
+ * expert's scale segment) are not written.  The expert of a row comes from
+ * the offsets, so any id type or expert window of moe_prepare_local works.
  *
  *   x          [T, H] BF16 or F16, H a multiple of 128, 16-byte aligned.
- *   topk_ids   [T, k] int32; output_permutation [T*k] int32;
+ *   output_permutation [T*k] int32;
  *   expert_offsets / blockscale_offsets [E+1] int32 (from moe_prepare).
  *   out_q      [T*k, H] uint8 (E4M3 bytes); out_scales [rows, H/128] fp32
  *              with rows >= blockscale_offsets[E].
  */
 moe_status_t moe_dispatch_rows_fp8(const void *x, moe_dtype_t x_dtype, int64_t num_tokens,
                                    int64_t hidden, int32_t top_k, int32_t num_experts,
-                                   const int32_t *topk_ids, const int32_t *output_permutation,
+                                   const int32_t *output_permutation,
                                    const int32_t *expert_offsets,
                                    const int32_t *blockscale_offsets, uint8_t *out_q,
                                    float *out_scales, moe_stream_t stream);
@@ -248,14 +255,14 @@ moe_status_t moe_problem_sizes(const int32_t *expert_counts, int32_t num_experts
  *     tile_idx_to_mn_limit[t] = padded_offsets[e] + expert_counts[e] (the
  *     end of that expert's real rows); later tiles up to max_tiles get -1
  *     in both;
- *   a valid slot i of expert e with dispatched row p is on padded row
- *     expanded_idx_to_permuted_idx[i] = padded_offsets[e] + p - expert_offsets[e]
- *     (-1 for slots whose id was invalid);
+ *   a slot i with dispatched row p = output_permutation[i] >= 0 of expert e
+ *     is on padded row expanded_idx_to_permuted_idx[i] =
+ *     padded_offsets[e] + p - expert_offsets[e] (-1 for unrouted slots);
  *   permuted_idx_to_expanded_idx is its inverse over all max_tiles *
  *     tile_size rows, -1 on padding rows and past the padded total.
  *
- *   topk_ids [T, k], expert_counts [E], expert_offsets [E+1],
- *   output_permutation [T*k]           int32, from moe_prepare
+ *   expert_counts [E], expert_offsets [E+1], output_permutation [T*k]
+ *                                      int32, from moe_prepare / _local
  *   padded_offsets [E+1], tile_idx_to_group_idx [max_tiles],
  *   tile_idx_to_mn_limit [max_tiles], expanded_idx_to_permuted_idx [T*k],
  *   permuted_idx_to_expanded_idx [max_tiles * tile_size],
@@ -266,8 +273,8 @@ moe_status_t moe_problem_sizes(const int32_t *expert_counts, int32_t num_experts
  * device), num_non_exiting_tiles is set to -1, total_num_padded_tokens and
  * padded_offsets hold the needed sizes and nothing else is written.
  */
-moe_status_t moe_tile_layout(const int32_t *topk_ids, int64_t num_tokens, int32_t top_k,
-                             int32_t num_experts, int32_t tile_size, const int32_t *expert_counts,
+moe_status_t moe_tile_layout(int64_t num_tokens, int32_t top_k, int32_t num_experts,
+                             int32_t tile_size, const int32_t *expert_counts,
                              const int32_t *expert_offsets, const int32_t *output_permutation,
                              int32_t max_tiles, int32_t *padded_offsets,
                              int32_t *tile_idx_to_group_idx, int32_t *tile_idx_to_mn_limit,
@@ -275,6 +282,41 @@ moe_status_t moe_tile_layout(const int32_t *topk_ids, int64_t num_tokens, int32_
                              int32_t *permuted_idx_to_expanded_idx,
                              int32_t *num_non_exiting_tiles, int32_t *total_num_padded_tokens,
                              moe_stream_t stream);
+
+/*
+ * moe_prepare for one rank's window of experts and for int64 ids (the
+ * local-expert slice local_expert_offset / num_local_experts of TensorRT-LLM
+ * PR #9592's grouped GEMM, and Mooncake PR #4581's int64 top-k index type).
+ * Slot i belongs to local expert topk_ids[i] - local_expert_offset when that
+ * lies in [0, num_local_experts); every other slot is excluded exactly as an
+ * invalid id is in moe_prepare (not counted, output_permutation -1, counted
+ * in diag[0]).  All outputs are sized by num_local_experts (E below); the
+ * workspace is moe_prepare_workspace_bytes(T, k, num_local_experts).
+ *
+ *   topk_ids  [T, k] int32 (id_type MOE_I32) or int64 (MOE_I64).
+ *   The other arguments are those of moe_prepare.
+ */
+moe_status_t moe_prepare_local(const void *topk_ids, moe_index_t id_type, int64_t num_tokens,
+                               int32_t top_k, int64_t local_expert_offset,
+                               int32_t num_local_experts, int32_t *expert_counts,
+                               int32_t *expert_offsets, int32_t *blockscale_offsets,
+                               int32_t blockscale_align, int32_t *input_permutation,
+                               int32_t *output_permutation, int32_t *diag, void *workspace,
+                               size_t workspace_bytes, moe_stream_t stream);
+
+/*
+ * Output memset (TensorRT-LLM PR #9592, moe_output_memset_inplace): zero
+ * out[t, :] for every token t with at least one routed slot
+ * (output_permutation[t*k + j] >= 0 for some j); every other row keeps its
+ * contents.  Used before an expert stage that accumulates into the output
+ * for this rank's experts only.
+ *
+ *   out [T, H] F32, F16 or BF16, H * sizeof a multiple of 16 bytes,
+ *   16-byte aligned; output_permutation [T*k] int32.
+ */
+moe_status_t moe_output_memset(void *out, moe_dtype_t dtype, int64_t num_tokens, int64_t hidden,
+                               int32_t top_k, const int32_t *output_permutation,
+                               moe_stream_t stream);
 
 /* Size of the device array that moe_prepare_no_alloc uses as scratch. */
 #define MOE_PREPARE_NO_ALLOC_SCRATCH_BYTES ((size_t)4 << 20)

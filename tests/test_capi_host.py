@@ -116,21 +116,49 @@ def test_dispatch_validation(lib):
 
 def test_dispatch_fp8_validation(lib):
     f = lib.moe_dispatch_rows_fp8
-    args = dict(x=P, dt=BF16, T=4, H=256, k=2, E=8, ids=P, op=P, off=P, bso=P, q=P, sc=P)
+    args = dict(x=P, dt=BF16, T=4, H=256, k=2, E=8, op=P, off=P, bso=P, q=P, sc=P)
 
     def call(**kw):
         a = dict(args, **kw)
-        return f(a["x"], a["dt"], a["T"], a["H"], a["k"], a["E"], a["ids"], a["op"], a["off"],
-                 a["bso"], a["q"], a["sc"], None)
+        return f(a["x"], a["dt"], a["T"], a["H"], a["k"], a["E"], a["op"], a["off"], a["bso"],
+                 a["q"], a["sc"], None)
 
     assert call(dt=F32) == UNSUPPORTED
     assert call(H=200) == INVALID                                    # H % 128 != 0
     assert call(E=0) == INVALID
-    for key in ("x", "ids", "op", "off", "bso", "q", "sc"):
+    for key in ("x", "op", "off", "bso", "q", "sc"):
         assert call(**{key: None}) == INVALID, key
     assert call(q=P + 8) == INVALID
     assert call(sc=P + 2) == INVALID
     assert call(T=0, x=None) == OK
+
+
+def test_prepare_local_and_memset_validation(lib):
+    pl = lib.moe_prepare_local
+    assert pl(P, 2, 4, 2, 0, 8, P, P, None, 1, P, P, None, None, 0, None) == INVALID   # bad id type
+    assert pl(P, 1, 4, 2, 0, 0, P, P, None, 1, P, P, None, None, 0, None) == INVALID   # no experts
+    assert pl(P, 1, 4, 2, 0, 2000, P, P, None, 1, P, P, None, None, 0, None) == UNSUPPORTED
+    assert pl(P, 1, 1000, 8, 5, 8, P, P, None, 1, P, P, None, None, 0, None) == WORKSPACE
+    om = lib.moe_output_memset
+    assert om(P, FP8, 4, 64, 2, P, None) == INVALID
+    assert om(P, BF16, 4, 12, 2, P, None) == INVALID                   # 24-byte rows
+    assert om(None, BF16, 4, 64, 2, P, None) == INVALID
+    assert om(P + 4, BF16, 4, 64, 2, P, None) == INVALID
+    assert om(None, BF16, 0, 64, 2, None, None) == OK
+
+
+def test_tile_layout_validation(lib):
+    tl = lib.moe_tile_layout
+    args = [4, 2, 8, 16, P, P, P, 4, P, P, P, P, P, P, P, None]
+    bad = list(args); bad[3] = 0
+    assert tl(*bad) == INVALID                                       # tile size 0
+    bad = list(args); bad[7] = 0
+    assert tl(*bad) == INVALID                                       # no tiles
+    bad = list(args); bad[7] = 1 << 20; bad[3] = 1 << 12
+    assert tl(*bad) == UNSUPPORTED                                   # rows past 2^31
+    bad = list(args); bad[6] = None
+    assert tl(*bad) == INVALID                                       # no permutation
+    assert lib.moe_problem_sizes(None, 8, 1, 1, 1, 1, P, P, None) == INVALID
 
 
 def test_combine_validation(lib):

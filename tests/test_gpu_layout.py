@@ -16,7 +16,7 @@ DEV = torch.device("cuda:0")
 def _layout_case(ids_np, E, tile, max_tiles=None):
     ids = torch.from_numpy(ids_np).to(DEV)
     meta = moe.moe_prepare(ids, E)
-    got = moe.moe_tile_layout(ids, meta, tile, max_tiles)
+    got = moe.moe_tile_layout(meta, ids_np.shape[1], tile, max_tiles)
     torch.cuda.synchronize()
     T, k = ids_np.shape
     S = T * k

@@ -181,7 +181,7 @@ def _fp8_run(ids_np, E, x, A):
     q = torch.full((T * k, H), 0xAB, dtype=torch.uint8, device=DEV)
     rows = T * k + E * (A - 1)
     sc = torch.full((rows, H // 128), float("nan"), device=DEV)
-    moe.moe_dispatch_rows_fp8(x, ids, meta.output_permutation, meta.expert_offsets,
+    moe.moe_dispatch_rows_fp8(x, k, meta.output_permutation, meta.expert_offsets,
                               meta.blockscale_offsets, out_q=q, out_scales=sc)
     torch.cuda.synchronize()
     ref_meta = oracle.prepare(ids_np, E, A)
@@ -238,7 +238,7 @@ def test_dispatch_fp8_full_workload_sampled():
     ids = torch.from_numpy(ids_np).to(DEV)
     A = w.block_align
     meta = moe.moe_prepare(ids, w.E, blockscale_align=A)
-    q, sc = moe.moe_dispatch_rows_fp8(x, ids, meta.output_permutation, meta.expert_offsets,
+    q, sc = moe.moe_dispatch_rows_fp8(x, w.k, meta.output_permutation, meta.expert_offsets,
                                       meta.blockscale_offsets, blockscale_align=A)
     torch.cuda.synchronize()
     ref_meta = oracle.prepare(ids_np, w.E, A)
