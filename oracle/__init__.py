@@ -34,7 +34,7 @@ from .build import build_oracle, oracle_lib_path
 __all__ = [
     "F32", "F16", "BF16", "lib", "prepare", "dispatch", "dispatch_fp8",
     "combine", "brute_prepare", "problem_sizes", "tile_layout", "prepare_local",
-    "output_memset", "f32_to_bf16", "f32_to_f16", "f16_to_f32",
+    "output_memset", "dispatch_nvfp4", "f32_to_e2m1", "e2m1_to_f32", "f32_to_bf16", "f32_to_f16", "f16_to_f32",
     "bf16_to_f32", "f32_to_e4m3", "e4m3_to_f32",
 ]
 
@@ -71,12 +71,18 @@ def lib():
                                                ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp]
         L.oracle_output_memset.restype = None
         L.oracle_output_memset.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32, _vp]
+        L.oracle_dispatch_nvfp4.restype = None
+        L.oracle_dispatch_nvfp4.argtypes = [_vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                            ctypes.c_int32, _vp, _vp, _vp, _vp, ctypes.c_int64,
+                                            _vp, _vp]
+        L.oracle_e2m1_to_f32.restype = ctypes.c_float
+        L.oracle_e2m1_to_f32.argtypes = [ctypes.c_uint8]
         L.oracle_problem_sizes.restype = None
         L.oracle_problem_sizes.argtypes = [_vp, ctypes.c_int32] + [ctypes.c_int32] * 4 + [_vp, _vp]
         L.oracle_tile_layout.restype = ctypes.c_int
         L.oracle_tile_layout.argtypes = [_vp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                          ctypes.c_int32, _vp, _vp, _vp, ctypes.c_int32] + [_vp] * 7
-        for name in ["oracle_f32_to_e4m3_n", "oracle_f32_to_bf16_n", "oracle_f32_to_f16_n",
+        for name in ["oracle_f32_to_e2m1_n", "oracle_f32_to_e4m3_n", "oracle_f32_to_bf16_n", "oracle_f32_to_f16_n",
                      "oracle_f16_to_f32_n", "oracle_bf16_to_f32_n", "oracle_e4m3_to_f32_n"]:
             fn = getattr(L, name)
             fn.restype = None
@@ -189,6 +195,33 @@ def output_memset(out: np.ndarray, output_perm: np.ndarray, k: int):
     T = out.shape[0]
     lib().oracle_output_memset(_ptr(out), out.nbytes // max(T, 1), T, k, _ptr(output_perm))
     return out
+
+
+def dispatch_nvfp4(x_bits: np.ndarray, x_dtype: str, ids: np.ndarray, meta: dict,
+                   q: np.ndarray | None = None, scales: np.ndarray | None = None):
+    """NVFP4 dispatch (see moe_oracle.c): (q [S, H/2] packed E2M1 codes,
+    scales [bso[E], H/16] E4M3 bytes).  Arrays passed in are written in place."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, H = x_bits.shape
+    k = ids.shape[1]
+    S = T * k
+    if q is None:
+        q = np.zeros((S, H // 2), np.uint8)
+    if scales is None:
+        scales = np.zeros((int(meta["bso"][-1]), H // 16), np.uint8)
+    lib().oracle_dispatch_nvfp4(_ptr(x_bits), _DT[x_dtype], T, H, k, _ptr(ids),
+                                _ptr(meta["input_perm"]), _ptr(meta["offsets"]), _ptr(meta["bso"]),
+                                S, _ptr(q), _ptr(scales))
+    return q, scales
+
+
+def f32_to_e2m1(a):
+    return _conv("oracle_f32_to_e2m1_n", a, np.float32, np.uint8)
+
+
+def e2m1_to_f32(codes):
+    return np.array([lib().oracle_e2m1_to_f32(int(c)) for c in np.asarray(codes).ravel()], np.float32)
 
 
 def problem_sizes(counts: np.ndarray, n1: int, k1: int, n2: int, k2: int):

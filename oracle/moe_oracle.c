@@ -526,3 +526,100 @@ void oracle_output_memset(void *out, int64_t row_bytes, int64_t T, int32_t k,
             memset(o + t * row_bytes, 0, (size_t)row_bytes);
     }
 }
+
+/* ------------------------------------------------------------------ */
+/* NVFP4 dispatch: E2M1 elements with one E4M3 scale per 16 elements.  */
+/* ------------------------------------------------------------------ */
+
+/*
+ * binary32 -> FP4 E2M1 (1 sign bit, 2 exponent bits with bias 1, 1 fraction
+ * bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6; no infinities or NaN), round to
+ * nearest even, saturating to +-6.  Returns the 4-bit code (sign in bit 3).
+ * NaN maps to +0 (the format has no NaN; inputs here are finite).
+ */
+uint8_t oracle_f32_to_e2m1(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    uint8_t sign = (uint8_t)((u >> 28) & 0x8u);
+    if ((u & 0x7fffffffu) > 0x7f800000u)
+        return 0;
+    double a = fabs((double)f);
+    if (a >= 6.0)
+        return (uint8_t)(sign | 0x7u);
+    if (a < 1.0) {                                   /* subnormal range: step 0.5 */
+        double q = round_half_even(a / 0.5);        /* 0, 1 or 2 (2 encodes 1.0) */
+        return (uint8_t)(sign | (uint8_t)q);
+    }
+    int ex;
+    frexp(a, &ex);
+    int e = ex - 1;                                  /* a in [2^e, 2^(e+1)), e in 0..2 */
+    double q = round_half_even(a / ldexp(1.0, e - 1)); /* in [2, 4] */
+    int code = (e + 1) * 2 + (int)q - 2;
+    if (code > 7)
+        code = 7;
+    return (uint8_t)(sign | (uint8_t)code);
+}
+
+float oracle_e2m1_to_f32(uint8_t c)
+{
+    int sign = (c >> 3) & 1;
+    int expo = (c >> 1) & 3;
+    int frac = c & 1;
+    double v = expo == 0 ? 0.5 * frac : ldexp(1.0 + 0.5 * frac, expo - 1);
+    return (float)(sign ? -v : v);
+}
+
+void oracle_f32_to_e2m1_n(const float *in, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_f32_to_e2m1(in[i]);
+}
+
+/*
+ * NVFP4 dispatch (the B200 NVFP4 MoE path of TensorRT-LLM PR #9592, block
+ * size scaling_vector_size = 16).  For each dispatched row p (token t =
+ * input_perm[p] / k, expert e = ids[input_perm[p]]) and each 16-column
+ * block b:
+ *   amax  = max |x[t, 16b .. 16b+15]|
+ *   sf    = e4m3(amax / 6)            (fp32 division, then E4M3 RNE, satfinite)
+ *   d     = the fp32 value of sf
+ *   q[p, c] = e2m1(x[t, c] / d)       (fp32 division, E2M1 RNE, saturating)
+ *             or 0 when d = 0
+ * Two codes per byte: element 2m in the low nibble, 2m+1 in the high one.
+ * The scale byte goes to scales[(bso[e] + p - offsets[e]) * (H/16) + b].
+ */
+void oracle_dispatch_nvfp4(const uint16_t *x, int x_dtype, int64_t T, int64_t H, int32_t k,
+                           const int32_t *ids, const int32_t *input_perm, const int32_t *offsets,
+                           const int32_t *bso, int64_t S, uint8_t *q, uint8_t *scales)
+{
+    (void)T;
+    int64_t nb = H / 16;
+    for (int64_t p = 0; p < S; ++p) {
+        int32_t i = input_perm[p];
+        if (i < 0)
+            continue;
+        int64_t t = i / k;
+        int32_t e = ids[i];
+        int64_t srow = (int64_t)bso[e] + (p - offsets[e]);
+        for (int64_t b = 0; b < nb; ++b) {
+            float amax = 0.0f;
+            for (int64_t c = b * 16; c < b * 16 + 16; ++c) {
+                float a = fabsf(load_as_f32(x, x_dtype, t * H + c));
+                if (a > amax)
+                    amax = a;
+            }
+            uint8_t sf = oracle_f32_to_e4m3(amax / 6.0f);
+            float d = oracle_e4m3_to_f32(sf);
+            for (int64_t c = b * 16; c < b * 16 + 16; c += 2) {
+                uint8_t lo = 0, hi = 0;
+                if (d != 0.0f) {
+                    lo = oracle_f32_to_e2m1(load_as_f32(x, x_dtype, t * H + c) / d);
+                    hi = oracle_f32_to_e2m1(load_as_f32(x, x_dtype, t * H + c + 1) / d);
+                }
+                q[p * (H / 2) + c / 2] = (uint8_t)(lo | (hi << 4));
+            }
+            scales[srow * nb + b] = sf;
+        }
+    }
+}

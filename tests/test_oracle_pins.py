@@ -475,3 +475,72 @@ def test_output_memset_zeroes_exactly_the_routed_tokens():
     assert (out[routed] == 0).all()
     np.testing.assert_array_equal(out[~routed], before[~routed])
     assert routed.any() and (~routed).any()
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 (E2M1 elements, one E4M3 scale per 16 elements)
+# ---------------------------------------------------------------------------
+
+E2M1_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]   # codes 0..7, from the format
+
+
+def test_e2m1_decode_all_codes():
+    got = oracle.e2m1_to_f32(np.arange(16))
+    np.testing.assert_array_equal(got[:8], E2M1_VALUES)
+    np.testing.assert_array_equal(got[8:], [-v for v in E2M1_VALUES])
+
+
+def test_e2m1_closed_forms():
+    cases = [(0.25, 0), (0.26, 1), (0.75, 2), (1.25, 2), (1.75, 4), (2.5, 4), (3.5, 6),
+             (5.0, 6), (5.01, 7), (6.0, 7), (100.0, 7), (-0.75, 10), (-5.0, 14), (-0.0, 8)]
+    got = oracle.f32_to_e2m1(np.array([v for v, _ in cases], np.float32))
+    np.testing.assert_array_equal(got, np.array([c for _, c in cases], np.uint8))
+
+
+def test_e2m1_encode_vs_bruteforce_nearest_even():
+    """Nearest representable magnitude by brute force over the 8 values, ties
+    to the even code (fraction bit 0), saturation at 6."""
+    rng = np.random.default_rng(8)
+    vals = np.array(E2M1_VALUES)
+    mids = (vals[1:] + vals[:-1]) / 2
+    f = np.concatenate([rng.uniform(-8, 8, 200_000), mids, -mids,
+                        np.nextafter(mids.astype(np.float32), np.float32(0)),
+                        np.nextafter(mids.astype(np.float32), np.float32(9))]).astype(np.float32)
+    a = np.minimum(np.abs(f).astype(np.float64), 6.0)
+    dist = np.abs(a[:, None] - vals[None, :])
+    best = dist.min(axis=1, keepdims=True)
+    cand = dist == best
+    even = cand & (np.arange(8)[None, :] % 2 == 0)
+    code = np.where(even.any(axis=1), even.argmax(axis=1), cand.argmax(axis=1))
+    code = code | np.where(np.signbit(f), 8, 0)
+    np.testing.assert_array_equal(oracle.f32_to_e2m1(f), code.astype(np.uint8))
+
+
+def test_dispatch_nvfp4_decode_bound_and_layout():
+    T, H, E, k, A = 40, 256, 8, 3, 4
+    rng = np.random.default_rng(9)
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    x = torch.randn(T, H, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
+    x[0, :16] = 0
+    m = oracle.prepare(ids, E, A)
+    q, sc = oracle.dispatch_nvfp4(x.view(torch.int16).numpy().view(np.uint16), "bf16", ids, m)
+    xr = x.float().numpy()[m["input_perm"] // k]
+    codes = np.stack([q & 0xF, q >> 4], axis=2).reshape(T * k, H)     # low nibble first
+    vals = oracle.e2m1_to_f32(codes).reshape(T * k, H).astype(np.float64)
+    e = ids.ravel()[m["input_perm"]]
+    srow = m["bso"][e] + np.arange(T * k) - m["offsets"][e]
+    d = oracle.e4m3_to_f32(sc[srow].ravel()).reshape(T * k, H // 16).astype(np.float64)
+    dd = np.repeat(d, 16, axis=1)
+    # the scale is e4m3(amax / 6): the amax element lands on +-6 or one e2m1 step below
+    blocks = np.abs(xr).reshape(T * k, H // 16, 16)
+    amax = blocks.max(axis=2)
+    np.testing.assert_array_equal(sc[srow], oracle.f32_to_e4m3((amax / 6.0).astype(np.float32)).reshape(amax.shape))
+    # every element within half an e2m1 step (of x / d) of its value, saturation aside
+    v = np.abs(xr) / np.where(dd == 0, 1, dd)
+    half = np.where(v < 2, 0.25, np.where(v < 4, 0.5, 1.0))
+    ok = (np.abs(vals * dd - xr) <= half * dd * (1 + 1e-6) + 1e-30) | (v > 6)
+    assert ok.all()
+    # token 0's first block is all zero: scale byte 0 and codes 0 on each of its k rows
+    rows0 = np.nonzero(m["input_perm"] // k == 0)[0]
+    assert len(rows0) == k
+    assert (sc[srow[rows0], 0] == 0).all() and (q[rows0, :8] == 0).all()
