@@ -523,9 +523,10 @@ def run_gpu(args, w):
 
 
 def time_next_rows(step, w, dev, reps=20):
-    """The grouped-GEMM metadata steps that follow prepare (tile-padded
-    layout with 128-row tiles, and the per-expert problem sizes), timed on
-    this workload's metadata as a CUDA graph of `reps` calls each."""
+    """The steps beside the timed path: the grouped-GEMM metadata that follows
+    prepare (tile-padded layout with 128-row tiles, per-expert problem
+    sizes) and the NVFP4 dispatch of this workload's activations, each timed
+    as a CUDA graph of `reps` calls."""
     import torch
     moe = step.moe
     meta = step.prepare()
@@ -559,6 +560,16 @@ def time_next_rows(step, w, dev, reps=20):
     us = timed(lambda: moe.moe_problem_sizes(meta.expert_counts, 2 * w.H, w.H, w.H, w.H))
     b = 4 * E + 24 * E
     out["problem_sizes"] = {"us": us, "algorithmic_bytes": b}
+    if step.x.dtype in (torch.bfloat16, torch.float16) and w.H % 16 == 0:
+        bso = meta.blockscale_offsets if meta.blockscale_offsets is not None else meta.expert_offsets
+        A = step.A or 1
+        q = torch.empty((S, w.H // 2), dtype=torch.uint8, device=dev)
+        sc = torch.empty((S + E * (A - 1), w.H // 16), dtype=torch.uint8, device=dev)
+        us = timed(lambda: moe.moe_dispatch_rows_nvfp4(step.x, w.k, meta.output_permutation,
+                                                       meta.expert_offsets, bso, out_q=q,
+                                                       out_scales=sc))
+        b = w.T * w.H * step.x.element_size() + S * (w.H // 2 + w.H // 16) + 4 * S + 8 * (E + 1)
+        out["dispatch_nvfp4"] = {"us": us, "algorithmic_bytes": b, "effective_gbs": b / us / 1e3}
     return out
 
 

@@ -28,6 +28,7 @@ __all__ = [
     "moe_prepare_workspace_bytes",
     "moe_dispatch_rows",
     "moe_dispatch_rows_fp8",
+    "moe_dispatch_rows_nvfp4",
     "moe_combine",
     "moe_prepare_dispatch",
     "moe_version",
@@ -236,6 +237,48 @@ def moe_dispatch_rows_fp8(x: torch.Tensor, top_k: int, output_permutation: torch
             expert_offsets.data_ptr(), blockscale_offsets.data_ptr(), out_q.data_ptr(),
             out_scales.data_ptr(), _stream(dev))
     _lib.check("moe_dispatch_rows_fp8", st)
+    return out_q, out_scales
+
+
+def moe_dispatch_rows_nvfp4(x: torch.Tensor, top_k: int, output_permutation: torch.Tensor,
+                            expert_offsets: torch.Tensor, blockscale_offsets: torch.Tensor, *,
+                            blockscale_align: int = 1, out_q: Optional[torch.Tensor] = None,
+                            out_scales: Optional[torch.Tensor] = None):
+    """NVFP4 dispatch (E2M1 codes two per byte, one E4M3 scale byte per 16
+    elements; see include/moe.h).  Returns (out_q uint8 [T*k, H/2],
+    out_scales uint8 [rows, H/16]).
+
+    Without ``out_scales`` the scale tensor is allocated with the upper bound
+    T*k + E*(blockscale_align - 1) rows (no device-to-host read).
+    """
+    _need(x, "x")
+    T, H = x.shape
+    k = top_k
+    E = expert_offsets.numel() - 1
+    S = T * k
+    dev = x.device
+    _need(output_permutation, "output_permutation", torch.int32, (S,), dev)
+    _need(expert_offsets, "expert_offsets", torch.int32, (E + 1,), dev)
+    _need(blockscale_offsets, "blockscale_offsets", torch.int32, (E + 1,), dev)
+    if x.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError("nvfp4 dispatch reads bf16 or fp16 activations")
+    if H % 16:
+        raise ValueError("nvfp4 dispatch needs a hidden size that is a multiple of 16")
+    if out_q is None:
+        out_q = torch.empty((S, H // 2), dtype=torch.uint8, device=dev)
+    _need(out_q, "out_q", torch.uint8, (S, H // 2), dev)
+    if out_scales is None:
+        out_scales = torch.empty((S + E * (blockscale_align - 1), H // 16), dtype=torch.uint8,
+                                 device=dev)
+    if out_scales.dtype == torch.float8_e4m3fn:
+        out_scales = out_scales.view(torch.uint8)
+    _need(out_scales, "out_scales", torch.uint8, None, dev)
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_dispatch_rows_nvfp4(
+            x.data_ptr(), _dtype_code(x.dtype), T, H, k, E, output_permutation.data_ptr(),
+            expert_offsets.data_ptr(), blockscale_offsets.data_ptr(), out_q.data_ptr(),
+            out_scales.data_ptr(), _stream(dev))
+    _lib.check("moe_dispatch_rows_nvfp4", st)
     return out_q, out_scales
 
 

@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(PKG, "libmoe.so")
 
 # moe_status_t / moe_dtype_t values (include/moe.h)
 MOE_OK = 0
-MOE_ERR_CUDA = 4
+MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = 1, 2, 3, 4
 MOE_F32, MOE_F16, MOE_BF16, MOE_FP8_E4M3 = 0, 1, 2, 3
 MOE_I32, MOE_I64 = 0, 1
 MAX_EXPERTS = 1024
@@ -30,6 +30,7 @@ EXPORTED = (
     "moe_prepare",
     "moe_dispatch_rows",
     "moe_dispatch_rows_fp8",
+    "moe_dispatch_rows_nvfp4",
     "moe_combine",
     "moe_prepare_dispatch",
     "moe_prepare_no_alloc",
@@ -54,6 +55,8 @@ _SIGNATURES = {
     "moe_dispatch_rows": (_int, [_vp, _int, _i64, _i64, _i32, _vp, _vp, _vp, _vp]),
     "moe_dispatch_rows_fp8": (_int, [_vp, _int, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp,
                                      _vp, _vp]),
+    "moe_dispatch_rows_nvfp4": (_int, [_vp, _int, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp,
+                                       _vp, _vp]),
     "moe_combine": (_int, [_vp, _int, _i64, _i64, _i32, _vp, _vp, _vp, _int, _vp]),
     "moe_prepare_dispatch": (_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp,
                                     _vp, _int, _i64, _vp, _vp]),

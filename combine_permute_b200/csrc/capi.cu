@@ -171,6 +171,28 @@ moe_status_t moe_dispatch_rows_fp8(const void *x, moe_dtype_t x_dtype, int64_t n
                                            out_q, out_scales, (cudaStream_t)stream));
 }
 
+moe_status_t moe_dispatch_rows_nvfp4(const void *x, moe_dtype_t x_dtype, int64_t num_tokens,
+                                     int64_t hidden, int32_t top_k, int32_t num_experts,
+                                     const int32_t *output_permutation,
+                                     const int32_t *expert_offsets,
+                                     const int32_t *blockscale_offsets, uint8_t *out_q,
+                                     uint8_t *out_scales, moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (x_dtype != MOE_BF16 && x_dtype != MOE_F16) return MOE_ERR_UNSUPPORTED;
+    if (hidden < 1 || hidden % 16 != 0 || num_experts < 1) return MOE_ERR_INVALID_ARG;
+    if (num_experts > 4 * moe::kMaxExperts || top_k > 4096) return MOE_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return MOE_OK;
+    if (!x || !output_permutation || !expert_offsets || !blockscale_offsets || !out_q ||
+        !out_scales)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || ((uintptr_t)out_q & 7u)) return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_dispatch_nvfp4(x, dt(x_dtype), num_tokens, hidden, top_k,
+                                             num_experts, output_permutation, expert_offsets,
+                                             blockscale_offsets, out_q, out_scales,
+                                             (cudaStream_t)stream));
+}
+
 moe_status_t moe_combine(const void *y, moe_dtype_t y_dtype, int64_t num_tokens, int64_t hidden,
                          int32_t top_k, const int32_t *output_permutation, const float *weights,
                          void *out, moe_dtype_t out_dtype, moe_stream_t stream) {

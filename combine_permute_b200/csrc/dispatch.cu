@@ -257,6 +257,81 @@ __global__ void __launch_bounds__(kFp8Threads)
     }
 }
 
+
+// NVFP4 dispatch.  A block walks tokens; per token it resolves the k
+// dispatched rows and their scale rows once (from the expert offsets staged
+// in shared memory), then each thread takes 16-element groups of the row:
+// two 16-byte loads, the group amax, its E4M3 scale sf = e4m3(amax / 6), and
+// the 16 E2M1 codes of x / value(sf), stored as 8 bytes to each of the k
+// rows (a warp writes 256 contiguous bytes of a row) plus the scale byte.
+template <typename XT>
+__global__ void __launch_bounds__(kFp8Threads)
+    dispatch_nvfp4_kernel(const XT *__restrict__ x, int64_t T, int64_t H, int k, int E,
+                          const int32_t *__restrict__ out_perm, const int32_t *__restrict__ offsets,
+                          const int32_t *__restrict__ bso, uint8_t *__restrict__ q,
+                          uint8_t *__restrict__ scales) {
+    extern __shared__ int smem[];
+    int *s_off = smem;             // [E+1] expert offsets
+    int *s_delta = s_off + E + 1;  // [E] scale row - dispatched row, per expert
+    int *s_p = s_delta + E;        // [k] this token's dispatched rows
+    int *s_srow = s_p + k;         // [k] and their scale rows
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int e = threadIdx.x; e <= E; e += kFp8Threads) {
+        s_off[e] = __ldg(offsets + e);
+        if (e < E) s_delta[e] = __ldg(bso + e) - __ldg(offsets + e);
+    }
+    const int64_t n16 = H / 16;  // groups per row = scale bytes per row
+    const int64_t S = T * k;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        __syncthreads();  // offsets staged; the previous token's rows consumed
+        for (int j = threadIdx.x; j < k; j += kFp8Threads) {
+            int p = __ldg(out_perm + t * k + j);
+            int srow = -1;
+            if (p >= 0 && p < S && p < s_off[E]) {
+                int lo = 0, hi = E;  // the expert whose rows hold p
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (s_off[mid] <= p) lo = mid;
+                    else hi = mid;
+                }
+                srow = p + s_delta[lo];
+            } else {
+                p = -1;
+            }
+            s_p[j] = p;
+            s_srow[j] = srow;
+        }
+        __syncthreads();
+        for (int64_t g = threadIdx.x; g < n16; g += kFp8Threads) {
+            const XT *src = x + t * H + g * 16;
+            float f[16];
+            unpack8<XT>(ld_stream_v4(src), f);
+            unpack8<XT>(ld_stream_v4(src + 8), f + 8);
+            float amax = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
+            const uint16_t sf = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xffu;
+            const float d = e4m3_to_f32(sf);
+            uint2 packed = make_uint2(0u, 0u);
+            if (d != 0.0f) {
+                uint32_t w[2] = {0u, 0u};
+#pragma unroll
+                for (int e = 0; e < 16; e += 2)
+                    w[e >> 3] |= cvt_e2m1x2(__fdiv_rn(f[e], d), __fdiv_rn(f[e + 1], d))
+                                 << (4 * (e & 7));
+                packed = make_uint2(w[0], w[1]);
+            }
+            for (int j = 0; j < k; ++j) {
+                const int p = s_p[j];
+                if (p < 0) continue;
+                *reinterpret_cast<uint2 *>(q + (int64_t)p * (H / 2) + g * 8) = packed;
+                scales[(int64_t)s_srow[j] * n16 + g] = (uint8_t)sf;
+            }
+        }
+    }
+}
+
 }  // namespace
 
 // Row split for the bulk dispatch: the number of chunks per row that
@@ -322,6 +397,22 @@ cudaError_t run_dispatch_fp8(const void *x, DType x_dtype, int64_t T, int64_t H,
                       out_perm, offsets, bso, q, scales);
     }
     auto kern = dispatch_fp8_kernel<__half>;
+    const int64_t grid = persistent_grid(kern, kFp8Threads, smem, T);
+    return launch(kern, grid, kFp8Threads, smem, stream, (const __half *)x, T, H, k, E, out_perm,
+                  offsets, bso, q, scales);
+}
+
+cudaError_t run_dispatch_nvfp4(const void *x, DType x_dtype, int64_t T, int64_t H, int k, int E,
+                               const int32_t *out_perm, const int32_t *offsets, const int32_t *bso,
+                               uint8_t *q, uint8_t *scales, cudaStream_t stream) {
+    const size_t smem = (size_t)(2 * E + 1 + 2 * k) * sizeof(int);
+    if (x_dtype == DType::BF16) {
+        auto kern = dispatch_nvfp4_kernel<__nv_bfloat16>;
+        const int64_t grid = persistent_grid(kern, kFp8Threads, smem, T);
+        return launch(kern, grid, kFp8Threads, smem, stream, (const __nv_bfloat16 *)x, T, H, k, E,
+                      out_perm, offsets, bso, q, scales);
+    }
+    auto kern = dispatch_nvfp4_kernel<__half>;
     const int64_t grid = persistent_grid(kern, kFp8Threads, smem, T);
     return launch(kern, grid, kFp8Threads, smem, stream, (const __half *)x, T, H, k, E, out_perm,
                   offsets, bso, q, scales);

@@ -51,6 +51,11 @@ cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int
 cudaError_t run_dispatch_fp8(const void *x, DType x_dtype, int64_t T, int64_t H, int k, int E,
                              const int32_t *out_perm, const int32_t *offsets, const int32_t *bso,
                              uint8_t *q, float *scales, cudaStream_t stream);
+// NVFP4 dispatch: E2M1 codes two per byte ([T*k, H/2]) and one E4M3 scale
+// byte per 16 elements ([rows, H/16], rows placed by the block-scale offsets).
+cudaError_t run_dispatch_nvfp4(const void *x, DType x_dtype, int64_t T, int64_t H, int k, int E,
+                               const int32_t *out_perm, const int32_t *offsets, const int32_t *bso,
+                               uint8_t *q, uint8_t *scales, cudaStream_t stream);
 
 cudaError_t run_output_memset(void *out, int64_t T, int64_t row_bytes, int k,
                               const int32_t *out_perm, cudaStream_t stream);

@@ -91,6 +91,25 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
     return r;
 }
 
+// Two fp32 values -> two FP4 E2M1 codes (round to nearest even, saturating
+// to +-6), `lo` in bits 0..3 and `hi` in bits 4..7.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
+        "cvt.u32.u8 %0, b;\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
+    return r;
+}
+
+// The value of an E4M3 byte, exactly, as fp32 (every E4M3 value is an fp16).
+__device__ __forceinline__ float e4m3_to_f32(uint16_t byte) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(byte));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu)));
+}
+
 // ---------------------------------------------------------------------------
 // Block-wide exclusive scan of n <= 4 * blockDim.x ints held in shared
 // memory (in place).  Returns the total.  All threads must call it.

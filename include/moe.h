@@ -203,6 +203,41 @@ moe_status_t moe_dispatch_rows_fp8(const void *x, moe_dtype_t x_dtype, int64_t n
                                    float *out_scales, moe_stream_t stream);
 
 /*
+ * Dispatch with NVFP4 quantisation (TensorRT-LLM PR #9592: the B200/GB200
+ * NVFP4 MoE path, "run_moe_nvfp4", with scaling_vector_size = 16).  The
+ * pages name the format and the block size only; this library takes the
+ * plain reading of it: one E4M3 scale per 16 consecutive elements of a row,
+ * FP4 E2M1 elements, no per-tensor global scale.  For every valid slot
+ * i = t*k + j with p = output_permutation[i] >= 0, e the expert whose rows
+ * hold p, and every 16-column group g:
+ *
+ *   amax = max |x[t, 16g .. 16g+15]|                 (in fp32)
+ *   sf   = e4m3_rn_satfinite(amax / 6)               (fp32 division)
+ *   d    = the value of sf
+ *   code(c) = e2m1_rn_satfinite(x[t, c] / d)         (fp32 division; 0 if d = 0)
+ *   out_q[p, c/2] holds code(c) in bits 0..3 for even c, bits 4..7 for odd c
+ *   out_scales[blockscale_offsets[e] + p - expert_offsets[e], g] = sf
+ *
+ * E2M1 magnitudes are 0, 0.5, 1, 1.5, 2, 3, 4, 6 (sign in bit 3); rounding is
+ * to nearest, ties to the even code, and magnitudes above 6 saturate.
+ * Rows and scale rows that no valid slot maps to are not written.
+ *
+ *   x          [T, H] BF16 or F16, H a multiple of 16, 16-byte aligned.
+ *   output_permutation [T*k] int32;
+ *   expert_offsets / blockscale_offsets [E+1] int32 (from moe_prepare).
+ *   out_q      [T*k, H/2] uint8, 8-byte aligned;
+ *   out_scales [rows, H/16] uint8 (E4M3 bytes), rows >= blockscale_offsets[E].
+ * Errors: MOE_ERR_UNSUPPORTED for an x type other than BF16/F16;
+ * MOE_ERR_INVALID_ARG for H not a multiple of 16, NULL or misaligned buffers.
+ */
+moe_status_t moe_dispatch_rows_nvfp4(const void *x, moe_dtype_t x_dtype, int64_t num_tokens,
+                                     int64_t hidden, int32_t top_k, int32_t num_experts,
+                                     const int32_t *output_permutation,
+                                     const int32_t *expert_offsets,
+                                     const int32_t *blockscale_offsets, uint8_t *out_q,
+                                     uint8_t *out_scales, moe_stream_t stream);
+
+/*
  * Combine (sglang PR #19058, "Changes", item 3 apply_shuffle_mul_sum:
  * gather + scale + reduce, fp32 accumulation, fp16 / bf16 / fp32):
  *
