@@ -91,6 +91,22 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
     return r;
 }
 
+// a / b rounded to nearest even, given rb = the correctly rounded 1/b
+// (__frcp_rn(b), taken once per divisor).  Markstein's division (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): q0 = RN(a * rb) is within one
+// ulp of a/b, the remainder a - q0*b is exact in one fma, and one fma
+// correction RN(q0 + r*rb) is the correctly rounded quotient, provided that
+// nothing underflows or overflows.  Callers keep b in [2^-60, 2^60] and
+// only use the result where |a/b| >= 2^-12 matters; below that the result
+// still has |value| < 2^-11 and the sign of a.  copysignf keeps the sign of
+// a zero dividend (the fma chain turns -0 into +0).
+__device__ __forceinline__ float div_rn_recip(float a, float b, float rb) {
+    const float q0 = __fmul_rn(a, rb);
+    const float r = __fmaf_rn(-q0, b, a);
+    return copysignf(__fmaf_rn(r, rb, q0), a);
+}
+
 // Two fp32 values -> two FP4 E2M1 codes (round to nearest even, saturating
 // to +-6), `lo` in bits 0..3 and `hi` in bits 4..7.
 __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {

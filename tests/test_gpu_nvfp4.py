@@ -67,13 +67,15 @@ def test_dispatch_nvfp4_vs_oracle(xdt, T, H, E, k, A):
     np.testing.assert_array_equal(sc, sc_ref)
 
 
-@pytest.mark.parametrize("scale_exp", [0, -3, 5])
-def test_dispatch_nvfp4_every_bf16_value(scale_exp):
-    """Every bf16 value of magnitude <= 6 * 2^scale_exp in groups whose amax
-    is exactly 6 * 2^scale_exp, so the scale is the power of two 2^scale_exp
-    and x / d is the value itself scaled: every e2m1 rounding tie, the
-    subnormal step, signed zeros and the saturation edge."""
-    top = 6.0 * 2.0 ** scale_exp
+@pytest.mark.parametrize("mant", range(8, 16))
+@pytest.mark.parametrize("scale_exp", [0, -7, 5])
+def test_dispatch_nvfp4_every_bf16_value(mant, scale_exp):
+    """Every bf16 value of magnitude <= amax in groups whose amax is
+    0.75 * mant * 2^scale_exp, so that amax / 6 is (mant / 8) * 2^scale_exp:
+    each of the 8 scale mantissas (at 2^-7 the odd ones round to the E4M3
+    subnormal grid), and on each every e2m1 rounding tie, the subnormal step, signed zeros and the
+    saturation edge."""
+    top = 0.75 * mant * 2.0 ** scale_exp
     allv = torch.arange(-(2 ** 15), 2 ** 15, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
     v = allv[torch.isfinite(allv.float()) & (allv.float().abs() <= top)]
     per = 15
@@ -93,6 +95,30 @@ def test_dispatch_nvfp4_every_bf16_value(scale_exp):
     q, sc, q_ref, sc_ref = _run(ids_np, 3, x, 1)
     np.testing.assert_array_equal(q, q_ref)
     np.testing.assert_array_equal(sc, sc_ref)
+
+
+def test_dispatch_nvfp4_every_fp16_value():
+    """Every finite fp16 value, in groups with amax 6 * 1.375 (scale
+    mantissa 11) and with amax 448 * 6 * 2 (the scale saturates at 448 and
+    x / d reaches 12: the e2m1 saturation)."""
+    allv = torch.arange(-(2 ** 15), 2 ** 15, dtype=torch.int32).to(torch.int16).view(torch.float16)
+    for top in (6 * 1.375, 448 * 6 * 2):
+        v = allv[torch.isfinite(allv.float()) & (allv.float().abs() <= top)]
+        per = 15
+        ngrp = (v.numel() + per - 1) // per
+        groups = torch.zeros(ngrp, 16, dtype=torch.float16)
+        groups[:, 0] = top
+        flat = groups[:, 1:].reshape(-1)
+        flat[: v.numel()] = v
+        groups[:, 1:] = flat.view(ngrp, per)
+        rows = (ngrp + 63) // 64
+        x = torch.zeros(rows * 64, 16, dtype=torch.float16)
+        x[:ngrp] = groups
+        x = x.view(rows, 16 * 64).to(DEV)
+        ids_np = (np.arange(rows, dtype=np.int32) % 2).reshape(rows, 1)
+        q, sc, q_ref, sc_ref = _run(ids_np, 2, x, 1)
+        np.testing.assert_array_equal(q, q_ref)
+        np.testing.assert_array_equal(sc, sc_ref)
 
 
 def test_dispatch_nvfp4_full_workload_sampled():

@@ -232,6 +232,54 @@ def test_dispatch_fp8_every_bf16_value():
     np.testing.assert_array_equal(sc.view(np.uint32), sc_ref.view(np.uint32))
 
 
+@pytest.mark.parametrize("amax", [417.5, 0.0999755859375, 3.0e15])
+def test_dispatch_fp8_every_bf16_value_odd_scale(amax):
+    """Every bf16 value of magnitude <= amax in 128-blocks whose amax is a
+    value with a non-power-of-two scale amax / 448: x / s is then a general
+    fp32 quotient, so this checks the correctly rounded division on every
+    bf16 dividend against the oracle's."""
+    allv = torch.arange(-(2 ** 15), 2 ** 15, dtype=torch.int32).to(torch.int16).view(torch.bfloat16)
+    v = allv[torch.isfinite(allv.float()) & (allv.float().abs() <= amax)]
+    per = 127
+    nblk = (v.numel() + per - 1) // per
+    blocks = torch.zeros(nblk, 128, dtype=torch.bfloat16)
+    blocks[:, 0] = amax
+    flat = blocks[:, 1:].reshape(-1)
+    flat[: v.numel()] = v
+    blocks[:, 1:] = flat.view(nblk, per)
+    rows = (nblk + 15) // 16
+    x = torch.zeros(rows * 16, 128, dtype=torch.bfloat16)
+    x[:nblk] = blocks
+    x = x.view(rows, 128 * 16).to(DEV)
+    T = x.shape[0]
+    ids_np = (np.arange(T, dtype=np.int32) % 3).reshape(T, 1)
+    q, sc, q_ref, sc_ref = _fp8_run(ids_np, 3, x, 1)
+    np.testing.assert_array_equal(q, q_ref)
+    np.testing.assert_array_equal(sc.view(np.uint32), sc_ref.view(np.uint32))
+
+
+def test_dispatch_fp8_extreme_scales():
+    """Blocks whose scale amax / 448 lies near and beyond 2^-60 and 2^60
+    (the range where the quotient takes the one-reciprocal route), with
+    random values and signed zeros inside them; all finite (2^110 * 448 is
+    below the bf16 maximum), since the contract is for finite activations."""
+    T, H = 64, 128 * 12
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(T, H, generator=g)
+    exps = torch.tensor([-130, -80, -62, -61, -60, -59, -20, 0, 20, 59, 60, 61, 62, 70, 100, 110],
+                        dtype=torch.float32)
+    blk = x.view(T, 12, 128)
+    e = exps[torch.randint(0, exps.numel(), (T, 12), generator=g)]
+    blk *= (2.0 ** e)[:, :, None] * 448.0 / blk.abs().amax(dim=2, keepdim=True)
+    x = blk.view(T, H)
+    x[:, 5::17] = -0.0
+    x = x.to(torch.bfloat16)
+    ids_np = (np.arange(T, dtype=np.int32) % 4).reshape(T, 1)
+    q, sc, q_ref, sc_ref = _fp8_run(ids_np, 4, x.to(DEV), 1)
+    np.testing.assert_array_equal(q, q_ref)
+    np.testing.assert_array_equal(sc.view(np.uint32), sc_ref.view(np.uint32))
+
+
 def test_dispatch_fp8_full_workload_sampled():
     w = CONFIGS["zipf_fp8_t16384_h4096_e288_k8"]
     ids_np, _, x, _ = make_workload(w, device=DEV, with_y=False)
