@@ -34,6 +34,8 @@ constexpr int kCopyUnroll = 8;  // 16-byte vectors in flight per thread
 // ---------------------------------------------------------------------------
 constexpr int kBulkMaxStages = 16;
 constexpr uint32_t kBulkSmem = 64 * 1024;   // stage ring per block
+constexpr int kQuantThreads = 256;          // quantised dispatch: target threads per block
+constexpr int kQuantMaxThreads = 512;       // and the most
 constexpr uint32_t kMaxPolls = 1u << 24;    // bounded mbarrier wait (each poll suspends briefly)
 
 __device__ unsigned g_dispatch_error;  // set when a bounded wait gave up
@@ -166,7 +168,6 @@ __global__ void __launch_bounds__(kCopyThreads)
 // stores s into the scale segment of the row's expert (found from the expert
 // offsets, so the kernel needs no ids).
 // ---------------------------------------------------------------------------
-constexpr int kFp8Threads = 256;
 
 template <typename XT>
 __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
@@ -175,174 +176,206 @@ __device__ __forceinline__ void unpack8(const uint4 &v, float *f) {
     for (int e = 0; e < 8; ++e) f[e] = Elem<XT>::to_f32(h[e]);
 }
 
-template <typename XT>
-__global__ void __launch_bounds__(kFp8Threads)
-    dispatch_fp8_kernel(const XT *__restrict__ x, int64_t T, int64_t H, int k, int E,
-                        const int32_t *__restrict__ out_perm, const int32_t *__restrict__ offsets,
-                        const int32_t *__restrict__ bso, uint8_t *__restrict__ q,
-                        float *__restrict__ scales) {
-    extern __shared__ int smem[];
-    int *s_off = smem;             // [E+1] expert offsets
-    int *s_delta = s_off + E + 1;  // [E] scale row - dispatched row, per expert
-    int *s_p = s_delta + E;        // [k] this token's dispatched rows
-    int *s_srow = s_p + k;         // [k] and their scale rows
-    pdl_wait();
-    pdl_launch_dependents();
-    for (int e = threadIdx.x; e <= E; e += kFp8Threads) {
+// FP8 E4M3 1x128 block quantisation of one 16-element group f (columns
+// 16g .. 16g+15).  The 8 groups of a 128-column block sit in 8 consecutive
+// lanes that are active together; `lanes` is the mask of the lanes of this
+// warp still in the row loop.  Returns the 16 E4M3 bytes; *scale = amax/448.
+__device__ __forceinline__ uint4 quant_fp8_group(const float *f, unsigned lanes, float *scale) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
+    amax = fmaxf(amax, __shfl_xor_sync(lanes, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(lanes, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(lanes, amax, 4));
+    uint4 packed = make_uint4(0u, 0u, 0u, 0u);
+    float s = 0.0f;
+    if (amax != 0.0f) {
+        s = __fdiv_rn(amax, 448.0f);
+        uint32_t w[4];
+        if (s >= 0x1p-60f && s <= 0x1p60f) {
+            // one reciprocal per block, three flops per element;
+            // bit-identical to x / s (div_rn_recip)
+            const float rs = __frcp_rn(s);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint16_t lo = cvt_e4m3x2(div_rn_recip(f[4 * e], s, rs),
+                                               div_rn_recip(f[4 * e + 1], s, rs));
+                const uint16_t hi = cvt_e4m3x2(div_rn_recip(f[4 * e + 2], s, rs),
+                                               div_rn_recip(f[4 * e + 3], s, rs));
+                w[e] = (uint32_t)lo | ((uint32_t)hi << 16);
+            }
+        } else {  // scales near the ends of the fp32 range
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint16_t lo = cvt_e4m3x2(__fdiv_rn(f[4 * e], s), __fdiv_rn(f[4 * e + 1], s));
+                const uint16_t hi =
+                    cvt_e4m3x2(__fdiv_rn(f[4 * e + 2], s), __fdiv_rn(f[4 * e + 3], s));
+                w[e] = (uint32_t)lo | ((uint32_t)hi << 16);
+            }
+        }
+        packed = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    *scale = s;
+    return packed;
+}
+
+// NVFP4 quantisation of one 16-element group: the E4M3 scale
+// sf = e4m3(amax / 6) and the 16 E2M1 codes of x / value(sf), element 2m in
+// the low nibble of byte m.  Returns the 8 code bytes; *sf_out = sf.
+__device__ __forceinline__ uint2 quant_nvfp4_group(const float *f, uint8_t *sf_out) {
+    float amax = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
+    const uint16_t sf = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xffu;
+    const float d = e4m3_to_f32(sf);
+    uint2 packed = make_uint2(0u, 0u);
+    if (d != 0.0f) {  // d is an E4M3 value: in [2^-9, 448]
+        const float rd = __frcp_rn(d);
+        uint32_t w[2] = {0u, 0u};
+#pragma unroll
+        for (int e = 0; e < 16; e += 2)
+            w[e >> 3] |= cvt_e2m1x2(div_rn_recip(f[e], d, rd), div_rn_recip(f[e + 1], d, rd))
+                         << (4 * (e & 7));
+        packed = make_uint2(w[0], w[1]);
+    }
+    *sf_out = (uint8_t)sf;
+    return packed;
+}
+
+// Lanes of this warp still in a loop over groups g = threadIdx.x + i*blockDim.x
+// < n (blockDim.x a multiple of 32): all of them, or those below the row end.
+__device__ __forceinline__ unsigned lanes_in_row(int64_t g, int64_t n) {
+    const int64_t rem = n - (g - (threadIdx.x & 31));
+    return rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+}
+
+// Stages the expert offsets and (block-scale row - dispatched row) per
+// expert, then for token t resolves its k dispatched rows and their scale
+// rows into s_p / s_srow (-1 for slots with no row).  Threads j < k write.
+__device__ __forceinline__ void stage_offsets(const int32_t *offsets, const int32_t *bso, int E,
+                                              int *s_off, int *s_delta) {
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
         s_off[e] = __ldg(offsets + e);
         if (e < E) s_delta[e] = __ldg(bso + e) - __ldg(offsets + e);
     }
-    const int64_t n16 = H / 16;  // 16-element groups per row
-    const int64_t nb = H / 128;
-    const int64_t S = T * k;
-    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        __syncthreads();  // offsets staged; the previous token's rows consumed
-        for (int j = threadIdx.x; j < k; j += kFp8Threads) {
-            int p = __ldg(out_perm + t * k + j);
-            int srow = -1;
-            if (p >= 0 && p < S && p < s_off[E]) {
-                int lo = 0, hi = E;  // the expert whose rows hold p
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (s_off[mid] <= p) lo = mid;
-                    else hi = mid;
-                }
-                srow = p + s_delta[lo];
-            } else {
-                p = -1;
+}
+
+__device__ __forceinline__ void resolve_rows(const int32_t *out_perm, int64_t t, int k, int64_t S,
+                                             int E, const int *s_off, const int *s_delta,
+                                             int *s_p, int *s_srow) {
+    for (int j = threadIdx.x; j < k; j += blockDim.x) {
+        int p = __ldg(out_perm + t * k + j);
+        int srow = -1;
+        if (p >= 0 && p < S && p < s_off[E]) {
+            int lo = 0, hi = E;  // the expert whose rows hold p
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (s_off[mid] <= p) lo = mid;
+                else hi = mid;
             }
-            s_p[j] = p;
-            s_srow[j] = srow;
+            srow = p + s_delta[lo];
+        } else {
+            p = -1;
         }
-        __syncthreads();
-        for (int64_t g = threadIdx.x; g < n16; g += kFp8Threads) {
-            const XT *src = x + t * H + g * 16;
-            float f[16];
-            unpack8<XT>(ld_stream_v4(src), f);
-            unpack8<XT>(ld_stream_v4(src + 8), f + 8);
-            float amax = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
-            // the 8 groups of one 128-column block are 8 consecutive lanes,
-            // active together (H is a multiple of 128); lanes past the row
-            // end have left the loop
-            const int64_t rem = n16 - (g - (threadIdx.x & 31));
-            const unsigned m = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
-            amax = fmaxf(amax, __shfl_xor_sync(m, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(m, amax, 2));
-            amax = fmaxf(amax, __shfl_xor_sync(m, amax, 4));
-            uint4 packed = make_uint4(0u, 0u, 0u, 0u);
-            float s = 0.0f;
-            if (amax != 0.0f) {
-                s = __fdiv_rn(amax, 448.0f);
-                uint32_t w[4];
-                if (s >= 0x1p-60f && s <= 0x1p60f) {
-                    // one reciprocal per block, three flops per element;
-                    // bit-identical to x / s (div_rn_recip)
-                    const float rs = __frcp_rn(s);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint16_t lo = cvt_e4m3x2(div_rn_recip(f[4 * e], s, rs),
-                                                       div_rn_recip(f[4 * e + 1], s, rs));
-                        const uint16_t hi = cvt_e4m3x2(div_rn_recip(f[4 * e + 2], s, rs),
-                                                       div_rn_recip(f[4 * e + 3], s, rs));
-                        w[e] = (uint32_t)lo | ((uint32_t)hi << 16);
-                    }
-                } else {  // scales near the ends of the fp32 range
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const uint16_t lo =
-                            cvt_e4m3x2(__fdiv_rn(f[4 * e], s), __fdiv_rn(f[4 * e + 1], s));
-                        const uint16_t hi =
-                            cvt_e4m3x2(__fdiv_rn(f[4 * e + 2], s), __fdiv_rn(f[4 * e + 3], s));
-                        w[e] = (uint32_t)lo | ((uint32_t)hi << 16);
-                    }
-                }
-                packed = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            const bool block_lead = (g & 7) == 0;
-            const int64_t b = g >> 3;
-            for (int j = 0; j < k; ++j) {
-                const int p = s_p[j];
-                if (p < 0) continue;
-                st_v4(q + (int64_t)p * H + g * 16, packed);
-                if (block_lead) scales[(int64_t)s_srow[j] * nb + b] = s;
-            }
+        s_p[j] = p;
+        s_srow[j] = srow;
+    }
+}
+
+// Quantised dispatch.  A block walks tokens; each thread owns one or two
+// 16-element groups of the row (longer rows: a loop over groups).  Per
+// group: the quantiser, then its code bytes stored to each of the k
+// dispatched rows, plus the scale from the lane that leads its scale block.
+template <typename XT, bool kFp4>
+__device__ __forceinline__ void quant_store_group(const uint4 &raw0, const uint4 &raw1, int64_t g,
+                                                  int64_t n16, int64_t qrow, int64_t srow_len,
+                                                  int k, const int *s_p, const int *s_srow,
+                                                  uint8_t *__restrict__ q, void *__restrict__ scales) {
+    float f[16];
+    unpack8<XT>(raw0, f);
+    unpack8<XT>(raw1, f + 8);
+    if constexpr (kFp4) {
+        uint8_t sf;
+        const uint2 packed = quant_nvfp4_group(f, &sf);
+        for (int j = 0; j < k; ++j) {
+            const int p = s_p[j];
+            if (p < 0) continue;
+            *reinterpret_cast<uint2 *>(q + (int64_t)p * qrow + g * 8) = packed;
+            static_cast<uint8_t *>(scales)[(int64_t)s_srow[j] * srow_len + g] = sf;
+        }
+    } else {
+        float sc;
+        const uint4 packed = quant_fp8_group(f, lanes_in_row(g, n16), &sc);
+        const bool block_lead = (g & 7) == 0;
+        for (int j = 0; j < k; ++j) {
+            const int p = s_p[j];
+            if (p < 0) continue;
+            st_v4(q + (int64_t)p * qrow + g * 16, packed);
+            if (block_lead)
+                static_cast<float *>(scales)[(int64_t)s_srow[j] * srow_len + (g >> 3)] = sc;
         }
     }
 }
 
-
-// NVFP4 dispatch.  A block walks tokens; per token it resolves the k
-// dispatched rows and their scale rows once (from the expert offsets staged
-// in shared memory), then each thread takes 16-element groups of the row:
-// two 16-byte loads, the group amax, its E4M3 scale sf = e4m3(amax / 6), and
-// the 16 E2M1 codes of x / value(sf), stored as 8 bytes to each of the k
-// rows (a warp writes 256 contiguous bytes of a row) plus the scale byte.
-template <typename XT>
-__global__ void __launch_bounds__(kFp8Threads)
-    dispatch_nvfp4_kernel(const XT *__restrict__ x, int64_t T, int64_t H, int k, int E,
+template <typename XT, bool kFp4, int kG>
+__global__ void __launch_bounds__(kQuantMaxThreads)
+    dispatch_quant_kernel(const XT *__restrict__ x, int64_t T, int64_t H, int k, int E,
                           const int32_t *__restrict__ out_perm, const int32_t *__restrict__ offsets,
                           const int32_t *__restrict__ bso, uint8_t *__restrict__ q,
-                          uint8_t *__restrict__ scales) {
+                          void *__restrict__ scales) {
     extern __shared__ int smem[];
     int *s_off = smem;             // [E+1] expert offsets
     int *s_delta = s_off + E + 1;  // [E] scale row - dispatched row, per expert
     int *s_p = s_delta + E;        // [k] this token's dispatched rows
     int *s_srow = s_p + k;         // [k] and their scale rows
+    const int64_t n16 = H / 16;  // 16-element groups per row
+    const int64_t S = T * k;
+    const int64_t qrow = kFp4 ? H / 2 : H;
+    const int64_t srow_len = kFp4 ? n16 : H / 128;  // scale elements per row
+    const int64_t nt = blockDim.x;
+    // kG > 0: the row has at most kG * blockDim.x groups; thread i owns
+    // groups i + r * blockDim.x (r < kG) of every token, and loads the next
+    // token's while this one's are quantised and stored.
+    uint4 nxt[kG > 0 ? 2 * kG : 1];
+    auto prefetch = [&](int64_t t) {
+#pragma unroll
+        for (int r = 0; r < kG; ++r) {
+            const int64_t g = threadIdx.x + r * nt;
+            if (g < n16 && t < T) {
+                const XT *src = x + t * H + g * 16;
+                nxt[2 * r] = ld_stream_v4(src);
+                nxt[2 * r + 1] = ld_stream_v4(src + 8);
+            }
+        }
+    };
     pdl_wait();
     pdl_launch_dependents();
-    for (int e = threadIdx.x; e <= E; e += kFp8Threads) {
-        s_off[e] = __ldg(offsets + e);
-        if (e < E) s_delta[e] = __ldg(bso + e) - __ldg(offsets + e);
-    }
-    const int64_t n16 = H / 16;  // groups per row = scale bytes per row
-    const int64_t S = T * k;
+    if constexpr (kG > 0) prefetch(blockIdx.x);
+    stage_offsets(offsets, bso, E, s_off, s_delta);
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        __syncthreads();  // offsets staged; the previous token's rows consumed
-        for (int j = threadIdx.x; j < k; j += kFp8Threads) {
-            int p = __ldg(out_perm + t * k + j);
-            int srow = -1;
-            if (p >= 0 && p < S && p < s_off[E]) {
-                int lo = 0, hi = E;  // the expert whose rows hold p
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (s_off[mid] <= p) lo = mid;
-                    else hi = mid;
-                }
-                srow = p + s_delta[lo];
-            } else {
-                p = -1;
-            }
-            s_p[j] = p;
-            s_srow[j] = srow;
-        }
-        __syncthreads();
-        for (int64_t g = threadIdx.x; g < n16; g += kFp8Threads) {
-            const XT *src = x + t * H + g * 16;
-            float f[16];
-            unpack8<XT>(ld_stream_v4(src), f);
-            unpack8<XT>(ld_stream_v4(src + 8), f + 8);
-            float amax = 0.0f;
+        if constexpr (kG > 0) {
+            uint4 cur[2 * kG];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) amax = fmaxf(amax, fabsf(f[e]));
-            const uint16_t sf = cvt_e4m3x2(__fdiv_rn(amax, 6.0f), 0.0f) & 0xffu;
-            const float d = e4m3_to_f32(sf);
-            uint2 packed = make_uint2(0u, 0u);
-            if (d != 0.0f) {  // d is an E4M3 value: in [2^-9, 448]
-                const float rd = __frcp_rn(d);
-                uint32_t w[2] = {0u, 0u};
+            for (int r = 0; r < 2 * kG; ++r) cur[r] = nxt[r];
+            prefetch(t + gridDim.x);  // in flight while this token is stored
+            __syncthreads();  // offsets staged; the previous token's rows consumed
+            resolve_rows(out_perm, t, k, S, E, s_off, s_delta, s_p, s_srow);
+            __syncthreads();
 #pragma unroll
-                for (int e = 0; e < 16; e += 2)
-                    w[e >> 3] |= cvt_e2m1x2(div_rn_recip(f[e], d, rd), div_rn_recip(f[e + 1], d, rd))
-                                 << (4 * (e & 7));
-                packed = make_uint2(w[0], w[1]);
+            for (int r = 0; r < kG; ++r) {
+                const int64_t g = threadIdx.x + r * nt;
+                if (g < n16)
+                    quant_store_group<XT, kFp4>(cur[2 * r], cur[2 * r + 1], g, n16, qrow, srow_len,
+                                                k, s_p, s_srow, q, scales);
             }
-            for (int j = 0; j < k; ++j) {
-                const int p = s_p[j];
-                if (p < 0) continue;
-                *reinterpret_cast<uint2 *>(q + (int64_t)p * (H / 2) + g * 8) = packed;
-                scales[(int64_t)s_srow[j] * n16 + g] = (uint8_t)sf;
+        } else {
+            __syncthreads();
+            resolve_rows(out_perm, t, k, S, E, s_off, s_delta, s_p, s_srow);
+            __syncthreads();
+            for (int64_t g = threadIdx.x; g < n16; g += nt) {
+                const XT *src = x + t * H + g * 16;
+                quant_store_group<XT, kFp4>(ld_stream_v4(src), ld_stream_v4(src + 8), g, n16, qrow,
+                                            srow_len, k, s_p, s_srow, q, scales);
             }
         }
     }
@@ -402,36 +435,48 @@ cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int
                   nvec, k, in_perm, (uint4 *)out);
 }
 
+// Quantised dispatch launcher.  Rows of up to 2 * kQuantThreads groups:
+// kG = ceil(groups / kQuantThreads) groups per thread (1 or 2) and
+// ceil(groups / kG) threads rounded up to a multiple of 32 (so that the 8
+// groups of an FP8 128-column block share a warp).  Longer rows: a plain
+// loop without the prefetch.
+template <typename XT, bool kFp4>
+static cudaError_t run_dispatch_quant_t(const XT *x, int64_t T, int64_t H, int k, int E,
+                                        const int32_t *out_perm, const int32_t *offsets,
+                                        const int32_t *bso, uint8_t *q, void *scales,
+                                        cudaStream_t stream) {
+    const int64_t n16 = H / 16;
+    const size_t smem = (size_t)(2 * E + 1 + 2 * k) * sizeof(int);
+    auto go = [&](auto kern, int64_t per_thread) {
+        int64_t threads = ((n16 + per_thread - 1) / per_thread + 31) / 32 * 32;
+        if (threads > kQuantMaxThreads) threads = kQuantMaxThreads;
+        const int64_t grid = persistent_grid(kern, (int)threads, smem, T);
+        return launch(kern, grid, (int)threads, smem, stream, x, T, H, k, E, out_perm, offsets,
+                      bso, q, scales);
+    };
+    if (n16 <= kQuantThreads) return go(dispatch_quant_kernel<XT, kFp4, 1>, 1);
+    if (n16 <= 2 * kQuantThreads) return go(dispatch_quant_kernel<XT, kFp4, 2>, 2);
+    return go(dispatch_quant_kernel<XT, kFp4, 0>, (n16 + kQuantMaxThreads - 1) / kQuantMaxThreads);
+}
+
 cudaError_t run_dispatch_fp8(const void *x, DType x_dtype, int64_t T, int64_t H, int k, int E,
                              const int32_t *out_perm, const int32_t *offsets, const int32_t *bso,
                              uint8_t *q, float *scales, cudaStream_t stream) {
-    const size_t smem = (size_t)(2 * E + 1 + 2 * k) * sizeof(int);
-    if (x_dtype == DType::BF16) {
-        auto kern = dispatch_fp8_kernel<__nv_bfloat16>;
-        const int64_t grid = persistent_grid(kern, kFp8Threads, smem, T);
-        return launch(kern, grid, kFp8Threads, smem, stream, (const __nv_bfloat16 *)x, T, H, k, E,
-                      out_perm, offsets, bso, q, scales);
-    }
-    auto kern = dispatch_fp8_kernel<__half>;
-    const int64_t grid = persistent_grid(kern, kFp8Threads, smem, T);
-    return launch(kern, grid, kFp8Threads, smem, stream, (const __half *)x, T, H, k, E, out_perm,
-                  offsets, bso, q, scales);
+    if (x_dtype == DType::BF16)
+        return run_dispatch_quant_t<__nv_bfloat16, false>((const __nv_bfloat16 *)x, T, H, k, E,
+                                                          out_perm, offsets, bso, q, scales, stream);
+    return run_dispatch_quant_t<__half, false>((const __half *)x, T, H, k, E, out_perm, offsets,
+                                               bso, q, scales, stream);
 }
 
 cudaError_t run_dispatch_nvfp4(const void *x, DType x_dtype, int64_t T, int64_t H, int k, int E,
                                const int32_t *out_perm, const int32_t *offsets, const int32_t *bso,
                                uint8_t *q, uint8_t *scales, cudaStream_t stream) {
-    const size_t smem = (size_t)(2 * E + 1 + 2 * k) * sizeof(int);
-    if (x_dtype == DType::BF16) {
-        auto kern = dispatch_nvfp4_kernel<__nv_bfloat16>;
-        const int64_t grid = persistent_grid(kern, kFp8Threads, smem, T);
-        return launch(kern, grid, kFp8Threads, smem, stream, (const __nv_bfloat16 *)x, T, H, k, E,
-                      out_perm, offsets, bso, q, scales);
-    }
-    auto kern = dispatch_nvfp4_kernel<__half>;
-    const int64_t grid = persistent_grid(kern, kFp8Threads, smem, T);
-    return launch(kern, grid, kFp8Threads, smem, stream, (const __half *)x, T, H, k, E, out_perm,
-                  offsets, bso, q, scales);
+    if (x_dtype == DType::BF16)
+        return run_dispatch_quant_t<__nv_bfloat16, true>((const __nv_bfloat16 *)x, T, H, k, E,
+                                                         out_perm, offsets, bso, q, scales, stream);
+    return run_dispatch_quant_t<__half, true>((const __half *)x, T, H, k, E, out_perm, offsets, bso,
+                                              q, scales, stream);
 }
 
 cudaError_t run_output_memset(void *out, int64_t T, int64_t row_bytes, int k,

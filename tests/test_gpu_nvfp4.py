@@ -149,6 +149,32 @@ def test_dispatch_nvfp4_full_workload_sampled():
     np.testing.assert_array_equal(sc[torch.from_numpy(srow).long().to(DEV)].cpu().numpy(), sc_sub)
 
 
+@pytest.mark.parametrize("H", [4096, 7168])
+def test_dispatch_nvfp4_plain_store_path(H):
+    """Outputs that are 8- but not 16-byte aligned take the plain-store
+    kernel instead of the bulk-store one; same bytes."""
+    T, E, k, A = 150, 64, 6, 4
+    rng = np.random.default_rng(H)
+    ids_np = _ids(rng, T, k, E, p_invalid=0.02)
+    x = torch.randn(T, H, device=DEV).to(torch.bfloat16)
+    meta = moe.moe_prepare(torch.from_numpy(ids_np).to(DEV), E, blockscale_align=A)
+    rows = T * k + E * (A - 1)
+    qbuf = torch.full((T * k * (H // 2) + 8,), 0xAB, dtype=torch.uint8, device=DEV)
+    sbuf = torch.full((rows * (H // 16) + 8,), 0xCD, dtype=torch.uint8, device=DEV)
+    q = qbuf[8:].view(T * k, H // 2)
+    sc = sbuf[8:].view(rows, H // 16)
+    assert q.data_ptr() % 16 == 8
+    moe.moe_dispatch_rows_nvfp4(x, k, meta.output_permutation, meta.expert_offsets,
+                                meta.blockscale_offsets, out_q=q, out_scales=sc)
+    torch.cuda.synchronize()
+    ref_meta = oracle.prepare(ids_np, E, A)
+    q_ref = np.full((T * k, H // 2), 0xAB, np.uint8)
+    sc_ref = np.full((rows, H // 16), 0xCD, np.uint8)
+    oracle.dispatch_nvfp4(bits(x), "bf16", ids_np, ref_meta, q_ref, sc_ref)
+    np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
+    np.testing.assert_array_equal(sc.cpu().numpy(), sc_ref)
+
+
 def test_dispatch_nvfp4_validation():
     lib = moe._lib.load()
     x = torch.zeros(4, 24, dtype=torch.bfloat16, device=DEV)

@@ -280,6 +280,30 @@ def test_dispatch_fp8_extreme_scales():
     np.testing.assert_array_equal(sc.view(np.uint32), sc_ref.view(np.uint32))
 
 
+def test_dispatch_fp8_plain_store_path():
+    """Scales that are 4- but not 16-byte aligned take the plain-store kernel
+    instead of the bulk-store one; same bytes."""
+    T, H, E, k, A = 150, 4096, 64, 6, 4
+    rng = np.random.default_rng(11)
+    ids_np = _ids_random(rng, T, k, E, p_invalid=0.02)
+    x = torch.randn(T, H, device=DEV).to(torch.bfloat16)
+    meta = moe.moe_prepare(torch.from_numpy(ids_np).to(DEV), E, blockscale_align=A)
+    rows = T * k + E * (A - 1)
+    q = torch.full((T * k, H), 0xAB, dtype=torch.uint8, device=DEV)
+    sbuf = torch.full((rows * (H // 128) + 1,), float("nan"), device=DEV)
+    sc = sbuf[1:].view(rows, H // 128)
+    assert sc.data_ptr() % 16 == 4
+    moe.moe_dispatch_rows_fp8(x, k, meta.output_permutation, meta.expert_offsets,
+                              meta.blockscale_offsets, out_q=q, out_scales=sc)
+    torch.cuda.synchronize()
+    ref_meta = oracle.prepare(ids_np, E, A)
+    q_ref = np.full((T * k, H), 0xAB, np.uint8)
+    sc_ref = np.full((rows, H // 128), np.nan, np.float32)
+    oracle.dispatch_fp8(bits(x), "bf16", ids_np, ref_meta, q_ref, sc_ref)
+    np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
+    np.testing.assert_array_equal(sc.cpu().numpy().view(np.uint32), sc_ref.view(np.uint32))
+
+
 def test_dispatch_fp8_full_workload_sampled():
     w = CONFIGS["zipf_fp8_t16384_h4096_e288_k8"]
     ids_np, _, x, _ = make_workload(w, device=DEV, with_y=False)
