@@ -11,16 +11,19 @@
 // per-warp counts, and across blocks by one of:
 //  * up to kSingleBlockSlots slots: nothing, one block does it all
 //    (prep_single_kernel);
-//  * above that, tiles of kTileSlots slots over the whole GPU:
-//    prep_rank_kernel ranks each tile, then runs a decoupled look-back over
-//    the tiles' per-expert aggregates (bounded waits, a window of
-//    predecessors read together) and stores rank(i) in output_permutation;
-//    the last tile holds the totals and writes counts and offsets.
-//    prep_finish_kernel, element-wise, adds the expert offset and writes both
+//  * above that, tiles of kTileSlots slots: each tile ranks its slots,
+//    publishes its per-expert aggregates and runs a decoupled look-back over
+//    the earlier tiles (bounded waits, a window of predecessors read
+//    together); the last tile holds the totals and writes counts and
+//    offsets.  When every tile fits on the GPU at once this is one
+//    cooperative launch (prep_onepass_kernel: the tiles wait, bounded, for
+//    the last one's offsets and write both permutations); otherwise
+//    prep_rank_kernel stores rank(i) in output_permutation and the
+//    element-wise prep_finish_kernel adds the expert offset and writes both
 //    permutations.  Tiles take their index from an atomic ticket, so a tile
 //    only ever waits on tiles that are already running; a wait that gives up
-//    reports through diag[1]; the ticket wraps to zero and the finish kernel
-//    clears every look-back word, so the workspace is all-zero between calls.
+//    reports through diag[1].  Look-back words carry the epoch of the call
+//    that wrote them, so the workspace needs zeroing once, not per call.
 #include "kernels.h"
 #include "launch.h"
 #include "moe_device.cuh"
