@@ -133,6 +133,28 @@ def test_dispatch_fp8_validation(lib):
     assert call(T=0, x=None) == OK
 
 
+def test_dispatch_nvfp4_validation(lib):
+    f = lib.moe_dispatch_rows_nvfp4
+    args = dict(x=P, dt=BF16, T=4, H=256, k=2, E=8, op=P, off=P, bso=P, q=P, sc=P)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(a["x"], a["dt"], a["T"], a["H"], a["k"], a["E"], a["op"], a["off"], a["bso"],
+                 a["q"], a["sc"], None)
+
+    assert call(dt=F32) == UNSUPPORTED
+    assert call(dt=FP8) == UNSUPPORTED
+    assert call(H=24) == INVALID                                     # H % 16 != 0
+    assert call(H=0) == INVALID
+    assert call(E=0) == INVALID
+    assert call(k=0) == INVALID
+    for key in ("x", "op", "off", "bso", "q", "sc"):
+        assert call(**{key: None}) == INVALID, key
+    assert call(x=P + 8) == INVALID                                  # x needs 16 bytes
+    assert call(q=P + 4) == INVALID                                  # codes need 8 bytes
+    assert call(T=0, x=None, q=None) == OK
+
+
 def test_prepare_local_and_memset_validation(lib):
     pl = lib.moe_prepare_local
     assert pl(P, 2, 4, 2, 0, 8, P, P, None, 1, P, P, None, None, 0, None) == INVALID   # bad id type
