@@ -16,10 +16,7 @@ inline int dtype_bytes(DType d) {
 // Prepare: a problem with at most kSingleBlockSlots slots runs as one block;
 // larger ones as tiles of kTileSlots slots over the whole GPU.
 constexpr int kSingleBlockSlots = 4096;
-constexpr int kTileThreads = 256;
-constexpr int kTileWarps = kTileThreads / 32;
-constexpr int kTileRounds = 8;  // rounds of 32 slots per warp
-constexpr int kTileSlots = kTileThreads * kTileRounds;
+constexpr int kTileSlots = 2048;  // slots per tile
 constexpr int kMaxExperts = 1024;
 constexpr int kFusedMaxSlots = 4096;
 

@@ -11,19 +11,20 @@
 // per-warp counts, and across blocks by one of:
 //  * up to kSingleBlockSlots slots: nothing, one block does it all
 //    (prep_single_kernel);
-//  * above that, tiles of kTileSlots slots: each tile ranks its slots,
-//    publishes its per-expert aggregates and runs a decoupled look-back over
-//    the earlier tiles (bounded waits, a window of predecessors read
+//  * above that, tiles of kTileSlots slots, each ranked by one block, which
+//    publishes its per-expert histogram and runs a decoupled look-back over
+//    the earlier tiles' (bounded waits, a window of predecessors read
 //    together); the last tile holds the totals and writes counts and
 //    offsets.  When every tile fits on the GPU at once this is one
-//    cooperative launch (prep_onepass_kernel: the tiles wait, bounded, for
-//    the last one's offsets and write both permutations); otherwise
-//    prep_rank_kernel stores rank(i) in output_permutation and the
-//    element-wise prep_finish_kernel adds the expert offset and writes both
-//    permutations.  Tiles take their index from an atomic ticket, so a tile
-//    only ever waits on tiles that are already running; a wait that gives up
-//    reports through diag[1].  Look-back words carry the epoch of the call
-//    that wrote them, so the workspace needs zeroing once, not per call.
+//    cooperative launch (prep_onepass_kernel, 512-thread tiles, tile =
+//    block index): the other tiles wait, bounded, for the last one's offsets
+//    and write both permutations.  Otherwise prep_rank_kernel (256-thread
+//    tiles, two per SM) takes tiles by an atomic ticket, so a tile only ever
+//    waits on tiles already running, and stores rank(i) in
+//    output_permutation; the element-wise prep_finish_kernel then adds the
+//    expert offset and writes both permutations.  A wait that gives up
+//    reports through diag[1].  Words in the workspace carry the epoch of the
+//    call that wrote them, so the workspace needs zeroing once, not per call.
 #include "kernels.h"
 #include "launch.h"
 #include "moe_device.cuh"
@@ -269,52 +270,40 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
 size_t single_block_smem(int E) { return (size_t)(kSingleWarps * (E + 1) + 2 * E) * sizeof(int); }
 
 // ---------------------------------------------------------------------------
-// Tiled path.  tile_rank_lookback() is the part both variants share: take a
-// tile ticket, rank the tile's slots within each warp's run, fold the warps
-// into the tile histogram, publish it and look back over the earlier tiles.
-// On return (after a block barrier) excl[c] holds the slots of column c in
-// earlier tiles, hist[c] this tile's, wcnt the per-warp exclusive prefixes,
-// and key/rank each thread's slots.
+// Tiled path.  A tile is kTileSlots consecutive slots, ranked by a block of
+// NT threads (NT / 32 warps, kTileSlots / NT rounds of 32 slots per warp).
+// tile_rank() ranks a tile's slots within each warp's run and folds the warps
+// into the tile histogram: hist[c] for c < E is the tile's count of expert c,
+// hist[E] its count of invalid ids; wcnt holds the per-warp exclusive
+// prefixes and key/rank each thread's slots.
 // ---------------------------------------------------------------------------
-struct TileCtx {
-    int tile;
-    unsigned epoch;
-    int64_t wbase;  // first slot of this warp's run
+template <int NT> struct TileShape {
+    static constexpr int kThreads = NT;
+    static constexpr int kWarps = NT / 32;
+    static constexpr int kRounds = kTileSlots / NT;
+    static_assert(NT * kRounds == kTileSlots, "a tile is kTileSlots slots");
 };
 
-template <typename IdT>
-__device__ __forceinline__ TileCtx tile_rank_lookback(
-    const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int G, const PrepWs &ws, int *wcnt,
-    int *hist, int *excl, unsigned *s_misc, int *s_invalid, int (&key)[kTileRounds],
-    int (&rank)[kTileRounds]) {
-    const int C = E + 1;  // one column per expert plus one for invalid ids
+template <typename IdT, int NT>
+__device__ __forceinline__ void tile_rank(const IdT *__restrict__ ids, int64_t base, int64_t S,
+                                          int E, int tile, int *wcnt, int *hist, int *s_invalid,
+                                          int (&key)[TileShape<NT>::kRounds],
+                                          int (&rank)[TileShape<NT>::kRounds]) {
+    constexpr int NW = TileShape<NT>::kWarps, NR = TileShape<NT>::kRounds;
+    const int C = E + 1;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned lt = lanemask_lt();
     const int nbits = key_bits(E);
-
-    for (int x = tid; x < kTileWarps * C; x += kTileThreads) wcnt[x] = 0;
-    if (tid == 0) {
-        *s_invalid = 0;
-        const unsigned t = atomicInc(ws.ticket, (unsigned)(G - 1));
-        // a counter left non-zero by an aborted call: stay in bounds; the
-        // bounded waits then report the failure through diag[1]
-        s_misc[0] = t < (unsigned)G ? t : t % (unsigned)G;
-        s_misc[1] = *(volatile unsigned *)ws.epoch;
-    }
-    __syncthreads();
-    TileCtx ctx;
-    ctx.tile = (int)s_misc[0];
-    ctx.epoch = s_misc[1];
-    ctx.wbase = (int64_t)ctx.tile * kTileSlots + (int64_t)warp * 32 * kTileRounds;
-
-    // ranks within each warp's run, per-warp counts
+    const int64_t wbase = (int64_t)tile * kTileSlots + (int64_t)warp * 32 * NR;
 #pragma unroll
-    for (int r = 0; r < kTileRounds; ++r)
-        key[r] = load_key(ids, ctx.wbase + r * 32 + lane, S, base, E);
+    for (int r = 0; r < NR; ++r) key[r] = load_key(ids, wbase + r * 32 + lane, S, base, E);
+    for (int x = tid; x < NW * C; x += NT) wcnt[x] = 0;
+    if (tid == 0) *s_invalid = 0;
+    __syncthreads();
     int *row = wcnt + warp * C;
     int bad = 0;
 #pragma unroll
-    for (int r = 0; r < kTileRounds; ++r) {
+    for (int r = 0; r < NR; ++r) {
         rank[r] = rank_round(key[r], E, nbits, row, lt);
         bad += key[r] == -1;
     }
@@ -322,22 +311,52 @@ __device__ __forceinline__ TileCtx tile_rank_lookback(
     for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
     if (lane == 0 && bad) atomicAdd(s_invalid, bad);
     __syncthreads();
-    fold_warp_counts<kTileThreads, kTileWarps>(wcnt, E, hist);
+    fold_warp_counts<NT, NW>(wcnt, E, hist);
     if (tid == 0) hist[E] = *s_invalid;
     __syncthreads();
+}
 
-    // publish this tile's aggregates
-    unsigned long long *mine = ws.state + (size_t)ctx.tile * C;
-    for (int c = tid; c < C; c += kTileThreads)
-        st_relaxed_u64(mine + c, lb_word(ctx.epoch, kFlagAgg, hist[c]));
+// Both permutations of a tile's slots: row = off[e] (expert offset, or 0) +
+// excl[e] (earlier tiles) + wcnt (earlier warps) + rank (earlier lanes and
+// rounds).  When `in_perm` is null only the rank part goes to out_perm.
+template <int NT>
+__device__ __forceinline__ void tile_write_rows(int64_t S, int E, int tile, const int *off,
+                                                const int *excl, const int *wcnt,
+                                                const int (&key)[TileShape<NT>::kRounds],
+                                                const int (&rank)[TileShape<NT>::kRounds],
+                                                int32_t *in_perm, int32_t *out_perm) {
+    constexpr int NR = TileShape<NT>::kRounds;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t wbase = (int64_t)tile * kTileSlots + (int64_t)warp * 32 * NR;
+    const int *row = wcnt + warp * (E + 1);
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        const int64_t i = wbase + r * 32 + lane;
+        if (i < S) {
+            const int e = key[r];
+            const int p = e >= 0 ? (off ? off[e] : 0) + excl[e] + row[e] + rank[r] : -1;
+            out_perm[i] = p;
+            if (in_perm && p >= 0 && p < S) in_perm[p] = (int)i;
+        }
+    }
+}
 
-    // decoupled look-back, one column per thread, kLookbackWindow
-    // predecessors read together
+// Decoupled look-back (two-kernel path): publish this tile's aggregates,
+// then per column sum the earlier tiles' values, kLookbackWindow
+// predecessors read together, stopping at an inclusive prefix; publish the
+// inclusive prefix.  excl[c] receives the slots of column c in earlier tiles.
+template <int NT>
+__device__ __forceinline__ void tile_lookback(const PrepWs &ws, int tile, unsigned epoch, int E,
+                                              const int *hist, int *excl) {
+    const int C = E + 1;
+    unsigned long long *mine = ws.state + (size_t)tile * C;
+    for (int c = threadIdx.x; c < C; c += NT)
+        st_relaxed_u64(mine + c, lb_word(epoch, kFlagAgg, hist[c]));
     bool gave_up = false;
-    for (int c = tid; c < C; c += kTileThreads) {
+    for (int c = threadIdx.x; c < C; c += NT) {
         int sum = 0;
         bool done = false;
-        for (int pred = ctx.tile - 1; pred >= 0 && !done && !gave_up; pred -= kLookbackWindow) {
+        for (int pred = tile - 1; pred >= 0 && !done && !gave_up; pred -= kLookbackWindow) {
             unsigned long long v[kLookbackWindow];
 #pragma unroll
             for (int q = 0; q < kLookbackWindow; ++q)
@@ -347,7 +366,7 @@ __device__ __forceinline__ TileCtx tile_rank_lookback(
                 if (done || gave_up || pred - q < 0) continue;
                 const unsigned long long *wp = ws.state + (size_t)(pred - q) * C + c;
                 int spins = 0;
-                while (lb_flag(v[q], ctx.epoch) == 0) {  // not published by this call yet
+                while (lb_flag(v[q], epoch) == 0) {  // not published by this call yet
                     if (++spins > kMaxSpins) {
                         gave_up = true;
                         break;
@@ -356,16 +375,15 @@ __device__ __forceinline__ TileCtx tile_rank_lookback(
                     v[q] = ld_relaxed_u64(wp);
                 }
                 sum += (int)(unsigned)(v[q] & 0xffffffffu);
-                if (lb_flag(v[q], ctx.epoch) == kFlagIncl) done = true;
+                if (lb_flag(v[q], epoch) == kFlagIncl) done = true;
             }
         }
         // publish even after giving up, so that no later tile waits on us
-        st_relaxed_u64(mine + c, lb_word(ctx.epoch, kFlagIncl, sum + hist[c]));
+        st_relaxed_u64(mine + c, lb_word(epoch, kFlagIncl, sum + hist[c]));
         excl[c] = sum;
     }
     if (gave_up) atomicExch(ws.timeout, 1u);
     __syncthreads();
-    return ctx;
 }
 
 // The block's exit: the last block of the call to finish reports a wait
@@ -385,49 +403,59 @@ __device__ __forceinline__ void tile_finish(const PrepWs &ws, int G, unsigned ep
 
 // Shared memory of the tiled kernels: per-warp rows, then hist, excl, off,
 // pad (one column per expert plus one for invalid ids each).
-size_t tile_smem(int E) { return (size_t)(kTileWarps + 4) * (E + 1) * sizeof(int); }
+template <int NT> size_t tile_smem(int E) {
+    return (size_t)(TileShape<NT>::kWarps + 4) * (E + 1) * sizeof(int);
+}
 
-// One-pass variant (all tiles resident together: cooperative launch).  The
-// last tile turns the totals into offsets, writes them and raises `ready`;
-// every tile waits for it (bounded), then writes its slots' final rows into
-// both permutations.
+constexpr int kOnepassThreads = 512;  // one-pass tiles: 16 warps of 4 rounds
+
+// One-pass variant (every tile resident at once: a cooperative launch, so
+// tile = blockIdx.x and a tile may wait on any other).  Each tile ranks its
+// slots and runs the look-back; the last tile turns the totals into offsets,
+// writes them and raises `ready`; every other tile waits for it (bounded),
+// reads the offsets and writes its slots' final rows into both
+// permutations.
 template <typename IdT>
-__global__ void __launch_bounds__(kTileThreads, 2)
+__global__ void __launch_bounds__(kOnepassThreads, 1)
     prep_onepass_kernel(const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int A, int G,
                         void *workspace, int32_t *counts, int32_t *offsets, int32_t *bso,
                         int32_t *in_perm, int32_t *out_perm, int32_t *diag) {
+    constexpr int NT = kOnepassThreads;
     extern __shared__ int smem[];
     __shared__ int warp_tmp[66];
-    __shared__ unsigned s_misc[2];
+    __shared__ unsigned s_epoch;
     __shared__ int s_invalid, s_total;
     const int C = E + 1;
-    int *wcnt = smem;                   // [kTileWarps][C]
-    int *hist = wcnt + kTileWarps * C;  // [C]
-    int *excl = hist + C;               // [C]
-    int *off = excl + C;                // [C] expert offsets
-    int *pad = off + C;                 // [C] scan scratch
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int *wcnt = smem;                              // [NW][C]
+    int *hist = wcnt + TileShape<NT>::kWarps * C;  // [C]
+    int *excl = hist + C;                          // [C]
+    int *off = excl + C;                           // [C] expert offsets
+    int *pad = off + C;                            // [C] scan scratch
+    const int tid = threadIdx.x;
+    const int tile = blockIdx.x;
     PrepWs ws = carve(workspace);
     pdl_wait();
     pdl_launch_dependents();
-    int key[kTileRounds], rank[kTileRounds];
-    const TileCtx ctx =
-        tile_rank_lookback(ids, base, S, E, G, ws, wcnt, hist, excl, s_misc, &s_invalid, key, rank);
-    if (ctx.tile == G - 1) {
+    if (tid == 0) s_epoch = *(volatile unsigned *)ws.epoch;
+    int key[TileShape<NT>::kRounds], rank[TileShape<NT>::kRounds];
+    tile_rank<IdT, NT>(ids, base, S, E, tile, wcnt, hist, &s_invalid, key, rank);
+    const unsigned epoch = s_epoch;
+    tile_lookback<NT>(ws, tile, epoch, E, hist, excl);
+    if (tile == G - 1) {
         // totals = earlier tiles + this one; offsets out, then release the others
-        for (int c = tid; c < C; c += kTileThreads) off[c] = excl[c] + hist[c];
+        for (int c = tid; c < C; c += NT) off[c] = excl[c] + hist[c];
         __syncthreads();
         if (tid == 0 && diag) diag[0] = off[E];
         const int total = offsets_from_totals(off, pad, E, A, true, counts, offsets, bso, warp_tmp);
         if (tid == 0) {
             s_total = total;
             __threadfence();
-            st_release_u32(ws.ready, ctx.epoch + 1);
+            st_release_u32(ws.ready, epoch + 1);
         }
     } else {
         if (tid == 0) {
             int spins = 0;
-            while (ld_acquire_u32(ws.ready) != ctx.epoch + 1) {
+            while (ld_acquire_u32(ws.ready) != epoch + 1) {
                 if (++spins > kMaxSpins) {
                     atomicExch(ws.timeout, 1u);
                     break;
@@ -436,70 +464,65 @@ __global__ void __launch_bounds__(kTileThreads, 2)
             }
         }
         __syncthreads();
-        for (int c = tid; c <= E; c += kTileThreads) off[c] = __ldcg(offsets + c);
+        for (int c = tid; c <= E; c += NT) off[c] = __ldcg(offsets + c);
         if (tid == 0) s_total = __ldcg(offsets + E);
     }
     __syncthreads();
     const int total = s_total;
-    const int *row = wcnt + warp * C;
-#pragma unroll
-    for (int r = 0; r < kTileRounds; ++r) {
-        const int64_t i = ctx.wbase + r * 32 + lane;
-        if (i < S) {
-            const int e = key[r];
-            const int p = e >= 0 ? off[e] + excl[e] + row[e] + rank[r] : -1;
-            out_perm[i] = p;
-            if (p >= 0 && p < S) in_perm[p] = (int)i;
-        }
-    }
-    const int64_t first = (int64_t)ctx.tile * kTileSlots;
+    tile_write_rows<NT>(S, E, tile, off, excl, wcnt, key, rank, in_perm, out_perm);
+    const int64_t first = (int64_t)tile * kTileSlots;
     const int64_t lo = first > total ? first : (int64_t)total;
     const int64_t hi = first + kTileSlots < S ? first + kTileSlots : S;
-    for (int64_t p = lo + tid; p < hi; p += kTileThreads) in_perm[p] = -1;
-    tile_finish(ws, G, ctx.epoch, diag);
+    for (int64_t p = lo + tid; p < hi; p += NT) in_perm[p] = -1;
+    tile_finish(ws, G, epoch, diag);
 }
 
 // Two-kernel variant, kernel 1 (any number of tiles): store rank(i) in
 // output_permutation (-1 for an invalid id); the last tile writes counts,
-// offsets and block-scale offsets.
+// offsets and block-scale offsets.  Tiles take their index from an atomic
+// ticket, so a tile only waits on tiles that are already running.
+constexpr int kRankThreads = 256;  // two-kernel tiles: 8 warps of 8 rounds
+
 template <typename IdT>
-__global__ void __launch_bounds__(kTileThreads, 2)
+__global__ void __launch_bounds__(kRankThreads, 2)
     prep_rank_kernel(const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int A, int G,
                      void *workspace, int32_t *counts, int32_t *offsets, int32_t *bso,
                      int32_t *out_perm, int32_t *diag) {
+    constexpr int NT = kRankThreads;
     extern __shared__ int smem[];
     __shared__ int warp_tmp[66];
     __shared__ unsigned s_misc[2];
     __shared__ int s_invalid;
     const int C = E + 1;
     int *wcnt = smem;
-    int *hist = wcnt + kTileWarps * C;
+    int *hist = wcnt + TileShape<NT>::kWarps * C;
     int *excl = hist + C;
     int *off = excl + C;
     int *pad = off + C;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     PrepWs ws = carve(workspace);
     pdl_wait();
     pdl_launch_dependents();
-    int key[kTileRounds], rank[kTileRounds];
-    const TileCtx ctx =
-        tile_rank_lookback(ids, base, S, E, G, ws, wcnt, hist, excl, s_misc, &s_invalid, key, rank);
-    const int *row = wcnt + warp * C;
-#pragma unroll
-    for (int r = 0; r < kTileRounds; ++r) {
-        const int64_t i = ctx.wbase + r * 32 + lane;
-        if (i < S) {
-            const int e = key[r];
-            out_perm[i] = e >= 0 ? excl[e] + row[e] + rank[r] : -1;
-        }
+    if (threadIdx.x == 0) {
+        const unsigned t = atomicInc(ws.ticket, (unsigned)(G - 1));
+        // a counter left non-zero by an aborted call: stay in bounds; the
+        // bounded waits then report the failure through diag[1]
+        s_misc[0] = t < (unsigned)G ? t : t % (unsigned)G;
+        s_misc[1] = *(volatile unsigned *)ws.epoch;
     }
-    if (ctx.tile == G - 1) {
-        for (int c = threadIdx.x; c < C; c += kTileThreads) off[c] = excl[c] + hist[c];
+    __syncthreads();
+    const int tile = (int)s_misc[0];
+    const unsigned epoch = s_misc[1];
+    int key[TileShape<NT>::kRounds], rank[TileShape<NT>::kRounds];
+    tile_rank<IdT, NT>(ids, base, S, E, tile, wcnt, hist, &s_invalid, key, rank);
+    tile_lookback<NT>(ws, tile, epoch, E, hist, excl);
+    tile_write_rows<NT>(S, E, tile, nullptr, excl, wcnt, key, rank, nullptr, out_perm);
+    if (tile == G - 1) {
+        for (int c = threadIdx.x; c < C; c += NT) off[c] = excl[c] + hist[c];
         __syncthreads();
         if (threadIdx.x == 0 && diag) diag[0] = off[E];
         offsets_from_totals(off, pad, E, A, true, counts, offsets, bso, warp_tmp);
     }
-    tile_finish(ws, G, ctx.epoch, diag);
+    tile_finish(ws, G, epoch, diag);
 }
 
 // Two-kernel variant, kernel 2 (element-wise): row = expert offset + rank;
@@ -572,14 +595,14 @@ cudaError_t launch_onepass(const IdT *ids, int64_t base, int64_t S, int E, int A
                            int32_t *in_perm, int32_t *out_perm, int32_t *diag,
                            cudaStream_t stream) {
     auto kern = prep_onepass_kernel<IdT>;
-    const size_t smem = tile_smem(E);
-    const int64_t resident = (int64_t)sm_count() * blocks_per_sm(kern, kTileThreads, smem);
+    const size_t smem = tile_smem<kOnepassThreads>(E);
+    const int64_t resident = (int64_t)sm_count() * blocks_per_sm(kern, kOnepassThreads, smem);
     if (G > resident) return cudaErrorCooperativeLaunchTooLarge;
     cudaError_t se = ensure_smem(kern, smem);
     if (se != cudaSuccess) return se;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)G, 1, 1);
-    cfg.blockDim = dim3(kTileThreads, 1, 1);
+    cfg.blockDim = dim3(kOnepassThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -609,8 +632,8 @@ cudaError_t run_prepare_t(const IdT *ids, int64_t base, int64_t S, int E, int A,
     cudaError_t e = launch_onepass(ids, base, S, E, A, G, workspace, counts, offsets, bso,
                                    in_perm, out_perm, diag, stream);
     if (e != cudaErrorCooperativeLaunchTooLarge) return e;
-    e = launch(prep_rank_kernel<IdT>, G, kTileThreads, tile_smem(E), stream, ids, base, S, E, A,
-               G, workspace, counts, offsets, bso, out_perm, diag);
+    e = launch(prep_rank_kernel<IdT>, G, kRankThreads, tile_smem<kRankThreads>(E), stream, ids,
+               base, S, E, A, G, workspace, counts, offsets, bso, out_perm, diag);
     if (e != cudaSuccess) return e;
     const int64_t grid = persistent_grid(prep_finish_kernel<IdT>, 256, 0, (S + 1023) / 1024);
     return launch(prep_finish_kernel<IdT>, grid, 256, 0, stream, ids, base, S, E,
