@@ -67,23 +67,33 @@ def algorithmic_bytes(w):
     return {"prepare": prepare, "dispatch": dispatch, "combine": combine}
 
 
-def src_hash():
+# Sources each timed kernel is built from: its own file and the shared headers.
+KERNEL_SOURCES = {
+    "dispatch": ["dispatch.cu", "kernels.h", "launch.h", "moe_device.cuh"],
+    "dispatch_nvfp4": ["dispatch.cu", "kernels.h", "launch.h", "moe_device.cuh"],
+    "combine": ["combine.cu", "kernels.h", "launch.h", "moe_device.cuh"],
+}
+
+
+def src_hash(step):
+    """sha256 (16 hex digits) of the sources the kernel of `step` is built from."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "combine_permute_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
+    for name in KERNEL_SOURCES[step]:
+        with open(os.path.join(ROOT, "combine_permute_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def committed_traffic(kernel_key):
     """dram read+write bytes per launch from the committed ncu summary, if it
-    was taken on the current kernel sources; else None."""
+    was taken on the kernel's current sources; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
         e = d["kernels"][kernel_key]
-        return e["dram_bytes_per_launch"] if e.get("src_hash") == src_hash() else None
+        step = kernel_key.split("@")[0]
+        return e["dram_bytes_per_launch"] if e.get("src_hash") == src_hash(step) else None
     except Exception:
         return None
 
