@@ -118,6 +118,13 @@ def _workspace(device: torch.device, nbytes: int) -> Optional[torch.Tensor]:
     return ws
 
 
+def _drop_workspace(device: torch.device, status: int) -> None:
+    """After a failed launch the cached workspace may hold a half-written
+    call's words; the library needs it all-zero again, so forget it."""
+    if status == _lib.MOE_ERR_CUDA:
+        _WORKSPACES.pop((device, torch.cuda.current_stream(device).cuda_stream), None)
+
+
 def moe_prepare_workspace_bytes(num_tokens: int, top_k: int, num_experts: int) -> int:
     return int(_lib.load().moe_prepare_workspace_bytes(num_tokens, top_k, num_experts))
 
@@ -172,6 +179,7 @@ def moe_prepare(topk_ids: torch.Tensor, num_experts: int, *, blockscale_align: O
             blockscale_align or 1, meta.input_permutation.data_ptr(),
             meta.output_permutation.data_ptr(), meta.diag.data_ptr(), _ptr(workspace), ws_bytes,
             _stream(dev))
+        _drop_workspace(dev, st)
     _lib.check("moe_prepare", st)
     return meta
 
@@ -401,6 +409,7 @@ def moe_prepare_local(topk_ids: torch.Tensor, local_expert_offset: int, num_loca
             _ptr(meta.input_permutation) if T * k else None,
             _ptr(meta.output_permutation) if T * k else None, meta.diag.data_ptr(),
             _ptr(workspace), ws_bytes, _stream(dev))
+        _drop_workspace(dev, st)
     _lib.check("moe_prepare_local", st)
     return meta
 
