@@ -301,7 +301,9 @@ class Step:
             self.xd = torch.empty((S, w.H), dtype=x.dtype, device=dev)
         from workloads.routing import torch_dtype
         self.out = torch.empty((w.T, w.H), dtype=torch_dtype(w.out_dtype), device=dev)
-        self.launches_per_step = 2 if self.fused else (2 if nws > 0 else 1) + 2
+        # prepare: one launch, or two when its tiles do not all fit on the GPU
+        # at once (the graph's kernel nodes give the exact count)
+        self.launches_per_step = 2 if self.fused else (2 if nws > 0 and S > 300_000 else 1) + 2
 
     def prepare(self):
         return self.moe.moe_prepare(self.ids, self.w.E, blockscale_align=self.A, workspace=self.ws,
@@ -374,6 +376,24 @@ class Ranks:
             self.dist.destroy_process_group()
 
 
+def graph_kernel_nodes(g):
+    """Kernel nodes of a captured CUDA graph (kept with keep_graph=True): the
+    kernels one replay launches.  None when the graph cannot be inspected."""
+    try:
+        from cuda.bindings import runtime as rt
+        graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(graph, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kinds = [rt.cudaGraphNodeGetType(node)[1] for node in nodes[:n]]
+        return sum(1 for kind in kinds if kind == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+    except Exception:
+        return None
+
+
 def whole_job_tokens_per_s(T: int, steps: int, world: int, max_elapsed_ms: float) -> float:
     """Tokens every rank processed, over the slowest rank's time."""
     return T * steps * world / (max_elapsed_ms * 1e-3)
@@ -434,14 +454,17 @@ def run_gpu(args, w):
     # ---- timed region 2 (the headline): the same step captured once as a
     #      CUDA graph and replayed K times, the way a serving loop launches it
     graph_ms, clocks = None, clocks_eager
+    kernels_per_step = None
     try:
-        g = torch.cuda.CUDAGraph()
+        g = torch.cuda.CUDAGraph(keep_graph=True)
         side = torch.cuda.Stream(dev)
         side.wait_stream(stream)
         with torch.cuda.stream(side):
             step.run()
             with torch.cuda.graph(g, stream=side):
                 step.run()
+        kernels_per_step = graph_kernel_nodes(g)
+        g.instantiate()
         torch.cuda.synchronize(dev)
         for _ in range(3):
             g.replay()
@@ -519,7 +542,9 @@ def run_gpu(args, w):
                      "algorithmic_bytes_per_launch": alg[dominant]},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": step.launches_per_step * K,
+        "gpu_launches": (kernels_per_step or step.launches_per_step) * K,
+        "gpu_launches_counted_from": ("kernel nodes of the captured step"
+                                      if kernels_per_step else "launches per step of each call"),
         "clocks": clocks.summary(),
         "breakdown": breakdown,
         "next_rows": next_rows,
