@@ -9,7 +9,9 @@
 // 32 consecutive slots, across a warp's rounds by a warp-private running
 // counter in shared memory, across warps by an exclusive scan of the
 // per-warp counts, and across blocks by one of:
-//  * up to kSingleBlockSlots slots: nothing, one block does it all
+//  * up to kSmallSlots slots: one block, one thread per slot, each slot's
+//    rank counted directly over the earlier slots (prep_small_kernel);
+//  * up to kSingleBlockSlots slots: one block does it all
 //    (prep_single_kernel);
 //  * above that, tiles of kTileSlots slots, each ranked by one block, which
 //    publishes its per-expert histogram and runs a decoupled look-back over
@@ -186,6 +188,85 @@ __device__ __forceinline__ unsigned long long lb_flag(unsigned long long w, unsi
 }
 
 // ---------------------------------------------------------------------------
+// Small batches (up to kSmallSlots slots): one thread per slot, in one
+// block.  A slot's rank is counted directly: the number of earlier slots
+// with the same expert, read from the keys staged in shared memory (a
+// broadcast read, four keys at a time).  Counts come from shared-memory
+// atomics, offsets from one block scan; three block barriers in all, where
+// the counting sort needs its ranking rounds and a fold over warps.  smem:
+// S + 4*(E+1) ints (keys, then counts / offsets, scan scratch).  `pos`, when
+// non-null, receives every slot's dispatched row (shared memory, S ints);
+// global outputs are written when `write` is set.  Every thread of the block
+// calls it; blockDim.x >= S.
+// ---------------------------------------------------------------------------
+constexpr int kSmallSlots = 512;
+
+template <typename IdT>
+__device__ __forceinline__ void small_prepare(const IdT *__restrict__ ids, int64_t base, int S,
+                                              int E, int A, int *smem, int *pos, bool write,
+                                              int32_t *counts, int32_t *offsets, int32_t *bso,
+                                              int32_t *in_perm, int32_t *out_perm,
+                                              int32_t *diag) {
+    __shared__ int warp_tmp[66];
+    __shared__ int s_invalid;
+    int *keys = smem;                           // [S], padded to a multiple of 4
+    int *cnt = keys + ((S + 3) & ~3);           // [E] counts, then expert offsets
+    int *pad = cnt + E;                         // [E] scan scratch
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int e = tid < S ? load_key(ids, tid, S, base, E) : -2;
+    for (int c = tid; c < E; c += nt) cnt[c] = 0;
+    if (tid < ((S + 3) & ~3)) keys[tid] = e;  // the padding keys are -2: no expert
+    if (tid == 0) s_invalid = 0;
+    __syncthreads();
+    int rank = 0;
+    if (e >= 0) {
+        const int4 *k4 = reinterpret_cast<const int4 *>(keys);
+        const int n4 = tid >> 2;
+        for (int j = 0; j < n4; ++j) {
+            const int4 v = k4[j];
+            rank += (v.x == e) + (v.y == e) + (v.z == e) + (v.w == e);
+        }
+        for (int j = n4 << 2; j < tid; ++j) rank += keys[j] == e;
+        atomicAdd(&cnt[e], 1);
+    }
+    const unsigned bad = __ballot_sync(0xffffffffu, e == -1);
+    if ((tid & 31) == 0 && bad) atomicAdd(&s_invalid, __popc(bad));
+    __syncthreads();
+    const int total = offsets_from_totals(cnt, pad, E, A, write, counts, offsets, bso, warp_tmp);
+    if (write && tid == 0 && diag) {
+        diag[0] = s_invalid;
+        diag[1] = 0;
+    }
+    __syncthreads();
+    if (tid < S) {
+        const int p = e >= 0 ? cnt[e] + rank : -1;
+        if (pos) pos[tid] = p;
+        if (write) {
+            out_perm[tid] = p;
+            if (p >= 0) in_perm[p] = tid;
+        }
+    }
+    if (write)
+        for (int p = total + tid; p < S; p += nt) in_perm[p] = -1;
+}
+
+template <typename IdT>
+__global__ void __launch_bounds__(kSmallSlots, 1)
+    prep_small_kernel(const IdT *__restrict__ ids, int64_t base, int S, int E, int A,
+                      int32_t *counts, int32_t *offsets, int32_t *bso, int32_t *in_perm,
+                      int32_t *out_perm, int32_t *diag) {
+    extern __shared__ int smem[];
+    pdl_wait();
+    pdl_launch_dependents();
+    small_prepare(ids, base, S, E, A, smem, nullptr, true, counts, offsets, bso, in_perm, out_perm,
+                  diag);
+}
+
+__host__ __device__ inline size_t small_smem(int E, int64_t S) {
+    return (size_t)(((S + 3) & ~3) + 2 * E) * sizeof(int);
+}
+
+// ---------------------------------------------------------------------------
 // One block (kSingleThreads threads, up to kSingleBlockSlots slots).  When
 // `pos` is non-null the dispatched row of every slot is also left there
 // (shared memory, S entries); global outputs are written when `write` is
@@ -278,7 +359,6 @@ size_t single_block_smem(int E) { return (size_t)(kSingleWarps * (E + 1) + 2 * E
 // prefixes and key/rank each thread's slots.
 // ---------------------------------------------------------------------------
 template <int NT> struct TileShape {
-    static constexpr int kThreads = NT;
     static constexpr int kWarps = NT / 32;
     static constexpr int kRounds = kTileSlots / NT;
     static_assert(NT * kRounds == kTileSlots, "a tile is kTileSlots slots");
@@ -558,11 +638,18 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
                          int64_t nvec, uint4 *__restrict__ out) {
     extern __shared__ int smem[];
     const int64_t S = T * k;
-    int *pos = smem + kSingleWarps * (E + 1) + 2 * E;  // [S]
+    int *pos;  // [S] dispatched row of every slot
     pdl_wait();
     pdl_launch_dependents();
-    single_block_prepare(ids, (int64_t)0, S, E, A, smem, pos, blockIdx.x == 0, counts, offsets,
-                         bso, in_perm, out_perm, diag);
+    if (S <= kSmallSlots) {
+        pos = smem + small_smem(E, S) / sizeof(int);
+        small_prepare(ids, (int64_t)0, (int)S, E, A, smem, pos, blockIdx.x == 0, counts, offsets,
+                      bso, in_perm, out_perm, diag);
+    } else {
+        pos = smem + kSingleWarps * (E + 1) + 2 * E;
+        single_block_prepare(ids, (int64_t)0, S, E, A, smem, pos, blockIdx.x == 0, counts,
+                             offsets, bso, in_perm, out_perm, diag);
+    }
     __syncthreads();
     const int64_t total = T * nvec;
     for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
@@ -625,6 +712,11 @@ template <typename IdT>
 cudaError_t run_prepare_t(const IdT *ids, int64_t base, int64_t S, int E, int A, int32_t *counts,
                           int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,
                           int32_t *diag, void *workspace, cudaStream_t stream) {
+    if (S <= kSmallSlots) {
+        const int threads = S < 32 ? 32 : (int)((S + 31) / 32 * 32);
+        return launch(prep_small_kernel<IdT>, 1, threads, small_smem(E, S), stream, ids, base,
+                      (int)S, E, A, counts, offsets, bso, in_perm, out_perm, diag);
+    }
     if (S <= kSingleBlockSlots)
         return launch(prep_single_kernel<IdT>, 1, kSingleThreads, single_block_smem(E), stream, ids,
                       base, S, E, A, counts, offsets, bso, in_perm, out_perm, diag);
@@ -659,7 +751,8 @@ cudaError_t run_prepare_dispatch(const int32_t *ids, int64_t T, int k, int E, in
                                  cudaStream_t stream) {
     const int64_t S = T * k;
     const int64_t nvec = row_bytes / 16;
-    const size_t smem = single_block_smem(E) + (size_t)S * sizeof(int);
+    const size_t smem = (S <= kSmallSlots ? small_smem(E, S) : single_block_smem(E)) +
+                        (size_t)S * sizeof(int);
     const int64_t units = (T * nvec + kSingleThreads - 1) / kSingleThreads;
     const int64_t grid = persistent_grid(prep_dispatch_kernel, kSingleThreads, smem, units);
     return launch(prep_dispatch_kernel, grid, kSingleThreads, smem, stream, ids, T, k, E, A,
