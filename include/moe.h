@@ -126,9 +126,10 @@ size_t moe_prepare_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t nu
  *                                      other outputs are then invalid), else
  *                                      0.
  *   workspace                          scratch of moe_prepare_workspace_bytes()
- *                                      bytes, 256-byte aligned, zero on entry
- *                                      (see above); may be NULL when that
- *                                      size is 0.
+ *                                      bytes, 256-byte aligned, zeroed before
+ *                                      its first use and then left to the
+ *                                      library (see above); may be NULL when
+ *                                      that size is 0.
  *
  * Batches of up to 4096 slots run in one block; larger ones as tiles over
  * the whole GPU (the only case that touches the workspace): one cooperative
