@@ -62,7 +62,8 @@ def test_prepare_tiny_vs_oracle(trial):
 
 
 @pytest.mark.parametrize("T,k,E", [
-    (1, 8, 256), (63, 8, 256), (512, 8, 256),          # single block, full single tile
+    (1, 8, 256), (63, 8, 256), (64, 8, 1024), (65, 8, 3),  # small path up to 512 slots, then
+    (512, 8, 256),                                     # single block, full single tile
     (513, 8, 256), (1024, 8, 7), (3001, 6, 64),          # two or more tiles, ragged tails
     (4095, 1, 1), (20000, 8, 1024), (9216, 8, 256),
     (40000, 3, 5), (70000, 8, 288),
@@ -73,6 +74,17 @@ def test_prepare_sizes_vs_oracle(T, k, E):
     ids = _ids_random(rng, T, k, E, p_invalid=0.03, distinct=False)
     _check_prepare(ids, E, A=128)
     _check_prepare(ids, E, A=None)
+
+
+def test_prepare_large_batch():
+    """100 M slots (2^24 tokens, top-6 of 4 experts; three quarters of the
+    slots on one expert, about 5 % invalid ids): about 49 000 tiles through
+    the two-kernel path, offsets near 10^8."""
+    T, k, E = 1 << 24, 6, 4
+    rng = np.random.default_rng(2024)
+    ids = rng.integers(-1, E, size=(T, k), dtype=np.int32)
+    ids[rng.random((T, k), dtype=np.float32) < 0.75] = 2
+    _check_prepare(ids, E, A=128)
 
 
 @pytest.mark.parametrize("T", [100, 5000])
