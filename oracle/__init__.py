@@ -15,6 +15,16 @@ step computes:
   (run_moe_fp8_block_scales), with 1x128 blocks and scale = amax / 448.
 * ``combine``: sglang PR #19058, item 3 (apply_shuffle_mul_sum: gather,
   scale by the router weight, reduce with fp32 accumulation).
+* ``dispatch_nvfp4``: the B200 NVFP4 MoE path of TensorRT-LLM PR #9592
+  (run_moe_nvfp4, scaling_vector_size = 16): E2M1 codes, one E4M3 scale per
+  16 elements.
+* ``problem_sizes`` and ``tile_layout``: the grouped-GEMM metadata that
+  follows prepare (sglang's problem_sizes1/2; TensorRT-LLM's moe_sort
+  outputs).
+* ``prepare_local`` and ``output_memset``: one rank's expert window
+  (local_expert_offset / num_local_experts) over int64 ids, and
+  moe_output_memset_inplace (TensorRT-LLM PR #9592; Mooncake PR #4581 for
+  the int64 top-k index type).
 
 The arithmetic lives in ``moe_oracle.c`` (built with gcc, ``-O2
 -ffp-contract=off``, single-threaded).  ``brute_prepare`` is a second,

@@ -21,7 +21,11 @@
  *     and review comments): "expanded idx" = t*k + j and "permuted idx" =
  *     dispatched row, int32 index tensors, and the FP8 block-scale MoE path
  *     (run_moe_fp8_block_scales), which oracle_dispatch_fp8 instantiates
- *     with 1x128 blocks and scale = amax / 448.
+ *     with 1x128 blocks and scale = amax / 448; the NVFP4 path
+ *     (run_moe_nvfp4, scaling_vector_size = 16: oracle_dispatch_nvfp4); the
+ *     moe_sort outputs of a tiled grouped GEMM (oracle_tile_layout); the
+ *     local-expert window and moe_output_memset_inplace
+ *     (oracle_prepare_local_i64, oracle_output_memset).
  *
  * Readings where the pages are silent (each one is listed in the design
  * notes):
