@@ -291,12 +291,8 @@ class Step:
                               diag=torch.empty(2, **i32))
         nws = moe.moe_prepare_workspace_bytes(w.T, w.k, E)
         self.ws = torch.zeros(max(nws, 1), dtype=torch.uint8, device=dev)
-        # The step launches prepare, dispatch and combine separately at every
-        # size: inside a CUDA graph that measured faster, also for tiny
-        # batches, than the one-launch prepare + dispatch path (which saves a
-        # host launch when calls are issued one by one; `next_rows` times it).
-        self.fused = False
-        self.fused_ok = (not self.fp8) and S <= moe._lib.FUSED_MAX_SLOTS
+        # tiny batches take the one-launch prepare + dispatch path
+        self.fused = (not self.fp8) and S <= moe._lib.FUSED_MAX_SLOTS
         if self.fp8:
             self.xq = torch.empty((S, w.H), dtype=torch.uint8, device=dev)
             self.scales = torch.empty((S + E * (w.block_align - 1), w.H // 128),
@@ -575,9 +571,8 @@ def run_gpu(args, w):
 def time_next_rows(step, w, dev, reps=20):
     """The steps beside the timed path: the grouped-GEMM metadata that follows
     prepare (tile-padded layout with 128-row tiles, per-expert problem
-    sizes), the NVFP4 dispatch of this workload's activations and, for tiny
-    batches, the one-launch prepare + dispatch, each timed as a CUDA graph of
-    `reps` calls."""
+    sizes) and the NVFP4 dispatch of this workload's activations, each timed
+    as a CUDA graph of `reps` calls."""
     import torch
     moe = step.moe
     meta = step.prepare()
@@ -621,11 +616,6 @@ def time_next_rows(step, w, dev, reps=20):
                                                        out_scales=sc))
         b = w.T * w.H * step.x.element_size() + S * (w.H // 2 + w.H // 16) + 4 * S + 8 * (E + 1)
         out["dispatch_nvfp4"] = {"us": us, "algorithmic_bytes": b, "effective_gbs": b / us / 1e3}
-    if step.fused_ok:
-        bufs = dict(step.meta_bufs)
-        bufs.pop("blockscale_offsets", None)
-        us = timed(lambda: moe.moe_prepare_dispatch(step.ids, w.E, step.x, out=step.xd, **bufs))
-        out["prepare_dispatch_one_launch"] = {"us": us}
     return out
 
 

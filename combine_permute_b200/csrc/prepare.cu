@@ -753,11 +753,14 @@ cudaError_t run_prepare_dispatch(const int32_t *ids, int64_t T, int k, int E, in
     const int64_t nvec = row_bytes / 16;
     const size_t smem = (S <= kSmallSlots ? small_smem(E, S) : single_block_smem(E)) +
                         (size_t)S * sizeof(int);
-    const int64_t units = (T * nvec + kSingleThreads - 1) / kSingleThreads;
-    const int64_t grid = persistent_grid(prep_dispatch_kernel, kSingleThreads, smem, units);
-    return launch(prep_dispatch_kernel, grid, kSingleThreads, smem, stream, ids, T, k, E, A,
-                  counts, offsets, bso, in_perm, out_perm, diag, (const uint4 *)x, nvec,
-                  (uint4 *)out);
+    // small batches: blocks of 256 threads (at least one thread per slot),
+    // so that more SMs share the copy; larger ones: the 1024-thread block
+    const int threads = S <= kSmallSlots ? (S <= 256 ? 256 : (int)((S + 31) / 32 * 32))
+                                         : kSingleThreads;
+    const int64_t units = (T * nvec + threads - 1) / threads;
+    const int64_t grid = persistent_grid(prep_dispatch_kernel, threads, smem, units);
+    return launch(prep_dispatch_kernel, grid, threads, smem, stream, ids, T, k, E, A, counts,
+                  offsets, bso, in_perm, out_perm, diag, (const uint4 *)x, nvec, (uint4 *)out);
 }
 
 }  // namespace moe
