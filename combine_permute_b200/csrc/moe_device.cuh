@@ -231,7 +231,7 @@ namespace moe {
 // ---------------------------------------------------------------------------
 // Bulk asynchronous copies (TMA engine, non-tensor form) and mbarriers.
 // All addresses are 16-byte aligned and sizes multiples of 16 bytes.  No
-// multicast form is used anywhere.
+// cluster-wide form is used anywhere.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
