@@ -127,49 +127,6 @@ __device__ __forceinline__ float e4m3_to_f32(uint16_t byte) {
 }
 
 // ---------------------------------------------------------------------------
-// Block-wide exclusive scan of n <= 4 * blockDim.x ints held in shared
-// memory (in place).  Returns the total.  All threads must call it.
-// `warp_tmp` needs blockDim.x / 32 + 1 ints.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ int block_exclusive_scan(int *data, int n, int *warp_tmp) {
-    const int tid = threadIdx.x, nt = blockDim.x;
-    const int per = (n + nt - 1) / nt;
-    const int beg = min(n, tid * per), end = min(n, beg + per);
-    int local = 0;
-    for (int i = beg; i < end; ++i) local += data[i];
-    // inclusive warp scan of the per-thread sums
-    const int lane = tid & 31, warp = tid >> 5;
-    int v = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        int u = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += u;
-    }
-    if (lane == 31) warp_tmp[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        const int nw = nt >> 5;
-        int w = lane < nw ? warp_tmp[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int u = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += u;
-        }
-        if (lane < nw) warp_tmp[lane] = w;  // inclusive warp totals
-        if (lane == nw - 1) warp_tmp[32] = w;
-    }
-    __syncthreads();
-    int run = v - local + (warp > 0 ? warp_tmp[warp - 1] : 0);
-    for (int i = beg; i < end; ++i) {
-        int c = data[i];
-        data[i] = run;
-        run += c;
-    }
-    const int total = warp_tmp[32];
-    __syncthreads();
-    return total;
-}
-
 // Two exclusive scans in one pass over n <= 32 * blockDim.x counts held in
 // shared memory: a[] in place, and pad[] <- exclusive scan of a[] each
 // rounded up to a multiple of A.  Returns the total of a; *pad_total gets
@@ -300,11 +257,6 @@ template <int N> __device__ __forceinline__ void bulk_wait_read() {
 // Wait until every committed bulk group has completed.
 __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
-// Make generic-proxy shared-memory writes visible to the async proxy.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 }  // namespace moe
