@@ -62,7 +62,7 @@ def algorithmic_bytes(w):
     prepare = 4 * S + 4 * E + 4 * (E + 1) + 8 * S + (4 * (E + 1) if fp8 else 0)
     dispatch = T * H * bx + S * H * bd + 4 * S
     if fp8:
-        dispatch += 4 * S + 4 * S * (H // 128) + 8 * (E + 1)  # ids, scales, offsets
+        dispatch += 4 * S * (H // 128) + 8 * (E + 1)  # scales, expert and scale offsets
     combine = S * H * by + 4 * S + 4 * S + T * H * bo
     return {"prepare": prepare, "dispatch": dispatch, "combine": combine}
 

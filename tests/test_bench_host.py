@@ -1,0 +1,61 @@
+"""Host-side pieces of bench.py: the algorithmic byte counts behind every
+roofline fraction (checked against the per-step byte table the method's
+sizes give), the graph step count, the whole-job throughput and the rule
+that a profile's traffic only counts for the sources it was taken on."""
+
+import json
+
+import pytest
+
+import bench
+from workloads import CONFIGS
+
+MB = 1e6
+
+# (dispatch, combine) minimal bytes per step in MB: every input read once,
+# every output written once; x read once although written k times.
+TABLE = {
+    "tiny_t32_h4096_e256_k8": (2.36, 2.36),
+    "uniform_t4096_h7168_e256_k8": (528.6, 528.7),
+    "khot_t9216_h7168_e256_k8": (1189.4, 1189.7),
+    "zipf_fp8_t16384_h4096_e288_k8": (688.4, 1209.0),
+    "zipf_fp16_t131072_h2048_e64_k6": (3761.2, 4301.3),
+}
+
+
+@pytest.mark.parametrize("name", list(TABLE))
+def test_algorithmic_bytes_match_the_table(name):
+    b = bench.algorithmic_bytes(CONFIGS[name])
+    d, c = TABLE[name]
+    assert abs(b["dispatch"] / MB - d) < 0.05 + 1e-3 * d
+    assert abs(b["combine"] / MB - c) < 0.05 + 1e-3 * c
+
+
+def test_algorithmic_bytes_closed_form_uniform():
+    w = CONFIGS["uniform_t4096_h7168_e256_k8"]
+    S = w.T * w.k
+    b = bench.algorithmic_bytes(w)
+    assert b["dispatch"] == w.T * w.H * 2 + S * w.H * 2 + 4 * S
+    assert b["combine"] == S * w.H * 2 + 8 * S + w.T * w.H * 2
+    assert b["prepare"] == 4 * S + 4 * w.E + 4 * (w.E + 1) + 8 * S
+
+
+@pytest.mark.parametrize("K,n", [(1, 1), (3, 3), (7, 7), (20, 10), (200, 10), (201, 3), (11, 1)])
+def test_steps_per_graph_divides_K(K, n):
+    assert bench.steps_per_graph(K) == n
+    assert K % bench.steps_per_graph(K) == 0
+
+
+def test_whole_job_throughput_counts_every_rank():
+    # 2 ranks x 10 steps x 4096 tokens in 20 ms (the slowest rank's time)
+    assert bench.whole_job_tokens_per_s(4096, 10, 2, 20.0) == pytest.approx(4096 * 20 / 0.02)
+
+
+def test_traffic_counts_only_for_the_captured_sources(monkeypatch):
+    key = "dispatch@uniform_t4096_h7168_e256_k8"
+    with open(bench.os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        entry = json.load(f)["kernels"][key]
+    monkeypatch.setattr(bench, "src_hash", lambda step: entry["src_hash"])
+    assert bench.committed_traffic(key) == entry["dram_bytes_per_launch"]
+    monkeypatch.setattr(bench, "src_hash", lambda step: "0" * 16)
+    assert bench.committed_traffic(key) is None
