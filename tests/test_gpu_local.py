@@ -76,6 +76,28 @@ def test_fp8_dispatch_and_tile_layout_on_an_expert_window():
     np.testing.assert_array_equal(lay.permuted_idx_to_expanded_idx.cpu().numpy(), lref["perm2exp"])
 
 
+def test_nvfp4_dispatch_on_an_expert_window_int64_ids():
+    """One rank's window of experts from int64 ids, then the NVFP4 dispatch
+    of its rows (scale rows padded to 16 per expert)."""
+    w = CONFIGS["uniform_t4096_h7168_e256_k8"].scaled(900)
+    ids_np, _, x, _ = make_workload(w, device=DEV, with_y=False)
+    ids64 = ids_np.astype(np.int64) + (1 << 33)   # ids beyond the int32 range
+    base, E, A = (1 << 33) + 64, 64, 16
+    meta, ref = _check_local(ids64, base, E, A)
+    rows = w.S + E * (A - 1)
+    q, sc = moe.moe_dispatch_rows_nvfp4(
+        x, w.k, meta.output_permutation, meta.expert_offsets, meta.blockscale_offsets,
+        out_q=torch.full((w.S, w.H // 2), 0xAB, dtype=torch.uint8, device=DEV),
+        out_scales=torch.full((rows, w.H // 16), 0xCD, dtype=torch.uint8, device=DEV))
+    torch.cuda.synchronize()
+    local = _shifted(ids64, base, E)
+    q_ref = np.full((w.S, w.H // 2), 0xAB, np.uint8)
+    sc_ref = np.full((rows, w.H // 16), 0xCD, np.uint8)
+    oracle.dispatch_nvfp4(bits(x), "bf16", local, ref, q_ref, sc_ref)
+    np.testing.assert_array_equal(q.cpu().numpy(), q_ref)
+    np.testing.assert_array_equal(sc.cpu().numpy(), sc_ref)
+
+
 @pytest.mark.parametrize("dtype,H", [("bf16", 7168), ("fp32", 1000), ("fp16", 8)])
 def test_output_memset_vs_oracle(dtype, H):
     w = CONFIGS["uniform_t4096_h7168_e256_k8"].scaled(700)
