@@ -621,7 +621,12 @@ def time_next_rows(step, w, dev, reps=20):
 
 def run_e2e(step, w, dev, K, W, barrier, max_over_ranks):
     """Same step through the public API with inputs copied in from pinned
-    host memory and the combined output read back, every step."""
+    host memory and the combined output read back, every step.  The copies
+    run on their own streams, double-buffered, so that step i+1's inputs
+    cross the host link while step i computes and step i-1's output is read
+    back (the way a serving loop streams batches); every step's copies are
+    inside the timed region."""
+    import copy as _copy
     import torch
     h_ids = torch.from_numpy(step.ids_np).pin_memory()
     h_wt = torch.from_numpy(step.wt_np).pin_memory()
@@ -630,32 +635,56 @@ def run_e2e(step, w, dev, K, W, barrier, max_over_ranks):
     h_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in (h_ids, h_wt, h_x, h_y))
     d2h = h_out.numel() * h_out.element_size()
-    stream = torch.cuda.current_stream(dev)
+    comp = torch.cuda.current_stream(dev)
     n = max(1, min(K, 20))
 
-    def one():
-        step.ids.copy_(h_ids, non_blocking=True)
-        step.wt.copy_(h_wt, non_blocking=True)
-        step.x.copy_(h_x, non_blocking=True)
-        step.y.copy_(h_y, non_blocking=True)
-        step.run()
-        h_out.copy_(step.out, non_blocking=True)
+    # a second set of input / output buffers; the metadata, workspace and
+    # dispatched rows are shared, since the computes run in order on one stream
+    other = _copy.copy(step)
+    for name in ("ids", "wt", "x", "y", "out"):
+        setattr(other, name, torch.empty_like(getattr(step, name)))
+    bufs = (step, other)
+    copy_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    h2d_done = [torch.cuda.Event(), torch.cuda.Event()]
+    comp_done = [torch.cuda.Event(), torch.cuda.Event()]
+    d2h_done = [torch.cuda.Event(), torch.cuda.Event()]
 
-    for _ in range(min(W, 3)):
-        one()
+    def run(count):
+        for i in range(count):
+            b = i % 2
+            st = bufs[b]
+            with torch.cuda.stream(copy_s):
+                if i >= 2:
+                    copy_s.wait_event(comp_done[b])  # step i-2 has read these inputs
+                st.ids.copy_(h_ids, non_blocking=True)
+                st.wt.copy_(h_wt, non_blocking=True)
+                st.x.copy_(h_x, non_blocking=True)
+                st.y.copy_(h_y, non_blocking=True)
+                h2d_done[b].record(copy_s)
+            comp.wait_event(h2d_done[b])
+            if i >= 2:
+                comp.wait_event(d2h_done[b])  # step i-2's output has been read back
+            st.run()
+            comp_done[b].record(comp)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(comp_done[b])
+                h_out.copy_(st.out, non_blocking=True)
+                d2h_done[b].record(d2h_s)
+
+    run(min(W, 3))
     torch.cuda.synchronize(dev)
     barrier()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(n):
-        one()
-    e.record(stream)
+    s.record(copy_s)
+    run(n)
+    e.record(d2h_s)
     torch.cuda.synchronize(dev)
     barrier()
     ms = max_over_ranks(s.elapsed_time(e))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     return {"value": w.T * n * world / (ms * 1e-3), "unit": "tokens/s", "steps": n,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "copies": "own streams, double-buffered, overlapping the compute"}
 
 
 def main():
