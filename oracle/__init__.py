@@ -34,6 +34,7 @@ stable ``sorted`` instead of the per-expert scan.
 
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 
@@ -45,7 +46,7 @@ __all__ = [
     "F32", "F16", "BF16", "lib", "prepare", "dispatch", "dispatch_fp8",
     "combine", "brute_prepare", "problem_sizes", "tile_layout", "prepare_local",
     "output_memset", "dispatch_nvfp4", "f32_to_e2m1", "e2m1_to_f32", "f32_to_bf16", "f32_to_f16", "f16_to_f32",
-    "bf16_to_f32", "f32_to_e4m3", "e4m3_to_f32",
+    "bf16_to_f32", "f32_to_e4m3", "e4m3_to_f32", "openmp", "threads",
 ]
 
 F32, F16, BF16 = 0, 1, 2
@@ -56,14 +57,43 @@ _i32p = ctypes.POINTER(ctypes.c_int32)
 _vp = ctypes.c_void_p
 
 
+_omp_lib = None
+_use_omp = False
+
+
+@contextlib.contextmanager
+def openmp():
+    """Within this block the oracle's calls run on its OpenMP build, which
+    shares the dispatch and combine row loops among the host cores (same
+    results; prepare stays one thread).  For the benchmark's CPU baseline."""
+    global _use_omp
+    prev = _use_omp
+    _use_omp = True
+    try:
+        yield threads(True)
+    finally:
+        _use_omp = prev
+
+
+def threads(openmp_build: bool = False) -> int:
+    """Threads the oracle's row loops use: 1, or the OpenMP build's count."""
+    return int(_load(openmp_build).oracle_threads())
+
+
 def lib():
     """The oracle shared library (built on first use if it is missing)."""
-    global _lib
-    if _lib is None:
-        path = oracle_lib_path()
+    return _load(_use_omp)
+
+
+def _load(openmp_build: bool):
+    global _lib, _omp_lib
+    if (_omp_lib if openmp_build else _lib) is None:
+        path = oracle_lib_path(openmp_build)
         if not os.path.exists(path):
-            build_oracle()
+            build_oracle(openmp=openmp_build)
         L = ctypes.CDLL(path)
+        L.oracle_threads.restype = ctypes.c_int
+        L.oracle_threads.argtypes = []
         L.oracle_prepare.restype = ctypes.c_int64
         L.oracle_prepare.argtypes = [_vp, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_int32, _vp, _vp, _vp, _vp, _vp]
@@ -97,8 +127,11 @@ def lib():
             fn = getattr(L, name)
             fn.restype = None
             fn.argtypes = [_vp, ctypes.c_int64, _vp]
-        _lib = L
-    return _lib
+        if openmp_build:
+            _omp_lib = L
+        else:
+            _lib = L
+    return _omp_lib if openmp_build else _lib
 
 
 def _ptr(a: np.ndarray):

@@ -55,6 +55,32 @@
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/*
+ * Timing build only: the benchmark's CPU baseline also compiles this file
+ * with -fopenmp, which shares the independent row loops of the dispatches
+ * and of combine among the host cores (ROWS_IN_PARALLEL).  Every iteration
+ * of those loops writes its own rows, so the results are the same bits.
+ * The build the tests check against has no _OPENMP and stays one thread.
+ */
+#ifdef _OPENMP
+#define ROWS_IN_PARALLEL _Pragma("omp parallel for schedule(static)")
+#else
+#define ROWS_IN_PARALLEL
+#endif
+
+/* Threads the row loops use (1 in the plain build). */
+int oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 enum { ORACLE_F32 = 0, ORACLE_F16 = 1, ORACLE_BF16 = 2 };
 
@@ -258,6 +284,7 @@ void oracle_dispatch(const void *x, int64_t row_bytes, int32_t k,
 {
     const unsigned char *src = (const unsigned char *)x;
     unsigned char *dst = (unsigned char *)out;
+    ROWS_IN_PARALLEL
     for (int64_t p = 0; p < S; ++p) {
         int32_t i = input_perm[p];
         if (i < 0)
@@ -287,6 +314,7 @@ void oracle_dispatch_fp8(const uint16_t *x, int x_dtype, int64_t T, int64_t H, i
 {
     (void)T;
     int64_t nb = H / 128;
+    ROWS_IN_PARALLEL
     for (int64_t p = 0; p < S; ++p) {
         int32_t i = input_perm[p];
         if (i < 0)
@@ -329,6 +357,7 @@ void oracle_dispatch_fp8(const uint16_t *x, int x_dtype, int64_t T, int64_t H, i
 void oracle_combine(const void *y, int y_dtype, int64_t T, int64_t H, int32_t k,
                     const int32_t *output_perm, const float *w, void *out, int out_dtype)
 {
+    ROWS_IN_PARALLEL
     for (int64_t t = 0; t < T; ++t) {
         for (int64_t h = 0; h < H; ++h) {
             float acc = 0.0f;
