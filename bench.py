@@ -5,7 +5,12 @@ One step = one pass of the whole path over one batch: routing metadata
 fp8 workload) and combine (moe_combine), on seeded synthetic inputs already
 resident in HBM.  Prints ONE JSON line (rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+By default every workload runs: the headline is the largest single-GPU one
+(T=131072, H=2048, E=64, top-6, fp16 -> fp32 combine) and the other four
+are reported under "per_workload" with the same fields.  ``--workload NAME``
+runs one workload alone as the headline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|all]
     python bench.py --impl reference ...   # the CPU oracle on the host cores
 
 Multi-GPU runs (torchrun, one process per GPU) are independent replicas:
@@ -33,7 +38,7 @@ sys.path.insert(0, ROOT)
 
 from workloads import CONFIGS, make_workload  # noqa: E402
 
-DEFAULT_WORKLOAD = "uniform_t4096_h7168_e256_k8"
+HEADLINE_WORKLOAD = "zipf_fp16_t131072_h2048_e64_k6"
 METRIC = "dispatch+combine tokens/s and effective HBM GB/s (% of B200 peak), 1 GPU"
 SPEC_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
@@ -195,56 +200,92 @@ def _host_inputs(w, T_sample):
     return ws, ids, wt, xb, yb
 
 
-def time_oracle(w, budget_s=12.0, steps=None):
-    """Time the oracle's full step on the host.  With ``steps`` None: whole
-    workload steps repeated until ``budget_s`` (at least one).  With
-    ``steps`` K: K steps, each on the first T_s tokens, T_s sized so that
-    the K steps take about ``budget_s``."""
+def oracle_sample_plan(w, step_budget_s, openmp=False):
+    """A bounded sample of workload ``w`` for the oracle: the same routing,
+    shapes and dtypes on the first T_s tokens, T_s sized from a 256-token
+    calibration step so that one oracle step takes about ``step_budget_s``.
+    Returns T_s and a function that runs one oracle step on it."""
     import oracle
     oracle.lib()
-    if steps is None:
-        ws, ids, wt, xb, yb = _host_inputs(w, w.T)
-        n, t0 = 0, time.perf_counter()
-        while True:
-            _oracle_step(oracle, ws, ids, wt, xb, yb)
-            n += 1
-            if time.perf_counter() - t0 >= budget_s:
-                break
-        dt = time.perf_counter() - t0
-        return dict(tokens=n * w.T, seconds=dt, sample=f"{n} full steps of {w.name} ({w.T} tokens each)")
-    # calibrate on a small slice, then size the per-step sample
+    ctx = oracle.openmp() if openmp else _null_ctx()
     cal_T = max(1, min(w.T, 256))
     ws, ids, wt, xb, yb = _host_inputs(w, cal_T)
-    t0 = time.perf_counter()
-    _oracle_step(oracle, ws, ids, wt, xb, yb)
-    per_tok = (time.perf_counter() - t0) / cal_T
-    T_s = int(max(1, min(w.T, budget_s / max(steps, 1) / max(per_tok, 1e-9))))
+    with ctx:
+        _oracle_step(oracle, ws, ids, wt, xb, yb)  # first call pays the loader
+        t0 = time.perf_counter()
+        _oracle_step(oracle, ws, ids, wt, xb, yb)
+        per_tok = (time.perf_counter() - t0) / cal_T
+    T_s = int(max(1, min(w.T, step_budget_s / max(per_tok, 1e-9))))
     ws, ids, wt, xb, yb = _host_inputs(w, T_s)
-    return dict(T_s=T_s, run=lambda: _oracle_step(oracle, ws, ids, wt, xb, yb),
-                sample=f"first {T_s} of {w.T} tokens of {w.name} per step")
+
+    def run():
+        with (oracle.openmp() if openmp else _null_ctx()):
+            _oracle_step(oracle, ws, ids, wt, xb, yb)
+    return T_s, run
+
+
+class _null_ctx:
+    def __enter__(self):
+        return None
+
+    def __exit__(self, *a):
+        return False
+
+
+def time_oracle(w, budget_s=12.0, openmp=False):
+    """The oracle's whole step (prepare, dispatch, combine) on a bounded token
+    sample of ``w``, repeated until ``budget_s`` has passed (at least twice):
+    tokens per second, the threads it used and what the sample was."""
+    import oracle
+    T_s, run = oracle_sample_plan(w, budget_s / 4, openmp)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        n += 1
+        if n >= 2 and time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    cores = oracle.threads(openmp)
+    build = ("the same C source built with OpenMP over the dispatch and combine rows "
+             "(prepare one thread)" if openmp else "plain single-threaded build")
+    return {"value": T_s * n / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} oracle steps on the first {T_s} of {w.T} tokens of {w.name}",
+            "build": build}
+
+
+def cpu_baseline(w, budget_s):
+    """The oracle timed on the host cores: the OpenMP build on every core
+    (the line's value and core count) and the plain build on one core."""
+    multi = time_oracle(w, budget_s * 0.4, openmp=True)
+    single = time_oracle(w, budget_s * 0.6, openmp=False)
+    out = dict(multi)
+    out["single_core"] = {k: single[k] for k in ("value", "cores", "sample", "build")}
+    return out
 
 
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import oracle
     K, W = args.steps, args.warmup
-    plan = time_oracle(w, budget_s=args.ref_budget, steps=K + W)
+    T_s, run = oracle_sample_plan(w, args.ref_budget / (K + W))
     for _ in range(W):
-        plan["run"]()
+        run()
     t0 = time.perf_counter()
     for _ in range(K):
-        plan["run"]()
+        run()
     dt = time.perf_counter() - t0
-    value = plan["T_s"] * K / dt
+    value = T_s * K / dt
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": K, "warmup": W, "ms_per_step": dt / K * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": _dtype_tag(w),
         "data": "synthetic",
         "config": _config(w, args.gpus),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": plan["sample"]},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.threads(),
+                         "kind": "oracle",
+                         "sample": f"first {T_s} of {w.T} tokens of {w.name} per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -259,8 +300,13 @@ def _config(w, n):
     return {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "k": w.k,
             "routing": w.routing.mode, "x_dtype": w.x_dtype, "dispatch_dtype": w.dispatch_dtype,
             "y_dtype": w.y_dtype, "out_dtype": w.out_dtype, "seed": w.seed,
-            "l2": "no flush: per-step working set > 126 MB L2",
+            "l2": ("no flush: per-step working set > 126 MB L2" if _step_bytes(w) > L2_BYTES
+                   else "no flush: the working set fits in L2 (a latency figure)"),
             "parallelism": "replicas" if n > 1 else "single GPU"}
+
+
+def _step_bytes(w):
+    return sum(algorithmic_bytes(w).values())
 
 
 # ---------------------------------------------------------------------------
@@ -405,18 +451,14 @@ def whole_job_tokens_per_s(T: int, steps: int, world: int, max_elapsed_ms: float
     return T * steps * world / (max_elapsed_ms * 1e-3)
 
 
-def run_gpu(args, w):
+def bench_workload(args, w, dev, ranks, cpu_budget_s):
+    """Times one workload: the eager per-call breakdown, the graph-replayed
+    headline steps, the end-to-end figure from host buffers and the steps
+    beside the path; returns the fields of its JSON entry (rank 0)."""
     import torch
 
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    ranks = Ranks("nccl", dev)
-    world, rank = ranks.world, ranks.rank
-    if world != args.gpus:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    world, rank, local = ranks.world, ranks.rank, ranks.local
     barrier, max_over_ranks = ranks.barrier, ranks.max_over_ranks
-
     step = Step(w, dev)
     K, W = args.steps, args.warmup
     stream = torch.cuda.current_stream(dev)
@@ -502,20 +544,17 @@ def run_gpu(args, w):
     # ---- end to end through the public API from pinned host buffers
     e2e = run_e2e(step, w, dev, K, W, barrier, max_over_ranks)
     next_rows = time_next_rows(step, w, dev)
+    fused, launches_per_step = step.fused, step.launches_per_step
+    del step
+    torch.cuda.empty_cache()
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        r = time_oracle(w, budget_s=args.cpu_budget)
-        cpu = {"value": r["tokens"] / r["seconds"], "unit": "tokens/s", "cores": 1,
-               "kind": "oracle", "sample": r["sample"]}
-
-    ranks.close()
+    cpu = cpu_baseline(w, cpu_budget_s) if (cpu_budget_s > 0 and rank == 0 and world == 1) else None
     if rank != 0:
-        return
+        return None
 
     peak, peak_kind = measured_peak()
     alg = algorithmic_bytes(w)
-    if step.fused:  # prepare and dispatch are one launch, timed together
+    if fused:  # prepare and dispatch are one launch, timed together
         alg = {"prepare_dispatch": alg["prepare"] + alg["dispatch"], "combine": alg["combine"]}
         per = {"prepare_dispatch": per["prepare"], "combine": per["combine"], "step": per["step"]}
     calls = [c for c in ("prepare", "dispatch", "prepare_dispatch", "combine") if c in alg]
@@ -524,7 +563,6 @@ def run_gpu(args, w):
     kernel_key = f"{dominant}@{w.name}"
     achieved = alg[dominant] / (kern[dominant] * 1e-3) / 1e9
     elapsed_ms = graph_ms if graph_ms is not None else eager_ms
-    value = whole_job_tokens_per_s(w.T, K, world, elapsed_ms)
     breakdown = {}
     for k in calls:
         gbs = alg[k] / (kern[k] * 1e-3) / 1e9
@@ -539,13 +577,11 @@ def run_gpu(args, w):
         "graph_ms_per_step": None if graph_ms is None else graph_ms / K,
         "effective_gbs": step_alg / (elapsed_ms / K * 1e-3) / 1e9,
         "frac_of_measured_peak": step_alg / (elapsed_ms / K * 1e-3) / 1e9 / peak}
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-        "warmup": W, "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": _dtype_tag(w), "data": "synthetic",
-        "config": dict(_config(w, world),
-                       launch=(f"cuda_graph of {n_graph} steps, replayed {K // n_graph} times"
-                               if graph_ms is not None else "eager")),
+    return {
+        "value": whole_job_tokens_per_s(w.T, K, world, elapsed_ms),
+        "ms_per_step": elapsed_ms / K,
+        "launch": (f"cuda_graph of {n_graph} steps, replayed {K // n_graph} times"
+                   if graph_ms is not None else "eager"),
         "eager_value": whole_job_tokens_per_s(w.T, K, world, eager_ms),
         "roofline": {"bound": "hbm", "kernel": kernel_key, "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
@@ -553,7 +589,7 @@ def run_gpu(args, w):
                      "algorithmic_bytes_per_launch": alg[dominant]},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": (kernels_per_step or step.launches_per_step) * K,
+        "gpu_launches": (kernels_per_step or launches_per_step) * K,
         "gpu_launches_counted_from": ("kernel nodes of the captured step"
                                       if kernels_per_step else "launches per step of each call"),
         "clocks": clocks.summary(),
@@ -565,6 +601,43 @@ def run_gpu(args, w):
                         "imbalance_ratio": float(counts.max() / max(counts.mean(), 1e-9))},
         "diag": diag,
     }
+
+
+def run_gpu(args, names):
+    """Every workload in ``names`` on this rank's GPU; the first is the
+    headline, the others go under "per_workload"."""
+    import torch
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ranks = Ranks("nccl", dev)
+    if ranks.world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={ranks.world}")
+    results = {}
+    for i, name in enumerate(names):
+        budget = 0.0 if args.no_cpu_baseline else args.cpu_budget * (1.0 if i == 0 else 0.5)
+        results[name] = bench_workload(args, CONFIGS[name], dev, ranks, budget)
+    world = ranks.world
+    ranks.close()
+    if ranks.rank != 0:
+        return
+    head_name = names[0]
+    w = CONFIGS[head_name]
+    r = results[head_name]
+    line = {
+        "metric": METRIC, "value": r["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": _dtype_tag(w),
+        "data": "synthetic",
+        "config": dict(_config(w, world), launch=r["launch"]),
+    }
+    line.update({k: v for k, v in r.items() if k not in ("value", "ms_per_step", "launch")})
+    if len(names) > 1:
+        line["per_workload"] = {
+            n: dict(results[n], config=dict(_config(CONFIGS[n], world), launch=results[n]["launch"]),
+                    dtype=_dtype_tag(CONFIGS[n]))
+            for n in names[1:]}
     print(json.dumps(line), flush=True)
 
 
@@ -621,20 +694,26 @@ def time_next_rows(step, w, dev, reps=20):
 
 def run_e2e(step, w, dev, K, W, barrier, max_over_ranks):
     """Same step through the public API with inputs copied in from pinned
-    host memory and the combined output read back, every step.  The copies
-    run on their own streams, double-buffered, so that step i+1's inputs
-    cross the host link while step i computes and step i-1's output is read
-    back (the way a serving loop streams batches); every step's copies are
-    inside the timed region."""
+    host memory and the combined output read back, every step, all inside
+    the timed region.  Two forms:
+
+    * pipelined (the value): the copies run on their own streams with two
+      sets of device buffers and two pinned outputs, so that step i+1's
+      inputs cross the host link while step i computes and step i-1's output
+      is read back (the way a serving loop streams batches);
+    * serialized: one stream, copy in, compute, copy out, step after step.
+
+    After the timed region one read-back output of each form is checked
+    against the device result of the same inputs."""
     import copy as _copy
     import torch
     h_ids = torch.from_numpy(step.ids_np).pin_memory()
     h_wt = torch.from_numpy(step.wt_np).pin_memory()
     h_x = step.x.cpu().pin_memory()
     h_y = step.y.cpu().pin_memory()
-    h_out = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    h_out = [torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in (h_ids, h_wt, h_x, h_y))
-    d2h = h_out.numel() * h_out.element_size()
+    d2h = h_out[0].numel() * h_out[0].element_size()
     comp = torch.cuda.current_stream(dev)
     n = max(1, min(K, 20))
 
@@ -649,18 +728,22 @@ def run_e2e(step, w, dev, K, W, barrier, max_over_ranks):
     comp_done = [torch.cuda.Event(), torch.cuda.Event()]
     d2h_done = [torch.cuda.Event(), torch.cuda.Event()]
 
-    def run(count):
+    def load(st, s):
+        with torch.cuda.stream(s):
+            st.ids.copy_(h_ids, non_blocking=True)
+            st.wt.copy_(h_wt, non_blocking=True)
+            st.x.copy_(h_x, non_blocking=True)
+            st.y.copy_(h_y, non_blocking=True)
+
+    def pipelined(count):
         for i in range(count):
             b = i % 2
             st = bufs[b]
             with torch.cuda.stream(copy_s):
                 if i >= 2:
                     copy_s.wait_event(comp_done[b])  # step i-2 has read these inputs
-                st.ids.copy_(h_ids, non_blocking=True)
-                st.wt.copy_(h_wt, non_blocking=True)
-                st.x.copy_(h_x, non_blocking=True)
-                st.y.copy_(h_y, non_blocking=True)
-                h2d_done[b].record(copy_s)
+            load(st, copy_s)
+            h2d_done[b].record(copy_s)
             comp.wait_event(h2d_done[b])
             if i >= 2:
                 comp.wait_event(d2h_done[b])  # step i-2's output has been read back
@@ -668,23 +751,38 @@ def run_e2e(step, w, dev, K, W, barrier, max_over_ranks):
             comp_done[b].record(comp)
             with torch.cuda.stream(d2h_s):
                 d2h_s.wait_event(comp_done[b])
-                h_out.copy_(st.out, non_blocking=True)
+                h_out[b].copy_(st.out, non_blocking=True)
                 d2h_done[b].record(d2h_s)
 
-    run(min(W, 3))
-    torch.cuda.synchronize(dev)
-    barrier()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record(copy_s)
-    run(n)
-    e.record(d2h_s)
-    torch.cuda.synchronize(dev)
-    barrier()
-    ms = max_over_ranks(s.elapsed_time(e))
+    def serialized(count):
+        for _ in range(count):
+            load(step, comp)
+            step.run()
+            h_out[0].copy_(step.out, non_blocking=True)
+
+    def timed(fn, first, last):
+        fn(min(W, 3))
+        torch.cuda.synchronize(dev)
+        barrier()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(first)
+        fn(n)
+        e.record(last)
+        torch.cuda.synchronize(dev)
+        barrier()
+        return max_over_ranks(s.elapsed_time(e))
+
+    ms_pipe = timed(pipelined, copy_s, d2h_s)
+    ok_pipe = bool(torch.equal(h_out[(n - 1) % 2], bufs[(n - 1) % 2].out.cpu()))
+    ms_ser = timed(serialized, comp, comp)
+    ok_ser = bool(torch.equal(h_out[0], step.out.cpu()))
     world = int(os.environ.get("WORLD_SIZE", "1"))
-    return {"value": w.T * n * world / (ms * 1e-3), "unit": "tokens/s", "steps": n,
+    return {"value": w.T * n * world / (ms_pipe * 1e-3), "unit": "tokens/s", "steps": n,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "copies": "own streams, double-buffered, overlapping the compute"}
+            "copies": "own streams, double-buffered, overlapping the compute",
+            "serialized": {"value": w.T * n * world / (ms_ser * 1e-3), "unit": "tokens/s",
+                           "copies": "one stream: copy in, compute, copy out"},
+            "read_back_matches_device": ok_pipe and ok_ser}
 
 
 def main():
@@ -692,20 +790,24 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(CONFIGS))
+    ap.add_argument("--workload", default="all", choices=["all"] + sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle time")
+    ap.add_argument("--cpu-budget", type=float, default=10.0,
+                    help="seconds of oracle time per workload (headline); half that for the others")
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="seconds of oracle time for the whole reference run")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    w = CONFIGS[args.workload]
-    if args.impl == "reference":
-        run_reference(args, w)
+    if args.workload == "all":
+        names = [HEADLINE_WORKLOAD] + [n for n in CONFIGS if n != HEADLINE_WORKLOAD]
     else:
-        run_gpu(args, w)
+        names = [args.workload]
+    if args.impl == "reference":
+        run_reference(args, CONFIGS[names[0]])
+    else:
+        run_gpu(args, names)
 
 
 if __name__ == "__main__":

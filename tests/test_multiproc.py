@@ -65,7 +65,7 @@ def test_reference_arm_single_process():
     assert len(lines) == 1
     d = lines[0]
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
-    assert d["config"]["workload"] == "uniform_t4096_h7168_e256_k8"
+    assert d["config"]["workload"] == "zipf_fp16_t131072_h2048_e64_k6"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
