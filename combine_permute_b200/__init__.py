@@ -27,6 +27,8 @@ __all__ = [
     "moe_prepare",
     "moe_prepare_workspace_bytes",
     "moe_dispatch_rows",
+    "moe_dispatch_error",
+    "moe_set_wait_limits",
     "moe_dispatch_rows_fp8",
     "moe_dispatch_rows_nvfp4",
     "moe_combine",
@@ -207,6 +209,28 @@ def moe_dispatch_rows(x: torch.Tensor, top_k: int, input_permutation: Optional[t
                                            out.data_ptr(), _stream(dev))
     _lib.check("moe_dispatch_rows", st)
     return out
+
+
+def moe_dispatch_error(device=None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Enqueues the read-and-clear of the TMA dispatch's error word on the
+    current stream of ``device``; returns the int32 [1] device tensor it is
+    written to (1: a bounded wait gave up since the last query, rows are
+    incomplete; 0 otherwise).  See include/moe.h."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if out is None:
+        out = torch.empty(1, dtype=torch.int32, device=dev)
+    _need(out, "out", torch.int32, (1,), dev)
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_dispatch_error(out.data_ptr(), _stream(dev))
+    _lib.check("moe_dispatch_error", st)
+    return out
+
+
+def moe_set_wait_limits(prepare_wait_us: int = -1, dispatch_polls: int = -1) -> None:
+    """Limits of the library's bounded waits (negative: the default), for
+    tests of the failure reporting.  See include/moe.h."""
+    _lib.check("moe_set_wait_limits",
+               _lib.load().moe_set_wait_limits(int(prepare_wait_us), int(dispatch_polls)))
 
 
 def moe_dispatch_rows_fp8(x: torch.Tensor, top_k: int, output_permutation: torch.Tensor,

@@ -29,6 +29,8 @@ EXPORTED = (
     "moe_prepare_workspace_bytes",
     "moe_prepare",
     "moe_dispatch_rows",
+    "moe_dispatch_error",
+    "moe_set_wait_limits",
     "moe_dispatch_rows_fp8",
     "moe_dispatch_rows_nvfp4",
     "moe_combine",
@@ -53,6 +55,8 @@ _SIGNATURES = {
     "moe_prepare": (_int, [_vp, _i64, _i32, _i32, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp,
                            ctypes.c_size_t, _vp]),
     "moe_dispatch_rows": (_int, [_vp, _int, _i64, _i64, _i32, _vp, _vp, _vp, _vp]),
+    "moe_dispatch_error": (_int, [_vp, _vp]),
+    "moe_set_wait_limits": (_int, [_i64, _i64]),
     "moe_dispatch_rows_fp8": (_int, [_vp, _int, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp,
                                      _vp, _vp]),
     "moe_dispatch_rows_nvfp4": (_int, [_vp, _int, _i64, _i64, _i32, _i32, _vp, _vp, _vp, _vp,

@@ -6,6 +6,7 @@
 
 #include "moe.h"
 #include "kernels.h"
+#include "launch.h"
 
 namespace {
 
@@ -147,6 +148,20 @@ moe_status_t moe_dispatch_rows(const void *x, moe_dtype_t dtype, int64_t num_tok
                                                    output_permutation, out, (cudaStream_t)stream));
     return from_cuda(moe::run_dispatch_gather(x, num_tokens, row_bytes, top_k, input_permutation,
                                               out, (cudaStream_t)stream));
+}
+
+moe_status_t moe_dispatch_error(int32_t *error, moe_stream_t stream) {
+    if (!error) return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_dispatch_error(error, (cudaStream_t)stream));
+}
+
+moe_status_t moe_set_wait_limits(int64_t prepare_wait_us, int64_t dispatch_polls) {
+    moe::prepare_wait_ns().store(prepare_wait_us < 0 ? moe::kDefaultPrepareWaitNs
+                                                     : (uint64_t)prepare_wait_us * 1000ull);
+    moe::dispatch_polls().store(dispatch_polls < 0 ? moe::kDefaultDispatchPolls
+                                : dispatch_polls > 0xffffffffll ? 0xffffffffu
+                                                                : (uint32_t)dispatch_polls);
+    return MOE_OK;
 }
 
 moe_status_t moe_dispatch_rows_fp8(const void *x, moe_dtype_t x_dtype, int64_t num_tokens,

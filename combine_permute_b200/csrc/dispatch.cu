@@ -1,14 +1,17 @@
 // Dispatch: lay token rows out grouped by expert (sglang PR #19058,
 // "Changes", item 2 shuffle_rows: dtype-agnostic row gather with 128-bit
-// vector accesses), and the same with a fused FP8 E4M3 1x128 block-scale
-// quantisation (the FP8 block-scale MoE path of TensorRT-LLM PR #9592).
+// vector accesses), and the same with a fused FP8 E4M3 1x128 block-scale or
+// NVFP4 quantisation (the FP8 block-scale and NVFP4 MoE paths of
+// TensorRT-LLM PR #9592).
 //
-// dispatch_scatter_kernel walks tokens: it reads each x row once into
-// registers (16-byte vectors) and stores it to the token's k dispatched
-// rows, so x crosses HBM once although it is written k times.
-// dispatch_gather_kernel walks dispatched rows and reads the source row
-// through input_permutation (the literal shuffle_rows form).
-// Both are persistent grid-stride kernels sized to fill every SM once.
+// dispatch_bulk_kernel is the scatter form on the TMA engine: it walks
+// tokens, stages each x row in shared memory once and bulk-stores it to the
+// token's k dispatched rows, so x crosses HBM once although it is written k
+// times.  dispatch_gather_kernel walks dispatched rows and reads the source
+// row through input_permutation (the literal shuffle_rows form, 16-byte
+// vectors).  dispatch_quant_kernel quantises each token row once and stores
+// the codes to its k rows.  All are persistent kernels sized to fill every
+// SM once.
 #include "kernels.h"
 #include "launch.h"
 #include "moe_device.cuh"
@@ -36,14 +39,15 @@ constexpr int kBulkMaxStages = 16;
 constexpr uint32_t kBulkSmem = 64 * 1024;   // stage ring per block
 constexpr int kQuantThreads = 256;          // quantised dispatch: target threads per block
 constexpr int kQuantMaxThreads = 512;       // and the most
-constexpr uint32_t kMaxPolls = 1u << 24;    // bounded mbarrier wait (each poll suspends briefly)
 
-__device__ unsigned g_dispatch_error;  // set when a bounded wait gave up
+// Set to 1 by a bulk dispatch block whose bounded wait for a staged chunk gave
+// up (its rows are then incomplete); read and cleared by dispatch_error_kernel.
+__device__ unsigned g_dispatch_error;
 
 __global__ void __launch_bounds__(32)
     dispatch_bulk_kernel(const char *__restrict__ x, int64_t T, int64_t row_bytes, int k,
                          const int32_t *__restrict__ out_perm, char *__restrict__ out,
-                         int64_t nch, uint32_t chunk, int stages) {
+                         int64_t nch, uint32_t chunk, int stages, uint32_t max_polls) {
     extern __shared__ __align__(128) unsigned char stage[];  // stages * chunk
     __shared__ __align__(8) uint64_t bar[kBulkMaxStages];
     const int lane = threadIdx.x;
@@ -85,7 +89,7 @@ __global__ void __launch_bounds__(32)
             const int j = lane + 32 * h;
             p[h] = j < k ? __ldg(out_perm + t * k + j) : -1;
         }
-        const bool ok = mbar_wait(&bar[s], (uint32_t)((n / stages) & 1), kMaxPolls);
+        const bool ok = mbar_wait(&bar[s], (uint32_t)((n / stages) & 1), max_polls);
         if (!__all_sync(0xffffffffu, ok)) {
             failed = true;
             break;
@@ -109,11 +113,18 @@ __global__ void __launch_bounds__(32)
     if (failed) {
         if (lane == 0) atomicExch(&g_dispatch_error, 1u);
         // let every load still in flight land before the block releases its
-        // shared memory (again bounded)
+        // shared memory (bounded by the default limit, whatever max_polls is)
         for (int64_t m = n; m < issued; ++m)
-            mbar_wait(&bar[m % stages], (uint32_t)((m / stages) & 1), kMaxPolls);
+            mbar_wait(&bar[m % stages], (uint32_t)((m / stages) & 1), kDefaultDispatchPolls);
     }
     bulk_wait_all();
+}
+
+// Copies the error word to *out and clears it (one thread).
+__global__ void dispatch_error_kernel(int32_t *out) {
+    pdl_wait();
+    pdl_launch_dependents();
+    *out = (int32_t)atomicExch(&g_dispatch_error, 0u);
 }
 
 __global__ void __launch_bounds__(kCopyThreads)
@@ -416,7 +427,11 @@ cudaError_t run_dispatch_scatter_split(const void *x, int64_t T, int64_t row_byt
     const size_t smem = (size_t)stages * chunk;
     const int64_t grid = persistent_grid(dispatch_bulk_kernel, 32, smem, T * nch);
     return launch(dispatch_bulk_kernel, grid, 32, smem, stream, (const char *)x, T, row_bytes, k,
-                  out_perm, (char *)out, nch, chunk, stages);
+                  out_perm, (char *)out, nch, chunk, stages, dispatch_polls().load());
+}
+
+cudaError_t run_dispatch_error(int32_t *out, cudaStream_t stream) {
+    return launch(dispatch_error_kernel, 1, 1, 0, stream, out);
 }
 
 cudaError_t run_dispatch_scatter(const void *x, int64_t T, int64_t row_bytes, int k,

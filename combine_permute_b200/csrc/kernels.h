@@ -42,6 +42,10 @@ cudaError_t run_dispatch_scatter_split(const void *x, int64_t T, int64_t row_byt
                                        const int32_t *out_perm, void *out, int64_t nsplit,
                                        cudaStream_t stream);
 
+// Writes the bulk dispatch's error word (1: a bounded wait gave up since
+// the last query) to *out and clears it.
+cudaError_t run_dispatch_error(int32_t *out, cudaStream_t stream);
+
 cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int k,
                                 const int32_t *in_perm, void *out, cudaStream_t stream);
 

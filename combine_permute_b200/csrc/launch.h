@@ -5,11 +5,30 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <map>
 #include <mutex>
 #include <tuple>
 
 namespace moe {
+
+// Limits of the bounded waits, read at every launch: how long a prepare
+// block waits for the other blocks (nanoseconds of the GPU's global timer,
+// default one second), and how many mbarrier polls the TMA dispatch makes
+// for one staged chunk before it gives up.  Only moe_set_wait_limits
+// changes them (tests of the failure reporting).
+constexpr uint64_t kDefaultPrepareWaitNs = 1000000000ull;
+constexpr uint32_t kDefaultDispatchPolls = 1u << 24;
+
+inline std::atomic<uint64_t> &prepare_wait_ns() {
+    static std::atomic<uint64_t> v{kDefaultPrepareWaitNs};
+    return v;
+}
+
+inline std::atomic<uint32_t> &dispatch_polls() {
+    static std::atomic<uint32_t> v{kDefaultDispatchPolls};
+    return v;
+}
 
 inline int current_device() {
     int d = 0;

@@ -37,7 +37,6 @@ namespace {
 
 constexpr unsigned long long kFlagAgg = 1ull << 32;   // word holds this tile's aggregate
 constexpr unsigned long long kFlagIncl = 2ull << 32;  // word holds the inclusive prefix
-constexpr int kMaxSpins = 1 << 20;  // x ~256 ns sleep: a wait gives up after ~0.3-1 s
 constexpr int kLookbackWindow = 8;  // predecessor tiles read together
 
 constexpr int kSingleThreads = 1024;
@@ -148,30 +147,43 @@ __device__ __forceinline__ int offsets_from_totals(int *tot, int *pad, int E, in
 
 __host__ __device__ inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
-// Workspace of the tiled path: a 256-byte header, then one 64-bit look-back
-// word per (tile, expert column).  A word holds epoch << 34 | flag << 32 |
-// value; it counts as published by this call only when its epoch field is
-// this call's epoch, so words left by earlier calls need no clearing.  The
-// epoch advances once per call (by the call's last block); the ticket and
-// done counters wrap back to zero.
+// Workspace of the tiled paths: a 256-byte header, then one 64-bit
+// look-back word per (tile, expert column) of the two-kernel path, then one
+// int32 histogram row per block of the one-launch path.  A look-back word
+// holds epoch << 34 | flag << 32 | value; it counts as published by this
+// call only when its epoch field is this call's epoch, so words left by
+// earlier calls need no clearing.  The epoch advances once per call (by the
+// call's last block); the ticket, done and barrier counters return to zero
+// at the end of every call.  The histogram rows are written before the grid
+// barrier and read after it, so they need no clearing either.
 struct PrepWs {
-    unsigned *ticket;   // tile tickets, wraps at G
-    unsigned *done;     // blocks finished, wraps at G
-    unsigned *epoch;    // this call's epoch
-    unsigned *ready;    // one-pass path: epoch + 1 once the offsets are out
-    unsigned *timeout;  // set when a bounded wait gave up
+    unsigned *ticket;     // tile tickets, wraps at G
+    unsigned *done;       // blocks finished, wraps at G
+    unsigned *epoch;      // this call's epoch
+    unsigned *timeout;    // set when a bounded wait gave up
+    unsigned *bar_count;  // one-launch path: blocks arrived at the grid barrier
+    unsigned *bar_gen;    // one-launch path: barrier generation
     unsigned long long *state;  // [G][E+1] look-back words
+    int *hist;                  // [G'][E+1] histogram rows, G' <= kMaxSyncTiles
 };
 
-__host__ __device__ inline PrepWs carve(void *ws) {
+// Most blocks of one one-launch prepare (one block per SM on B200, with room
+// for parts with more SMs); it bounds the histogram rows of the workspace.
+constexpr int kMaxSyncTiles = 256;
+
+__host__ __device__ inline int64_t tiles_of(int64_t S) { return (S + kTileSlots - 1) / kTileSlots; }
+
+__host__ __device__ inline PrepWs carve(void *ws, int64_t S, int E) {
     char *b = (char *)ws;
     PrepWs w;
     w.ticket = (unsigned *)b;
     w.done = (unsigned *)(b + 4);
     w.epoch = (unsigned *)(b + 8);
-    w.ready = (unsigned *)(b + 12);
     w.timeout = (unsigned *)(b + 16);
+    w.bar_count = (unsigned *)(b + 20);
+    w.bar_gen = (unsigned *)(b + 24);
     w.state = (unsigned long long *)(b + 256);
+    w.hist = (int *)(b + 256 + align256((size_t)tiles_of(S) * ((size_t)E + 1) * 8));
     return w;
 }
 
@@ -351,32 +363,27 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
 size_t single_block_smem(int E) { return (size_t)(kSingleWarps * (E + 1) + 2 * E) * sizeof(int); }
 
 // ---------------------------------------------------------------------------
-// Tiled path.  A tile is kTileSlots consecutive slots, ranked by a block of
-// NT threads (NT / 32 warps, kTileSlots / NT rounds of 32 slots per warp).
-// tile_rank() ranks a tile's slots within each warp's run and folds the warps
-// into the tile histogram: hist[c] for c < E is the tile's count of expert c,
-// hist[E] its count of invalid ids; wcnt holds the per-warp exclusive
-// prefixes and key/rank each thread's slots.
+// Tiled paths.  A tile is a run of consecutive slots ranked by one block of
+// NT threads: warp w takes nr rounds of 32 consecutive slots starting at
+// first + w * 32 * nr (nr <= NR, the register capacity).  rank_tile() ranks
+// the slots within each warp's run and folds the warps into the tile
+// histogram: hist[c] for c < E is the tile's count of expert c, hist[E] its
+// count of invalid ids; wcnt holds the per-warp exclusive prefixes and
+// key / rank each thread's slots.
 // ---------------------------------------------------------------------------
-template <int NT> struct TileShape {
-    static constexpr int kWarps = NT / 32;
-    static constexpr int kRounds = kTileSlots / NT;
-    static_assert(NT * kRounds == kTileSlots, "a tile is kTileSlots slots");
-};
-
-template <typename IdT, int NT>
-__device__ __forceinline__ void tile_rank(const IdT *__restrict__ ids, int64_t base, int64_t S,
-                                          int E, int tile, int *wcnt, int *hist, int *s_invalid,
-                                          int (&key)[TileShape<NT>::kRounds],
-                                          int (&rank)[TileShape<NT>::kRounds]) {
-    constexpr int NW = TileShape<NT>::kWarps, NR = TileShape<NT>::kRounds;
+template <typename IdT, int NT, int NR>
+__device__ __forceinline__ void rank_tile(const IdT *__restrict__ ids, int64_t base, int64_t S,
+                                          int E, int64_t first, int nr, int *wcnt, int *hist,
+                                          int *s_invalid, int (&key)[NR], int (&rank)[NR]) {
+    constexpr int NW = NT / 32;
     const int C = E + 1;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned lt = lanemask_lt();
     const int nbits = key_bits(E);
-    const int64_t wbase = (int64_t)tile * kTileSlots + (int64_t)warp * 32 * NR;
+    const int64_t wbase = first + (int64_t)warp * 32 * nr;
 #pragma unroll
-    for (int r = 0; r < NR; ++r) key[r] = load_key(ids, wbase + r * 32 + lane, S, base, E);
+    for (int r = 0; r < NR; ++r)
+        key[r] = r < nr ? load_key(ids, wbase + r * 32 + lane, S, base, E) : -2;
     for (int x = tid; x < NW * C; x += NT) wcnt[x] = 0;
     if (tid == 0) *s_invalid = 0;
     __syncthreads();
@@ -384,7 +391,7 @@ __device__ __forceinline__ void tile_rank(const IdT *__restrict__ ids, int64_t b
     int bad = 0;
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
-        rank[r] = rank_round(key[r], E, nbits, row, lt);
+        if (r < nr) rank[r] = rank_round(key[r], E, nbits, row, lt);
         bad += key[r] == -1;
     }
 #pragma unroll
@@ -399,20 +406,18 @@ __device__ __forceinline__ void tile_rank(const IdT *__restrict__ ids, int64_t b
 // Both permutations of a tile's slots: row = off[e] (expert offset, or 0) +
 // excl[e] (earlier tiles) + wcnt (earlier warps) + rank (earlier lanes and
 // rounds).  When `in_perm` is null only the rank part goes to out_perm.
-template <int NT>
-__device__ __forceinline__ void tile_write_rows(int64_t S, int E, int tile, const int *off,
-                                                const int *excl, const int *wcnt,
-                                                const int (&key)[TileShape<NT>::kRounds],
-                                                const int (&rank)[TileShape<NT>::kRounds],
+template <int NT, int NR>
+__device__ __forceinline__ void write_tile_rows(int64_t S, int E, int64_t first, int nr,
+                                                const int *off, const int *excl, const int *wcnt,
+                                                const int (&key)[NR], const int (&rank)[NR],
                                                 int32_t *in_perm, int32_t *out_perm) {
-    constexpr int NR = TileShape<NT>::kRounds;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t wbase = (int64_t)tile * kTileSlots + (int64_t)warp * 32 * NR;
+    const int64_t wbase = first + (int64_t)warp * 32 * nr;
     const int *row = wcnt + warp * (E + 1);
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
         const int64_t i = wbase + r * 32 + lane;
-        if (i < S) {
+        if (r < nr && i < S) {
             const int e = key[r];
             const int p = e >= 0 ? (off ? off[e] : 0) + excl[e] + row[e] + rank[r] : -1;
             out_perm[i] = p;
@@ -427,7 +432,8 @@ __device__ __forceinline__ void tile_write_rows(int64_t S, int E, int tile, cons
 // inclusive prefix.  excl[c] receives the slots of column c in earlier tiles.
 template <int NT>
 __device__ __forceinline__ void tile_lookback(const PrepWs &ws, int tile, unsigned epoch, int E,
-                                              const int *hist, int *excl) {
+                                              const int *hist, int *excl,
+                                              unsigned long long wait_ns) {
     const int C = E + 1;
     unsigned long long *mine = ws.state + (size_t)tile * C;
     for (int c = threadIdx.x; c < C; c += NT)
@@ -445,13 +451,15 @@ __device__ __forceinline__ void tile_lookback(const PrepWs &ws, int tile, unsign
             for (int q = 0; q < kLookbackWindow; ++q) {
                 if (done || gave_up || pred - q < 0) continue;
                 const unsigned long long *wp = ws.state + (size_t)(pred - q) * C + c;
-                int spins = 0;
+                unsigned long long t0 = 0;
                 while (lb_flag(v[q], epoch) == 0) {  // not published by this call yet
-                    if (++spins > kMaxSpins) {
+                    const unsigned long long now = globaltimer_ns();
+                    if (t0 == 0) t0 = now;
+                    if (now - t0 >= wait_ns) {
                         gave_up = true;
                         break;
                     }
-                    __nanosleep(256);
+                    __nanosleep(128);
                     v[q] = ld_relaxed_u64(wp);
                 }
                 sum += (int)(unsigned)(v[q] & 0xffffffffu);
@@ -481,105 +489,128 @@ __device__ __forceinline__ void tile_finish(const PrepWs &ws, int G, unsigned ep
     }
 }
 
+constexpr int kRankThreads = 256;                  // two-kernel tiles: 8 warps
+constexpr int kRankRounds = kTileSlots / kRankThreads;  // of 8 rounds
+constexpr int kSyncThreads = 512;                  // one-launch tiles: 16 warps
+constexpr int kSyncMaxRounds = 16;                 // of up to 16 rounds (8192 slots)
+constexpr int kSyncMinRounds = 4;
+
 // Shared memory of the tiled kernels: per-warp rows, then hist, excl, off,
-// pad (one column per expert plus one for invalid ids each).
-template <int NT> size_t tile_smem(int E) {
-    return (size_t)(TileShape<NT>::kWarps + 4) * (E + 1) * sizeof(int);
+// pad (one column per expert plus one for invalid ids each); the one-launch
+// kernel adds the G histogram rows it stages.
+template <int NT> size_t tile_smem(int E, int G = 0) {
+    return (size_t)(NT / 32 + 4 + G) * (E + 1) * sizeof(int);
 }
 
-constexpr int kOnepassThreads = 512;  // one-pass tiles: 16 warps of 4 rounds
-
-// One-pass variant (every tile resident at once: a cooperative launch, so
-// tile = blockIdx.x and a tile may wait on any other).  Each tile ranks its
-// slots and runs the look-back; the last tile turns the totals into offsets,
-// writes them and raises `ready`; every other tile waits for it (bounded),
-// reads the offsets and writes its slots' final rows into both
-// permutations.
+// One-launch prepare (a cooperative launch: every block resident, so blocks
+// may wait on one another).  Block b ranks slots [b*nr*NT, (b+1)*nr*NT),
+// publishes its histogram row and arrives at a grid barrier (bounded wait).
+// After it, every block stages all G rows in shared memory, sums them into
+// the totals and its own exclusive prefix over earlier blocks, scans the
+// totals into the expert offsets (block 0 writes counts, offsets and
+// block-scale offsets) and writes its slots' rows into both permutations.
 template <typename IdT>
-__global__ void __launch_bounds__(kOnepassThreads, 1)
-    prep_onepass_kernel(const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int A, int G,
-                        void *workspace, int32_t *counts, int32_t *offsets, int32_t *bso,
-                        int32_t *in_perm, int32_t *out_perm, int32_t *diag) {
-    constexpr int NT = kOnepassThreads;
+__global__ void __launch_bounds__(kSyncThreads, 1)
+    prep_sync_kernel(const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int A, int G,
+                     int nr, void *workspace, unsigned long long wait_ns, int32_t *counts,
+                     int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,
+                     int32_t *diag) {
+    constexpr int NT = kSyncThreads, NW = NT / 32, NR = kSyncMaxRounds;
     extern __shared__ int smem[];
     __shared__ int warp_tmp[66];
     __shared__ unsigned s_epoch;
-    __shared__ int s_invalid, s_total;
+    __shared__ int s_invalid;
     const int C = E + 1;
-    int *wcnt = smem;                              // [NW][C]
-    int *hist = wcnt + TileShape<NT>::kWarps * C;  // [C]
-    int *excl = hist + C;                          // [C]
-    int *off = excl + C;                           // [C] expert offsets
-    int *pad = off + C;                            // [C] scan scratch
+    int *wcnt = smem;           // [NW][C]
+    int *hist = wcnt + NW * C;  // [C] this tile's counts
+    int *excl = hist + C;       // [C] earlier tiles' counts
+    int *tot = excl + C;        // [C] totals, then expert offsets
+    int *pad = tot + C;         // [C] scan scratch
+    int *rows = pad + C;        // [G][C] every tile's counts
     const int tid = threadIdx.x;
     const int tile = blockIdx.x;
-    PrepWs ws = carve(workspace);
+    const int64_t first = (int64_t)tile * nr * NT;
+    PrepWs ws = carve(workspace, S, E);
     pdl_wait();
     pdl_launch_dependents();
-    if (tid == 0) s_epoch = *(volatile unsigned *)ws.epoch;
-    int key[TileShape<NT>::kRounds], rank[TileShape<NT>::kRounds];
-    tile_rank<IdT, NT>(ids, base, S, E, tile, wcnt, hist, &s_invalid, key, rank);
-    const unsigned epoch = s_epoch;
-    tile_lookback<NT>(ws, tile, epoch, E, hist, excl);
-    if (tile == G - 1) {
-        // totals = earlier tiles + this one; offsets out, then release the others
-        for (int c = tid; c < C; c += NT) off[c] = excl[c] + hist[c];
-        __syncthreads();
-        if (tid == 0 && diag) diag[0] = off[E];
-        const int total = offsets_from_totals(off, pad, E, A, true, counts, offsets, bso, warp_tmp);
-        if (tid == 0) {
-            s_total = total;
+    if (tid == 0) s_epoch = ld_relaxed_u32(ws.epoch);
+    int key[NR], rank[NR];
+    rank_tile<IdT, NT, NR>(ids, base, S, E, first, nr, wcnt, hist, &s_invalid, key, rank);
+    for (int c = tid; c < C; c += NT) ws.hist[(size_t)tile * C + c] = hist[c];
+    __syncthreads();
+    if (tid == 0) {  // grid barrier: arrive, then wait for the generation to move
+        const unsigned gen = ld_relaxed_u32(ws.bar_gen);
+        __threadfence();
+        if (atomicAdd(ws.bar_count, 1u) == (unsigned)(G - 1)) {
+            atomicExch(ws.bar_count, 0u);
             __threadfence();
-            st_release_u32(ws.ready, epoch + 1);
-        }
-    } else {
-        if (tid == 0) {
-            int spins = 0;
-            while (ld_acquire_u32(ws.ready) != epoch + 1) {
-                if (++spins > kMaxSpins) {
+            st_release_u32(ws.bar_gen, gen + 1);
+        } else {
+            const unsigned long long t0 = globaltimer_ns();
+            while (ld_acquire_u32(ws.bar_gen) == gen) {
+                if (globaltimer_ns() - t0 >= wait_ns) {
                     atomicExch(ws.timeout, 1u);
                     break;
                 }
-                __nanosleep(128);
+                __nanosleep(32);
             }
+            __threadfence();
         }
-        __syncthreads();
-        for (int c = tid; c <= E; c += NT) off[c] = __ldcg(offsets + c);
-        if (tid == 0) s_total = __ldcg(offsets + E);
     }
     __syncthreads();
-    const int total = s_total;
-    tile_write_rows<NT>(S, E, tile, off, excl, wcnt, key, rank, in_perm, out_perm);
-    const int64_t first = (int64_t)tile * kTileSlots;
+    // stage the G rows (L2 only: they were written by other SMs), then sum
+    const int n = G * C;
+    const int *src = ws.hist;
+    if ((n & 3) == 0) {
+        const int4 *s4 = reinterpret_cast<const int4 *>(src);
+        int4 *d4 = reinterpret_cast<int4 *>(rows);
+        for (int x = tid; x < (n >> 2); x += NT) d4[x] = __ldcg(s4 + x);
+    } else {
+        for (int x = tid; x < n; x += NT) rows[x] = __ldcg(src + x);
+    }
+    __syncthreads();
+    for (int c = tid; c < C; c += NT) {
+        int before = 0, all = 0;
+        for (int t = 0; t < G; ++t) {
+            const int v = rows[t * C + c];
+            before += t < tile ? v : 0;
+            all += v;
+        }
+        excl[c] = before;
+        tot[c] = all;
+    }
+    __syncthreads();
+    if (tile == 0 && tid == 0 && diag) diag[0] = tot[E];
+    const int total = offsets_from_totals(tot, pad, E, A, tile == 0, counts, offsets, bso, warp_tmp);
+    write_tile_rows<NT, NR>(S, E, first, nr, tot, excl, wcnt, key, rank, in_perm, out_perm);
     const int64_t lo = first > total ? first : (int64_t)total;
-    const int64_t hi = first + kTileSlots < S ? first + kTileSlots : S;
+    const int64_t end = first + (int64_t)nr * NT;
+    const int64_t hi = end < S ? end : S;
     for (int64_t p = lo + tid; p < hi; p += NT) in_perm[p] = -1;
-    tile_finish(ws, G, epoch, diag);
+    tile_finish(ws, G, s_epoch, diag);
 }
 
 // Two-kernel variant, kernel 1 (any number of tiles): store rank(i) in
 // output_permutation (-1 for an invalid id); the last tile writes counts,
 // offsets and block-scale offsets.  Tiles take their index from an atomic
 // ticket, so a tile only waits on tiles that are already running.
-constexpr int kRankThreads = 256;  // two-kernel tiles: 8 warps of 8 rounds
-
 template <typename IdT>
 __global__ void __launch_bounds__(kRankThreads, 2)
     prep_rank_kernel(const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int A, int G,
-                     void *workspace, int32_t *counts, int32_t *offsets, int32_t *bso,
-                     int32_t *out_perm, int32_t *diag) {
-    constexpr int NT = kRankThreads;
+                     void *workspace, unsigned long long wait_ns, int32_t *counts,
+                     int32_t *offsets, int32_t *bso, int32_t *out_perm, int32_t *diag) {
+    constexpr int NT = kRankThreads, NR = kRankRounds;
     extern __shared__ int smem[];
     __shared__ int warp_tmp[66];
     __shared__ unsigned s_misc[2];
     __shared__ int s_invalid;
     const int C = E + 1;
     int *wcnt = smem;
-    int *hist = wcnt + TileShape<NT>::kWarps * C;
+    int *hist = wcnt + (NT / 32) * C;
     int *excl = hist + C;
     int *off = excl + C;
     int *pad = off + C;
-    PrepWs ws = carve(workspace);
+    PrepWs ws = carve(workspace, S, E);
     pdl_wait();
     pdl_launch_dependents();
     if (threadIdx.x == 0) {
@@ -587,15 +618,16 @@ __global__ void __launch_bounds__(kRankThreads, 2)
         // a counter left non-zero by an aborted call: stay in bounds; the
         // bounded waits then report the failure through diag[1]
         s_misc[0] = t < (unsigned)G ? t : t % (unsigned)G;
-        s_misc[1] = *(volatile unsigned *)ws.epoch;
+        s_misc[1] = ld_relaxed_u32(ws.epoch);
     }
     __syncthreads();
     const int tile = (int)s_misc[0];
     const unsigned epoch = s_misc[1];
-    int key[TileShape<NT>::kRounds], rank[TileShape<NT>::kRounds];
-    tile_rank<IdT, NT>(ids, base, S, E, tile, wcnt, hist, &s_invalid, key, rank);
-    tile_lookback<NT>(ws, tile, epoch, E, hist, excl);
-    tile_write_rows<NT>(S, E, tile, nullptr, excl, wcnt, key, rank, nullptr, out_perm);
+    const int64_t first = (int64_t)tile * kTileSlots;
+    int key[NR], rank[NR];
+    rank_tile<IdT, NT, NR>(ids, base, S, E, first, NR, wcnt, hist, &s_invalid, key, rank);
+    tile_lookback<NT>(ws, tile, epoch, E, hist, excl, wait_ns);
+    write_tile_rows<NT, NR>(S, E, first, NR, nullptr, excl, wcnt, key, rank, nullptr, out_perm);
     if (tile == G - 1) {
         for (int c = threadIdx.x; c < C; c += NT) off[c] = excl[c] + hist[c];
         __syncthreads();
@@ -667,29 +699,49 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
 
 size_t prepare_workspace_bytes(int64_t S, int E) {
     if (S <= kSingleBlockSlots) return 0;
-    const int64_t G = (S + kTileSlots - 1) / kTileSlots;
-    return 256 + align256((size_t)G * ((size_t)E + 1) * 8);
+    const int64_t G = tiles_of(S);
+    const int64_t Gs = G < kMaxSyncTiles ? G : kMaxSyncTiles;
+    return 256 + align256((size_t)G * ((size_t)E + 1) * 8) +
+           align256((size_t)Gs * ((size_t)E + 1) * 4);
 }
 
 namespace {
 
-// One cooperative launch of prep_onepass_kernel when every tile fits on the
+// Tile shape of the one-launch path: nr rounds of kSyncThreads slots per
+// block (at least kSyncMinRounds, more when the blocks would not all be
+// resident), G = ceil(S / (nr * kSyncThreads)) blocks.  False when the
+// problem needs more than kSyncMaxRounds rounds or kMaxSyncTiles blocks.
+bool sync_shape(int64_t S, int64_t resident, int *nr_out, int *G_out) {
+    const int64_t cap = resident < kMaxSyncTiles ? resident : kMaxSyncTiles;
+    if (cap < 1) return false;
+    int64_t nr = (S + cap * kSyncThreads - 1) / (cap * kSyncThreads);
+    if (nr < kSyncMinRounds) nr = kSyncMinRounds;
+    if (nr > kSyncMaxRounds) return false;
+    *nr_out = (int)nr;
+    *G_out = (int)((S + nr * kSyncThreads - 1) / (nr * kSyncThreads));
+    return true;
+}
+
+// One cooperative launch of prep_sync_kernel when every block fits on the
 // GPU at once; returns cudaErrorCooperativeLaunchTooLarge (nothing launched)
-// when the tiles do not fit or the launch form is refused.
+// when they do not or the launch form is refused.
 template <typename IdT>
-cudaError_t launch_onepass(const IdT *ids, int64_t base, int64_t S, int E, int A, int G,
-                           void *workspace, int32_t *counts, int32_t *offsets, int32_t *bso,
-                           int32_t *in_perm, int32_t *out_perm, int32_t *diag,
-                           cudaStream_t stream) {
-    auto kern = prep_onepass_kernel<IdT>;
-    const size_t smem = tile_smem<kOnepassThreads>(E);
-    const int64_t resident = (int64_t)sm_count() * blocks_per_sm(kern, kOnepassThreads, smem);
+cudaError_t launch_sync(const IdT *ids, int64_t base, int64_t S, int E, int A, void *workspace,
+                        int32_t *counts, int32_t *offsets, int32_t *bso, int32_t *in_perm,
+                        int32_t *out_perm, int32_t *diag, cudaStream_t stream) {
+    auto kern = prep_sync_kernel<IdT>;
+    int nr = 0, G = 0;
+    if (!sync_shape(S, (int64_t)sm_count(), &nr, &G)) return cudaErrorCooperativeLaunchTooLarge;
+    const size_t smem = tile_smem<kSyncThreads>(E, G);
+    if (smem > 200 * 1024) return cudaErrorCooperativeLaunchTooLarge;
+    const int64_t resident = (int64_t)sm_count() * blocks_per_sm(kern, kSyncThreads, smem);
     if (G > resident) return cudaErrorCooperativeLaunchTooLarge;
     cudaError_t se = ensure_smem(kern, smem);
     if (se != cudaSuccess) return se;
+    const unsigned long long wait_ns = prepare_wait_ns().load();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)G, 1, 1);
-    cfg.blockDim = dim3(kOnepassThreads, 1, 1);
+    cfg.blockDim = dim3(kSyncThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[2];
@@ -700,8 +752,8 @@ cudaError_t launch_onepass(const IdT *ids, int64_t base, int64_t S, int E, int A
     cfg.attrs = attr;
     for (int n : {2, 1}) {  // with programmatic serialization if allowed, else without
         cfg.numAttrs = n;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ids, base, S, E, A, G, workspace, counts,
-                                           offsets, bso, in_perm, out_perm, diag);
+        cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ids, base, S, E, A, G, nr, workspace,
+                                           wait_ns, counts, offsets, bso, in_perm, out_perm, diag);
         if (e == cudaSuccess) return cudaGetLastError();
         cudaGetLastError();
     }
@@ -720,12 +772,13 @@ cudaError_t run_prepare_t(const IdT *ids, int64_t base, int64_t S, int E, int A,
     if (S <= kSingleBlockSlots)
         return launch(prep_single_kernel<IdT>, 1, kSingleThreads, single_block_smem(E), stream, ids,
                       base, S, E, A, counts, offsets, bso, in_perm, out_perm, diag);
-    const int G = (int)((S + kTileSlots - 1) / kTileSlots);
-    cudaError_t e = launch_onepass(ids, base, S, E, A, G, workspace, counts, offsets, bso,
-                                   in_perm, out_perm, diag, stream);
+    cudaError_t e = launch_sync(ids, base, S, E, A, workspace, counts, offsets, bso, in_perm,
+                                out_perm, diag, stream);
     if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+    const int G = (int)tiles_of(S);
     e = launch(prep_rank_kernel<IdT>, G, kRankThreads, tile_smem<kRankThreads>(E), stream, ids,
-               base, S, E, A, G, workspace, counts, offsets, bso, out_perm, diag);
+               base, S, E, A, G, workspace, (unsigned long long)prepare_wait_ns().load(), counts,
+               offsets, bso, out_perm, diag);
     if (e != cudaSuccess) return e;
     const int64_t grid = persistent_grid(prep_finish_kernel<IdT>, 256, 0, (S + 1023) / 1024);
     return launch(prep_finish_kernel<IdT>, grid, 256, 0, stream, ids, base, S, E,

@@ -124,7 +124,14 @@ size_t moe_prepare_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t nu
  *                                      outside [0, E); diag[1] = 1 if a
  *                                      bounded inter-block wait gave up (the
  *                                      other outputs are then invalid), else
- *                                      0.
+ *                                      0.  A wait gives up after about one
+ *                                      second (moe_set_wait_limits); the
+ *                                      kernel still ends and the call's
+ *                                      stream stays usable.  A workspace
+ *                                      whose counters were disturbed (not
+ *                                      zeroed before first use, or written
+ *                                      by anything but the library) shows
+ *                                      up here: zero it and call again.
  *   workspace                          scratch of moe_prepare_workspace_bytes()
  *                                      bytes, 256-byte aligned, zeroed before
  *                                      its first use and then left to the
@@ -133,7 +140,9 @@ size_t moe_prepare_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t nu
  *
  * Batches of up to 4096 slots run in one block; larger ones as tiles over
  * the whole GPU (the only case that touches the workspace): one cooperative
- * launch when every tile fits on the GPU at once, else two kernels.
+ * launch with one grid barrier when every tile fits on the GPU at once (up
+ * to 16 rounds of 512 slots per SM: about 1.2 million slots on B200), else
+ * two kernels with a decoupled look-back between tiles.
  *
  * Dispatched order: by expert ascending, and within an expert by expanded
  * index ascending (token, then slot): a stable counting sort, so the result
@@ -171,6 +180,36 @@ moe_status_t moe_prepare(const int32_t *topk_ids, int64_t num_tokens, int32_t to
 moe_status_t moe_dispatch_rows(const void *x, moe_dtype_t dtype, int64_t num_tokens,
                                int64_t hidden, int32_t top_k, const int32_t *input_permutation,
                                const int32_t *output_permutation, void *out, moe_stream_t stream);
+
+/*
+ * Failure report of the TMA dispatch (the scatter form of moe_dispatch_rows,
+ * taken when output_permutation is given).  Each of its blocks waits,
+ * bounded, for every chunk of x it stages in shared memory; a block whose
+ * wait gave up stops, lets its copies in flight finish and sets a device
+ * error word, so the call's rows are then incomplete although the call
+ * returned MOE_OK.  This enqueues on `stream` one tiny kernel that writes
+ * that word to *error (device memory, int32: 1 if some wait gave up since
+ * the previous query on this device, else 0) and clears it.  Order it after
+ * the dispatches it should cover.  No counterpart in the pages (they give
+ * no failure reporting); it is this library's bounded-wait contract.
+ * Errors: MOE_ERR_INVALID_ARG for a NULL `error`.
+ */
+moe_status_t moe_dispatch_error(int32_t *error, moe_stream_t stream);
+
+/*
+ * Limits of the bounded waits, for tests of the failure reporting:
+ *   prepare_wait_us   how long a prepare block waits for other blocks, in
+ *                     microseconds of the GPU's global timer (default
+ *                     1000000, one second); 0 gives up at the first check
+ *                     that finds the awaited value missing.
+ *   dispatch_polls    mbarrier polls the TMA dispatch makes for one staged
+ *                     chunk (default 2^24); 0 gives up at once.
+ * A negative value restores that default.  The limits apply, process-wide,
+ * to every launch made after the call (a CUDA graph keeps those it was
+ * captured with).  Lower them only to test the failure reporting: a wait
+ * that gives up leaves that call's outputs invalid.  Never fails.
+ */
+moe_status_t moe_set_wait_limits(int64_t prepare_wait_us, int64_t dispatch_polls);
 
 /*
  * Dispatch with FP8 E4M3 1x128 block-scale quantisation (TensorRT-LLM PR

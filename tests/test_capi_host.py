@@ -237,3 +237,10 @@ def test_valid_call_without_gpu_reports_cuda_error(lib):
         pytest.skip("a GPU is present")
     st = lib.moe_combine(P, BF16, 4, 64, 2, P, P, P, BF16, None)
     assert st == CUDA
+
+
+def test_dispatch_error_and_wait_limits_validation(lib):
+    # the error query needs somewhere to write; the limits call never fails
+    assert lib.moe_dispatch_error(None, None) == INVALID
+    assert lib.moe_set_wait_limits(0, 0) == OK
+    assert lib.moe_set_wait_limits(-1, -1) == OK  # back to the defaults
