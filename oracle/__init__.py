@@ -21,6 +21,11 @@ step computes:
 * ``problem_sizes`` and ``tile_layout``: the grouped-GEMM metadata that
   follows prepare (sglang's problem_sizes1/2; TensorRT-LLM's moe_sort
   outputs).
+* ``ep_recv_layout``: the receiving rank's side of the expert-parallel
+  exchange between GPUs (Mooncake PR #4581, dispatch / combine across
+  ranks; TensorRT-LLM PR #9592, all-to-all communication and the local
+  expert window): where each received row goes in the expert-grouped
+  layout.
 * ``prepare_local`` and ``output_memset``: one rank's expert window
   (local_expert_offset / num_local_experts) over int64 ids, and
   moe_output_memset_inplace (TensorRT-LLM PR #9592; Mooncake PR #4581 for
@@ -46,7 +51,7 @@ __all__ = [
     "F32", "F16", "BF16", "lib", "prepare", "dispatch", "dispatch_fp8",
     "combine", "brute_prepare", "problem_sizes", "tile_layout", "prepare_local",
     "output_memset", "dispatch_nvfp4", "f32_to_e2m1", "e2m1_to_f32", "f32_to_bf16", "f32_to_f16", "f16_to_f32",
-    "bf16_to_f32", "f32_to_e4m3", "e4m3_to_f32", "openmp", "threads",
+    "bf16_to_f32", "f32_to_e4m3", "e4m3_to_f32", "openmp", "threads", "ep_recv_layout",
 ]
 
 F32, F16, BF16 = 0, 1, 2
@@ -115,6 +120,8 @@ def _load(openmp_build: bool):
         L.oracle_dispatch_nvfp4.argtypes = [_vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
                                             ctypes.c_int32, _vp, _vp, _vp, _vp, ctypes.c_int64,
                                             _vp, _vp]
+        L.oracle_ep_recv_layout.restype = ctypes.c_int64
+        L.oracle_ep_recv_layout.argtypes = [_vp, ctypes.c_int32, ctypes.c_int32] + [_vp] * 4
         L.oracle_e2m1_to_f32.restype = ctypes.c_float
         L.oracle_e2m1_to_f32.argtypes = [ctypes.c_uint8]
         L.oracle_problem_sizes.restype = None
@@ -351,3 +358,22 @@ def f16_to_f32(a):
 
 def e4m3_to_f32(a):
     return _conv("oracle_e4m3_to_f32_n", a, np.uint8, np.float32)
+
+
+def ep_recv_layout(counts: np.ndarray):
+    """Receive layout of one rank in the expert-parallel exchange.
+
+    ``counts`` [R, El] int32: rows source rank s sends for local expert le.
+    Returns recv_offsets [R+1], local_offsets [El+1], recv_to_local [N] and
+    local_to_recv [N] (int32), N = counts.sum().
+    """
+    c = np.ascontiguousarray(counts, dtype=np.int32)
+    R, El = c.shape
+    n = int(c.astype(np.int64).sum())
+    ro = np.zeros(R + 1, np.int32)
+    lo = np.zeros(El + 1, np.int32)
+    r2l = np.zeros(n, np.int32)
+    l2r = np.zeros(n, np.int32)
+    got = lib().oracle_ep_recv_layout(_ptr(c), R, El, _ptr(ro), _ptr(lo), _ptr(r2l), _ptr(l2r))
+    assert got == n
+    return dict(recv_offsets=ro, local_offsets=lo, recv_to_local=r2l, local_to_recv=l2r)

@@ -656,3 +656,63 @@ void oracle_dispatch_nvfp4(const uint16_t *x, int x_dtype, int64_t T, int64_t H,
         }
     }
 }
+
+/* ------------------------------------------------------------------ */
+/* Expert-parallel exchange: the receiving rank's layout.              */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Mooncake PR #4581 (expert-parallel dispatch / combine between GPUs) and
+ * TensorRT-LLM PR #9592 (all-to-all communication; one rank's experts are
+ * the window local_expert_offset .. + num_local_experts).  R ranks each own
+ * El consecutive experts.  A source rank's dispatched rows are sorted by
+ * expert, so the rows it sends to this rank form one block ordered by local
+ * expert.  c[s*El + le] is the number of rows source s sends for local
+ * expert le.
+ *
+ *   received buffer: the source blocks in source order,
+ *     recv_offsets[s] = sum over s' < s and all le of c[s'][le]   ([R+1])
+ *   grouped layout: by local expert, then source, then the source's order,
+ *     local_offsets[le] = sum over le' < le and all s of c[s][le'] ([El+1])
+ *   received row q = recv_offsets[s] + sum_{le' < le} c[s][le'] + m
+ *     and grouped row g = local_offsets[le] + sum_{s' < s} c[s'][le] + m
+ *     are the same row (0 <= m < c[s][le]):
+ *     recv_to_local[q] = g, local_to_recv[g] = q.
+ * Returns the number of received rows.
+ */
+int64_t oracle_ep_recv_layout(const int32_t *c, int32_t R, int32_t El, int32_t *recv_offsets,
+                              int32_t *local_offsets, int32_t *recv_to_local,
+                              int32_t *local_to_recv)
+{
+    int64_t acc = 0;
+    for (int32_t s = 0; s < R; ++s) {
+        recv_offsets[s] = (int32_t)acc;
+        for (int32_t le = 0; le < El; ++le)
+            acc += c[(int64_t)s * El + le];
+    }
+    recv_offsets[R] = (int32_t)acc;
+    int64_t n = acc;
+    acc = 0;
+    for (int32_t le = 0; le < El; ++le) {
+        local_offsets[le] = (int32_t)acc;
+        for (int32_t s = 0; s < R; ++s)
+            acc += c[(int64_t)s * El + le];
+    }
+    local_offsets[El] = (int32_t)acc;
+    /* walk the grouped layout in its own order and find each row's place in
+       the received buffer */
+    int64_t g = 0;
+    for (int32_t le = 0; le < El; ++le) {
+        for (int32_t s = 0; s < R; ++s) {
+            int64_t q = recv_offsets[s];
+            for (int32_t l2 = 0; l2 < le; ++l2)
+                q += c[(int64_t)s * El + l2];
+            for (int32_t m = 0; m < c[(int64_t)s * El + le]; ++m) {
+                recv_to_local[q + m] = (int32_t)g;
+                local_to_recv[g] = (int32_t)(q + m);
+                ++g;
+            }
+        }
+    }
+    return n;
+}

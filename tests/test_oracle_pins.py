@@ -544,3 +544,70 @@ def test_dispatch_nvfp4_decode_bound_and_layout():
     rows0 = np.nonzero(m["input_perm"] // k == 0)[0]
     assert len(rows0) == k
     assert (sc[srow[rows0], 0] == 0).all() and (q[rows0, :8] == 0).all()
+
+
+# ---------------------------------------------------------------------------
+# Expert-parallel exchange: the receiving rank's layout
+# ---------------------------------------------------------------------------
+
+def test_ep_recv_layout_hand_worked():
+    # 2 source ranks, 3 local experts.  Source 0 sends 2 rows of expert 0 and
+    # 1 of expert 2 (received rows 0, 1 | 2); source 1 sends 1 row of expert
+    # 0 and 3 of expert 1 (received rows 3 | 4, 5, 6).  Grouped by expert,
+    # then source: expert 0 = rows 0, 1 (source 0), 3 (source 1); expert 1 =
+    # rows 4, 5, 6; expert 2 = row 2.
+    lay = oracle.ep_recv_layout(np.array([[2, 0, 1], [1, 3, 0]], np.int32))
+    assert lay["recv_offsets"].tolist() == [0, 3, 7]
+    assert lay["local_offsets"].tolist() == [0, 3, 6, 7]
+    assert lay["local_to_recv"].tolist() == [0, 1, 3, 4, 5, 6, 2]
+    assert lay["recv_to_local"].tolist() == [0, 1, 6, 2, 3, 4, 5]
+
+
+@pytest.mark.parametrize("R,El,seed", [(1, 5, 0), (2, 3, 1), (4, 8, 2), (8, 1, 3), (3, 7, 4)])
+def test_ep_recv_layout_invariants(R, El, seed):
+    rng = np.random.default_rng(seed)
+    c = rng.integers(0, 6, size=(R, El)).astype(np.int32)
+    c[rng.random((R, El)) < 0.3] = 0
+    lay = oracle.ep_recv_layout(c)
+    n = int(c.sum())
+    r2l, l2r = lay["recv_to_local"], lay["local_to_recv"]
+    assert sorted(r2l.tolist()) == list(range(n)) and (r2l[l2r] == np.arange(n)).all()
+    # every received row lands inside its local expert's grouped range, and
+    # each (source, expert) run stays in order
+    q = 0
+    for s in range(R):
+        for le in range(El):
+            g = r2l[q:q + c[s, le]]
+            assert (g >= lay["local_offsets"][le]).all() and (g < lay["local_offsets"][le + 1]).all()
+            assert (np.diff(g) == 1).all()
+            q += c[s, le]
+
+
+@pytest.mark.parametrize("R,El,k,seed", [(2, 4, 2, 0), (4, 3, 3, 1), (3, 5, 1, 2)])
+def test_ep_exchange_reproduces_the_global_prepare(R, El, k, seed):
+    """Exchange + regroup on every rank equals one prepare over all ranks'
+    tokens taken together (in rank order), restricted to the rank's expert
+    window: the stable order expert, then global slot, is the order
+    expert, then source rank, then the source's own slot order."""
+    rng = np.random.default_rng(seed)
+    E = R * El
+    T = [int(rng.integers(0, 9)) for _ in range(R)]
+    ids = [np.stack([rng.permutation(E)[:k] for _ in range(t)]).astype(np.int32)
+           if t else np.zeros((0, k), np.int32) for t in T]
+    for r in range(R):                       # a few invalid ids
+        if T[r]:
+            ids[r][0, 0] = -1
+    metas = [oracle.prepare(i, E) for i in ids]
+    g = oracle.prepare(np.concatenate(ids), E)
+    tok0 = np.concatenate([[0], np.cumsum(T)])
+    for dst in range(R):
+        lo, hi = dst * El, (dst + 1) * El
+        c = np.stack([m["counts"][lo:hi] for m in metas])
+        lay = oracle.ep_recv_layout(c)
+        # global slot index of every received row, source blocks in order
+        recv = np.concatenate([tok0[s] * k + metas[s]["input_perm"][metas[s]["offsets"][lo]:
+                                                                     metas[s]["offsets"][hi]]
+                               for s in range(R)])
+        assert np.array_equal(recv[lay["local_to_recv"]],
+                              g["input_perm"][g["offsets"][lo]:g["offsets"][hi]])
+        assert np.array_equal(lay["local_offsets"], g["offsets"][lo:hi + 1] - g["offsets"][lo])
