@@ -538,6 +538,17 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
         print(f"cuda graph timing unavailable: {exc}", file=sys.stderr)
         graph_ms = None
 
+    # ---- timed region 3: the per-call breakdown inside the graph.  The same
+    #      n steps captured in a second graph with timing events recorded
+    #      between the calls (event nodes of the graph, on the kernels'
+    #      stream); replayed K / n times, so every call is timed K times
+    #      without the host launch gaps of the eager region.
+    per_graph = None
+    try:
+        per_graph = time_calls_in_graph(step, dev, K, n_graph)
+    except Exception as exc:
+        print(f"in-graph call timing unavailable: {exc}", file=sys.stderr)
+
     counts = step.meta_bufs["expert_counts"].cpu().numpy()
     diag = step.meta_bufs["diag"].cpu().numpy().tolist()
 
@@ -557,8 +568,16 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
     if fused:  # prepare and dispatch are one launch, timed together
         alg = {"prepare_dispatch": alg["prepare"] + alg["dispatch"], "combine": alg["combine"]}
         per = {"prepare_dispatch": per["prepare"], "combine": per["combine"], "step": per["step"]}
+        if per_graph is not None:
+            per_graph = {"prepare_dispatch": per_graph["prepare"],
+                         "combine": per_graph["combine"], "step": per_graph["step"]}
     calls = [c for c in ("prepare", "dispatch", "prepare_dispatch", "combine") if c in alg]
-    kern = {c: statistics.mean(per[c]) for c in calls}
+    # the breakdown and the roofline use the in-graph times (the calls as the
+    # headline's graph runs them); the eager ones add each launch's host and
+    # event gap (several microseconds a call) and are kept beside them
+    timed = per_graph if per_graph is not None else per
+    kern = {c: statistics.mean(timed[c]) for c in calls}
+    eager_kern = {c: statistics.mean(per[c]) for c in calls}
     dominant = max((c for c in calls if c != "prepare"), key=lambda c: kern[c])
     kernel_key = f"{dominant}@{w.name}"
     achieved = alg[dominant] / (kern[dominant] * 1e-3) / 1e9
@@ -566,13 +585,17 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
     breakdown = {}
     for k in calls:
         gbs = alg[k] / (kern[k] * 1e-3) / 1e9
-        breakdown[k] = {"us_mean": kern[k] * 1e3, "latency_ms": percentiles(per[k]),
+        breakdown[k] = {"us_mean": kern[k] * 1e3, "latency_ms": percentiles(timed[k]),
+                        "timed": "in graph" if per_graph is not None else "eager",
                         "tokens_per_s": w.T / (kern[k] * 1e-3), "algorithmic_bytes": alg[k],
                         "effective_gbs": gbs, "frac_of_measured_peak": gbs / peak,
-                        "frac_of_8tbs_spec": gbs / SPEC_HBM_GBS}
+                        "frac_of_8tbs_spec": gbs / SPEC_HBM_GBS,
+                        "eager_us_mean": eager_kern[k] * 1e3,
+                        "eager_latency_ms": percentiles(per[k])}
     step_alg = sum(alg.values())
     breakdown["end_to_end"] = {
-        "latency_ms": percentiles(per["step"]),
+        "latency_ms": percentiles(timed["step"]),
+        "eager_latency_ms": percentiles(per["step"]),
         "eager_ms_per_step": eager_ms / K,
         "graph_ms_per_step": None if graph_ms is None else graph_ms / K,
         "effective_gbs": step_alg / (elapsed_ms / K * 1e-3) / 1e9,
@@ -639,6 +662,46 @@ def run_gpu(args, names):
                     dtype=_dtype_tag(CONFIGS[n]))
             for n in names[1:]}
     print(json.dumps(line), flush=True)
+
+
+def time_calls_in_graph(step, dev, K, n_graph):
+    """Per-call durations (ms) of n_graph consecutive steps captured as one
+    CUDA graph with timing events recorded between the calls, the graph
+    replayed K / n_graph times: K samples per call."""
+    import torch
+    ev = lambda: torch.cuda.Event(enable_timing=True, external=True)  # noqa: E731
+    marks = [[ev() for _ in range(4)] for _ in range(n_graph)]
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            for m in marks:
+                m[0].record(side)
+                if step.fused:
+                    meta = step.prepare_dispatch()
+                    m[1].record(side)
+                else:
+                    meta = step.prepare()
+                    m[1].record(side)
+                    step.dispatch(meta)
+                m[2].record(side)
+                step.combine(meta)
+                m[3].record(side)
+    torch.cuda.synchronize(dev)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    per = {"prepare": [], "dispatch": [], "combine": [], "step": []}
+    for _ in range(K // n_graph):
+        g.replay()
+        torch.cuda.synchronize(dev)
+        for m in marks:
+            per["prepare"].append(m[0].elapsed_time(m[1]))
+            per["dispatch"].append(m[1].elapsed_time(m[2]))
+            per["combine"].append(m[2].elapsed_time(m[3]))
+            per["step"].append(m[0].elapsed_time(m[3]))
+    del g
+    return per
 
 
 def time_next_rows(step, w, dev, reps=20):

@@ -38,6 +38,8 @@ __all__ = [
     "moe_tile_layout",
     "moe_prepare_local",
     "moe_output_memset",
+    "moe_ep_recv_layout",
+    "EpRecvLayout",
     "TileLayout",
     "library_path",
 ]
@@ -57,6 +59,14 @@ class TileLayout(NamedTuple):
     permuted_idx_to_expanded_idx: torch.Tensor  # [max_tiles * tile_size]
     num_non_exiting_tiles: torch.Tensor         # [1] (-1: max_tiles too small)
     total_num_padded_tokens: torch.Tensor       # [1]
+
+
+class EpRecvLayout(NamedTuple):
+    recv_offsets: torch.Tensor    # [R+1] int32
+    local_offsets: torch.Tensor   # [El+1] int32
+    recv_to_local: torch.Tensor   # [N] int32
+    local_to_recv: torch.Tensor   # [N] int32
+    num_recv: torch.Tensor        # [1] int32
 
 
 class PrepareResult(NamedTuple):
@@ -448,3 +458,26 @@ def moe_output_memset(out: torch.Tensor, output_permutation: torch.Tensor, top_k
                                            output_permutation.data_ptr(), _stream(out.device))
     _lib.check("moe_output_memset", st)
     return out
+
+
+def moe_ep_recv_layout(recv_expert_counts: torch.Tensor, num_recv: int) -> EpRecvLayout:
+    """Receiving rank's layout of the expert-parallel exchange (see
+    include/moe.h).  ``recv_expert_counts`` [R, El] int32 on the GPU;
+    ``num_recv`` = its sum (the caller knows it from the count exchange),
+    which sizes the two row maps."""
+    _need(recv_expert_counts, "recv_expert_counts", torch.int32)
+    if recv_expert_counts.dim() != 2:
+        raise ValueError("recv_expert_counts must be [num_ranks, num_local_experts]")
+    R, El = recv_expert_counts.shape
+    dev = recv_expert_counts.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    lay = EpRecvLayout(torch.empty(R + 1, **i32), torch.empty(El + 1, **i32),
+                       torch.empty(num_recv, **i32), torch.empty(num_recv, **i32),
+                       torch.empty(1, **i32))
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_ep_recv_layout(
+            recv_expert_counts.data_ptr(), R, El, num_recv, lay.recv_offsets.data_ptr(),
+            lay.local_offsets.data_ptr(), _ptr(lay.recv_to_local) if num_recv else None,
+            _ptr(lay.local_to_recv) if num_recv else None, lay.num_recv.data_ptr(), _stream(dev))
+    _lib.check("moe_ep_recv_layout", st)
+    return lay

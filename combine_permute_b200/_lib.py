@@ -20,6 +20,7 @@ MOE_F32, MOE_F16, MOE_BF16, MOE_FP8_E4M3 = 0, 1, 2, 3
 MOE_I32, MOE_I64 = 0, 1
 MAX_EXPERTS = 1024
 FUSED_MAX_SLOTS = 4096
+EP_MAX_GROUPS = 8192
 
 # every symbol include/moe.h declares
 EXPORTED = (
@@ -40,6 +41,7 @@ EXPORTED = (
     "moe_tile_layout",
     "moe_prepare_local",
     "moe_output_memset",
+    "moe_ep_recv_layout",
 )
 
 _vp = ctypes.c_void_p
@@ -72,6 +74,7 @@ _SIGNATURES = {
     "moe_prepare_local": (_int, [_vp, _int, _i64, _i32, _i64, _i32, _vp, _vp, _vp, _i32, _vp,
                                  _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "moe_output_memset": (_int, [_vp, _int, _i64, _i64, _i32, _vp, _vp]),
+    "moe_ep_recv_layout": (_int, [_vp, _i32, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
 
 _lib = None

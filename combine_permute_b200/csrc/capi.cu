@@ -286,4 +286,19 @@ moe_status_t moe_tile_layout(int64_t num_tokens, int32_t top_k, int32_t num_expe
         (cudaStream_t)stream));
 }
 
+moe_status_t moe_ep_recv_layout(const int32_t *recv_expert_counts, int32_t num_ranks,
+                                int32_t num_local_experts, int64_t capacity,
+                                int32_t *recv_offsets, int32_t *local_offsets,
+                                int32_t *recv_to_local, int32_t *local_to_recv,
+                                int32_t *num_recv, moe_stream_t stream) {
+    if (num_ranks < 1 || num_local_experts < 1 || capacity < 0) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)num_ranks * num_local_experts > moe::kMaxEpGroups) return MOE_ERR_UNSUPPORTED;
+    if (!recv_expert_counts || !recv_offsets || !local_offsets || !num_recv)
+        return MOE_ERR_INVALID_ARG;
+    if (capacity > 0 && (!recv_to_local || !local_to_recv)) return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_ep_recv_layout(recv_expert_counts, num_ranks, num_local_experts,
+                                             capacity, recv_offsets, local_offsets, recv_to_local,
+                                             local_to_recv, num_recv, (cudaStream_t)stream));
+}
+
 }  // extern "C"

@@ -19,6 +19,7 @@ constexpr int kSingleBlockSlots = 4096;
 constexpr int kTileSlots = 2048;  // slots per tile
 constexpr int kMaxExperts = 1024;
 constexpr int kFusedMaxSlots = 4096;
+constexpr int kMaxEpGroups = 8192;  // ranks x local experts of one exchange layout
 
 size_t prepare_workspace_bytes(int64_t S, int E);
 
@@ -73,5 +74,13 @@ cudaError_t run_tile_layout(int64_t S, int E, int tile, const int32_t *counts,
                             int32_t *padded_offsets, int32_t *tile_group, int32_t *tile_limit,
                             int32_t *exp2perm, int32_t *perm2exp, int32_t *num_tiles,
                             int32_t *total_padded, cudaStream_t stream);
+
+// Receiving rank's layout of the expert-parallel exchange: counts [R][El]
+// -> recv_offsets [R+1], local_offsets [El+1], the two row maps (written when
+// the number of received rows is at most `capacity`) and that number.
+cudaError_t run_ep_recv_layout(const int32_t *counts, int R, int El, int64_t capacity,
+                               int32_t *recv_offsets, int32_t *local_offsets,
+                               int32_t *recv_to_local, int32_t *local_to_recv,
+                               int32_t *num_recv, cudaStream_t stream);
 
 }  // namespace moe

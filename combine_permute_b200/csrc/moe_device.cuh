@@ -66,6 +66,34 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned *p) {
     return v;
 }
 
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Atomic add with acquire-release semantics at GPU scope; returns the old value.
+__device__ __forceinline__ unsigned long long atom_add_acq_rel_u64(unsigned long long *p,
+                                                                  unsigned long long v) {
+    unsigned long long old;
+    asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v)
+                 : "memory");
+    return old;
+}
+
+// Atomic add with release semantics at GPU scope, no result.
+__device__ __forceinline__ void red_add_release_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Wrapping increment (atomicInc semantics) with acquire-release semantics.
+__device__ __forceinline__ unsigned atom_inc_acq_rel_u32(unsigned *p, unsigned limit) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.inc.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(limit)
+                 : "memory");
+    return old;
+}
+
 // Nanoseconds of the GPU's global timer: the clock behind every bounded wait.
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
     unsigned long long t;

@@ -147,43 +147,46 @@ __device__ __forceinline__ int offsets_from_totals(int *tot, int *pad, int E, in
 
 __host__ __device__ inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
 
-// Workspace of the tiled paths: a 256-byte header, then one 64-bit
-// look-back word per (tile, expert column) of the two-kernel path, then one
-// int32 histogram row per block of the one-launch path.  A look-back word
-// holds epoch << 34 | flag << 32 | value; it counts as published by this
-// call only when its epoch field is this call's epoch, so words left by
-// earlier calls need no clearing.  The epoch advances once per call (by the
-// call's last block); the ticket, done and barrier counters return to zero
-// at the end of every call.  The histogram rows are written before the grid
-// barrier and read after it, so they need no clearing either.
+// Workspace of the tiled paths, in three fixed parts: a 256-byte header
+// (counters), the one-launch path's histogram rows (a fixed kSyncHistBytes,
+// int32 rows of E+1 counts, one per block), then one 64-bit look-back word
+// per (tile, expert column) of the two-kernel path.  The parts never move
+// with the problem size, so no call reads another path's data as its own.
+// A look-back word holds epoch << 34 | flag << 32 | value; it counts as
+// published by this call only when its epoch field is this call's epoch, so
+// words left by earlier calls need no clearing.  The epoch advances once per
+// two-kernel call (by its last block); the ticket, done and barrier-arrival
+// counters return to zero at the end of every call.  The histogram rows are
+// written before the grid barrier and read after it, so they need no
+// clearing either.
 struct PrepWs {
     unsigned *ticket;     // tile tickets, wraps at G
     unsigned *done;       // blocks finished, wraps at G
     unsigned *epoch;      // this call's epoch
     unsigned *timeout;    // set when a bounded wait gave up
-    unsigned *bar_count;  // one-launch path: blocks arrived at the grid barrier
-    unsigned *bar_gen;    // one-launch path: barrier generation
-    unsigned long long *state;  // [G][E+1] look-back words
-    int *hist;                  // [G'][E+1] histogram rows, G' <= kMaxSyncTiles
+    unsigned long long *bar;    // one-launch path: generation << 32 | blocks arrived
+    int *hist;                  // [G][E+1] histogram rows of the one-launch path
+    unsigned long long *state;  // [G][E+1] look-back words of the two-kernel path
 };
 
 // Most blocks of one one-launch prepare (one block per SM on B200, with room
-// for parts with more SMs); it bounds the histogram rows of the workspace.
+// for parts with more SMs) and, with at most kSyncThreads columns a row, the
+// fixed size of its histogram rows.
 constexpr int kMaxSyncTiles = 256;
+constexpr size_t kSyncHistBytes = (size_t)kMaxSyncTiles * 512 * sizeof(int);
 
 __host__ __device__ inline int64_t tiles_of(int64_t S) { return (S + kTileSlots - 1) / kTileSlots; }
 
-__host__ __device__ inline PrepWs carve(void *ws, int64_t S, int E) {
+__host__ __device__ inline PrepWs carve(void *ws) {
     char *b = (char *)ws;
     PrepWs w;
     w.ticket = (unsigned *)b;
     w.done = (unsigned *)(b + 4);
     w.epoch = (unsigned *)(b + 8);
     w.timeout = (unsigned *)(b + 16);
-    w.bar_count = (unsigned *)(b + 20);
-    w.bar_gen = (unsigned *)(b + 24);
-    w.state = (unsigned long long *)(b + 256);
-    w.hist = (int *)(b + 256 + align256((size_t)tiles_of(S) * ((size_t)E + 1) * 8));
+    w.bar = (unsigned long long *)(b + 24);
+    w.hist = (int *)(b + 256);
+    w.state = (unsigned long long *)(b + 256 + kSyncHistBytes);
     return w;
 }
 
@@ -492,23 +495,34 @@ __device__ __forceinline__ void tile_finish(const PrepWs &ws, int G, unsigned ep
 constexpr int kRankThreads = 256;                  // two-kernel tiles: 8 warps
 constexpr int kRankRounds = kTileSlots / kRankThreads;  // of 8 rounds
 constexpr int kSyncThreads = 512;                  // one-launch tiles: 16 warps
+static_assert(kSyncThreads <= 512, "a histogram row of the one-launch path fits kSyncHistBytes");
 constexpr int kSyncMaxRounds = 16;                 // of up to 16 rounds (8192 slots)
 constexpr int kSyncMinRounds = 4;
 
-// Shared memory of the tiled kernels: per-warp rows, then hist, excl, off,
-// pad (one column per expert plus one for invalid ids each); the one-launch
-// kernel adds the G histogram rows it stages.
-template <int NT> size_t tile_smem(int E, int G = 0) {
-    return (size_t)(NT / 32 + 4 + G) * (E + 1) * sizeof(int);
-}
+// Shared memory of the two-kernel tiles: per-warp rows, then hist, excl,
+// off, pad (one column per expert plus one for invalid ids each).
+template <int NT> size_t tile_smem(int E) { return (size_t)(NT / 32 + 4) * (E + 1) * sizeof(int); }
 
 // One-launch prepare (a cooperative launch: every block resident, so blocks
-// may wait on one another).  Block b ranks slots [b*nr*NT, (b+1)*nr*NT),
-// publishes its histogram row and arrives at a grid barrier (bounded wait).
-// After it, every block stages all G rows in shared memory, sums them into
-// the totals and its own exclusive prefix over earlier blocks, scans the
-// totals into the expert offsets (block 0 writes counts, offsets and
-// block-scale offsets) and writes its slots' rows into both permutations.
+// may wait on one another; E + 1 <= kSyncThreads).  Block b ranks slots
+// [b*nr*NT, (b+1)*nr*NT) within each warp's run, folds the warps into its
+// histogram row, publishes the row and arrives at a grid barrier (one 64-bit
+// word, generation << 32 | arrivals: the last arrival resets the count and
+// advances the generation in one atomic; the others wait for the generation
+// to move, bounded).  Then every block stages all G rows in shared memory;
+// thread c sums column c into the total and this block's prefix over earlier
+// blocks, and three exclusive scans over the experts run in registers: the
+// expert offsets, the block-scale offsets (block 0 writes both and the
+// counts) and this block's own offsets.  Every slot's row goes to
+// output_permutation; the block's slots are also staged in shared memory in
+// dispatched order, so that input_permutation is written in runs of
+// consecutive rows rather than one scattered word per slot.  Blocks count
+// themselves out on a second word whose high half counts the waits that gave
+// up; the last one reports them in diag[1].
+template <int NT> size_t sync_smem(int E, int G, int nr) {
+    return ((size_t)(NT / 32 + 4 + G) * (E + 1) + 2 * (size_t)nr * NT) * sizeof(int);
+}
+
 template <typename IdT>
 __global__ void __launch_bounds__(kSyncThreads, 1)
     prep_sync_kernel(const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int A, int G,
@@ -517,77 +531,194 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
                      int32_t *diag) {
     constexpr int NT = kSyncThreads, NW = NT / 32, NR = kSyncMaxRounds;
     extern __shared__ int smem[];
-    __shared__ int warp_tmp[66];
-    __shared__ unsigned s_epoch;
+    __shared__ int s_wsum[3][NW];
     __shared__ int s_invalid;
     const int C = E + 1;
-    int *wcnt = smem;           // [NW][C]
-    int *hist = wcnt + NW * C;  // [C] this tile's counts
-    int *excl = hist + C;       // [C] earlier tiles' counts
-    int *tot = excl + C;        // [C] totals, then expert offsets
-    int *pad = tot + C;         // [C] scan scratch
-    int *rows = pad + C;        // [G][C] every tile's counts
-    const int tid = threadIdx.x;
+    int *wcnt = smem;            // [NW][C] per-warp counts, then exclusive prefixes
+    int *excl = wcnt + NW * C;   // [C] earlier blocks' counts
+    int *off = excl + C;         // [C] expert offsets
+    int *lofs = off + C;         // [C] this block's offsets of its own slots
+    int *rows = wcnt + (NW + 4) * C;  // [G][C] every block's counts (16-byte aligned)
+    int *s_slot = rows + G * C;       // [nr*NT] this block's slots in dispatched order
+    int *s_row = s_slot + nr * NT;    // [nr*NT] and their rows
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x;
     const int64_t first = (int64_t)tile * nr * NT;
-    PrepWs ws = carve(workspace, S, E);
+    const PrepWs ws = carve(workspace);
+    for (int x = tid; x < NW * C; x += NT) wcnt[x] = 0;  // shared memory only: before the wait
+    if (tid == 0) s_invalid = 0;
     pdl_wait();
     pdl_launch_dependents();
-    if (tid == 0) s_epoch = ld_relaxed_u32(ws.epoch);
+
+    // rank within each warp's run of nr * 32 consecutive slots
+    const unsigned lt = lanemask_lt();
+    const int nbits = key_bits(E);
+    const int64_t wbase = first + (int64_t)warp * 32 * nr;
     int key[NR], rank[NR];
-    rank_tile<IdT, NT, NR>(ids, base, S, E, first, nr, wcnt, hist, &s_invalid, key, rank);
-    for (int c = tid; c < C; c += NT) ws.hist[(size_t)tile * C + c] = hist[c];
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+        key[r] = r < nr ? load_key(ids, wbase + r * 32 + lane, S, base, E) : -2;
     __syncthreads();
-    if (tid == 0) {  // grid barrier: arrive, then wait for the generation to move
-        const unsigned gen = ld_relaxed_u32(ws.bar_gen);
-        __threadfence();
-        if (atomicAdd(ws.bar_count, 1u) == (unsigned)(G - 1)) {
-            atomicExch(ws.bar_count, 0u);
-            __threadfence();
-            st_release_u32(ws.bar_gen, gen + 1);
+    int *row = wcnt + warp * C;
+    int bad = 0;
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        if (r < nr) rank[r] = rank_round(key[r], E, nbits, row, lt);
+        bad += key[r] == -1;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
+    if (lane == 0 && bad) atomicAdd(&s_invalid, bad);
+    __syncthreads();
+
+    // fold the warps: column c becomes exclusive over warps; publish the row
+    if (tid < C) {
+        int run = 0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            const int v = wcnt[w * C + tid];
+            wcnt[w * C + tid] = run;
+            run += v;
+        }
+        ws.hist[(size_t)tile * C + tid] = tid < E ? run : s_invalid;
+    }
+    __syncthreads();
+    unsigned done_old = 0, gave_up = 0;
+    if (tid == 0) {
+        // grid barrier: the arrival releases this block's row (published
+        // before the block barrier above) and, for the last arrival,
+        // acquires every other row
+        const unsigned long long old = atom_add_acq_rel_u64(ws.bar, 1ull);
+        const unsigned gen = (unsigned)(old >> 32);
+        if ((unsigned)old == (unsigned)(G - 1)) {
+            red_add_release_u64(ws.bar, (1ull << 32) - (unsigned long long)G);
         } else {
             const unsigned long long t0 = globaltimer_ns();
-            while (ld_acquire_u32(ws.bar_gen) == gen) {
+            while ((unsigned)(ld_acquire_u64(ws.bar) >> 32) == gen) {
                 if (globaltimer_ns() - t0 >= wait_ns) {
-                    atomicExch(ws.timeout, 1u);
+                    gave_up = 1;
                     break;
                 }
                 __nanosleep(32);
             }
-            __threadfence();
         }
+        // count this block out; the result is needed only at the end
+        done_old = atomicAdd(ws.done, 1u + (gave_up << 16));
     }
     __syncthreads();
-    // stage the G rows (L2 only: they were written by other SMs), then sum
+
+    // stage the G rows (L2 only: other SMs wrote them), then per column the
+    // total, the prefix over earlier blocks and this block's own count
     const int n = G * C;
-    const int *src = ws.hist;
     if ((n & 3) == 0) {
-        const int4 *s4 = reinterpret_cast<const int4 *>(src);
+        const int4 *s4 = reinterpret_cast<const int4 *>(ws.hist);
         int4 *d4 = reinterpret_cast<int4 *>(rows);
         for (int x = tid; x < (n >> 2); x += NT) d4[x] = __ldcg(s4 + x);
     } else {
-        for (int x = tid; x < n; x += NT) rows[x] = __ldcg(src + x);
+        for (int x = tid; x < n; x += NT) rows[x] = __ldcg(ws.hist + x);
     }
     __syncthreads();
-    for (int c = tid; c < C; c += NT) {
-        int before = 0, all = 0;
+    int before = 0, all = 0, mine = 0;
+    if (tid < C) {
         for (int t = 0; t < G; ++t) {
-            const int v = rows[t * C + c];
+            const int v = rows[t * C + tid];
             before += t < tile ? v : 0;
             all += v;
         }
-        excl[c] = before;
-        tot[c] = all;
+        mine = rows[tile * C + tid];
+    }
+    // three exclusive scans over the experts: counts, counts rounded up to
+    // A, this block's counts (warp shuffles, then the warp sums)
+    const int cnt = tid < E ? all : 0;
+    const int padded = (cnt + A - 1) / A * A;
+    const int own = tid < E ? mine : 0;
+    int ia = cnt, ip = padded, io = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int ua = __shfl_up_sync(0xffffffffu, ia, o);
+        const int up = __shfl_up_sync(0xffffffffu, ip, o);
+        const int uo = __shfl_up_sync(0xffffffffu, io, o);
+        if (lane >= o) {
+            ia += ua;
+            ip += up;
+            io += uo;
+        }
+    }
+    if (lane == 31) {
+        s_wsum[0][warp] = ia;
+        s_wsum[1][warp] = ip;
+        s_wsum[2][warp] = io;
     }
     __syncthreads();
-    if (tile == 0 && tid == 0 && diag) diag[0] = tot[E];
-    const int total = offsets_from_totals(tot, pad, E, A, tile == 0, counts, offsets, bso, warp_tmp);
-    write_tile_rows<NT, NR>(S, E, first, nr, tot, excl, wcnt, key, rank, in_perm, out_perm);
+    int ba = 0, bp = 0, bo = 0, total = 0, pad_total = 0, own_total = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+        const int xa = s_wsum[0][w], xp = s_wsum[1][w], xo = s_wsum[2][w];
+        if (w < warp) {
+            ba += xa;
+            bp += xp;
+            bo += xo;
+        }
+        total += xa;
+        pad_total += xp;
+        own_total += xo;
+    }
+    const int ex_off = ba + ia - cnt;
+    if (tid < C) {
+        excl[tid] = before;
+        off[tid] = ex_off;
+        lofs[tid] = bo + io - own;
+    }
+    if (tile == 0) {
+        if (tid < E) {
+            counts[tid] = cnt;
+            offsets[tid] = ex_off;
+            if (bso) bso[tid] = bp + ip - padded;
+        }
+        if (tid == 0) {
+            offsets[E] = total;
+            if (bso) bso[E] = pad_total;
+        }
+        if (tid == E && diag) diag[0] = all;  // column E counts the invalid ids
+    }
+    __syncthreads();
+
+    // rows: slot i of expert e is this block's lr-th slot of e, lr = earlier
+    // warps + its rank in the warp's run; output_permutation directly,
+    // input_permutation through the staged dispatched order
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+        const int64_t i = wbase + r * 32 + lane;
+        if (r < nr && i < S) {
+            const int e = key[r];
+            int p = -1;
+            if (e >= 0) {
+                const int lr = row[e] + rank[r];
+                p = off[e] + excl[e] + lr;
+                const int lp = lofs[e] + lr;
+                if (lp >= 0 && lp < nr * NT) {
+                    s_slot[lp] = (int)i;
+                    s_row[lp] = p;
+                }
+            }
+            out_perm[i] = p;
+        }
+    }
+    __syncthreads();
+    const int nown = own_total < nr * NT ? own_total : nr * NT;
+    for (int lp = tid; lp < nown; lp += NT) {
+        const int p = s_row[lp];
+        if (p >= 0 && p < S) in_perm[p] = s_slot[lp];
+    }
     const int64_t lo = first > total ? first : (int64_t)total;
     const int64_t end = first + (int64_t)nr * NT;
     const int64_t hi = end < S ? end : S;
     for (int64_t p = lo + tid; p < hi; p += NT) in_perm[p] = -1;
-    tile_finish(ws, G, s_epoch, diag);
+    if (tid == 0 && (done_old & 0xffffu) == (unsigned)(G - 1)) {
+        const unsigned to = (done_old >> 16) + gave_up;
+        atomicExch(ws.done, 0u);
+        if (diag) diag[1] = to ? 1 : 0;
+    }
 }
 
 // Two-kernel variant, kernel 1 (any number of tiles): store rank(i) in
@@ -610,7 +741,7 @@ __global__ void __launch_bounds__(kRankThreads, 2)
     int *excl = hist + C;
     int *off = excl + C;
     int *pad = off + C;
-    PrepWs ws = carve(workspace, S, E);
+    PrepWs ws = carve(workspace);
     pdl_wait();
     pdl_launch_dependents();
     if (threadIdx.x == 0) {
@@ -699,10 +830,7 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
 
 size_t prepare_workspace_bytes(int64_t S, int E) {
     if (S <= kSingleBlockSlots) return 0;
-    const int64_t G = tiles_of(S);
-    const int64_t Gs = G < kMaxSyncTiles ? G : kMaxSyncTiles;
-    return 256 + align256((size_t)G * ((size_t)E + 1) * 8) +
-           align256((size_t)Gs * ((size_t)E + 1) * 4);
+    return 256 + kSyncHistBytes + align256((size_t)tiles_of(S) * ((size_t)E + 1) * 8);
 }
 
 namespace {
@@ -710,8 +838,10 @@ namespace {
 // Tile shape of the one-launch path: nr rounds of kSyncThreads slots per
 // block (at least kSyncMinRounds, more when the blocks would not all be
 // resident), G = ceil(S / (nr * kSyncThreads)) blocks.  False when the
-// problem needs more than kSyncMaxRounds rounds or kMaxSyncTiles blocks.
-bool sync_shape(int64_t S, int64_t resident, int *nr_out, int *G_out) {
+// problem needs more than kSyncMaxRounds rounds or kMaxSyncTiles blocks,
+// or has more experts than a block has threads.
+bool sync_shape(int64_t S, int E, int64_t resident, int *nr_out, int *G_out) {
+    if (E + 1 > kSyncThreads) return false;
     const int64_t cap = resident < kMaxSyncTiles ? resident : kMaxSyncTiles;
     if (cap < 1) return false;
     int64_t nr = (S + cap * kSyncThreads - 1) / (cap * kSyncThreads);
@@ -731,8 +861,8 @@ cudaError_t launch_sync(const IdT *ids, int64_t base, int64_t S, int E, int A, v
                         int32_t *out_perm, int32_t *diag, cudaStream_t stream) {
     auto kern = prep_sync_kernel<IdT>;
     int nr = 0, G = 0;
-    if (!sync_shape(S, (int64_t)sm_count(), &nr, &G)) return cudaErrorCooperativeLaunchTooLarge;
-    const size_t smem = tile_smem<kSyncThreads>(E, G);
+    if (!sync_shape(S, E, (int64_t)sm_count(), &nr, &G)) return cudaErrorCooperativeLaunchTooLarge;
+    const size_t smem = sync_smem<kSyncThreads>(E, G, nr);
     if (smem > 200 * 1024) return cudaErrorCooperativeLaunchTooLarge;
     const int64_t resident = (int64_t)sm_count() * blocks_per_sm(kern, kSyncThreads, smem);
     if (G > resident) return cudaErrorCooperativeLaunchTooLarge;

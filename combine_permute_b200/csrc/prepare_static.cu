@@ -26,13 +26,20 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_scratch_addr[kMaxDevices];  // device address of g_prepare_scratch, per device
 
-// Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached.
-cudaError_t scratch_address(int dev, void **out) {
+// Device address of the scratch array on the current device (with that
+// device current).  Outside stream capture it is looked up on every call and
+// the cache refreshed, so that a context torn down and created again (after
+// cudaDeviceReset, say) never leaves a stale address behind; while a stream
+// is being captured the cached address is used, since the first call on the
+// device came before any capture.
+cudaError_t scratch_address(int dev, cudaStream_t stream, void **out) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> g(g_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    if (cap == cudaStreamCaptureStatusNone || g_scratch_addr[dev] == nullptr) {
         void *p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_prepare_scratch);
+        e = cudaGetSymbolAddress(&p, g_prepare_scratch);
         if (e != cudaSuccess) return e;
         g_scratch_addr[dev] = p;
     }
@@ -67,7 +74,7 @@ extern "C" moe_status_t moe_prepare_no_alloc(const int32_t *topk_ids, int64_t nu
         cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return moe::status_from_cuda(e);
         if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-        e = scratch_address(dev, &scratch);
+        e = scratch_address(dev, (cudaStream_t)stream, &scratch);
         if (e != cudaSuccess) return moe::status_from_cuda(e);
         // the array keeps whatever the last call left: the look-back words
         // must start at zero

@@ -408,8 +408,8 @@ moe_status_t moe_output_memset(void *out, moe_dtype_t dtype, int64_t num_tokens,
  * workspace the call uses one fixed device array of
  * MOE_PREPARE_NO_ALLOC_SCRATCH_BYTES (4 MiB), which every GPU that loads the
  * library holds until the process exits.  A problem that needs more scratch
- * than that (moe_prepare_workspace_bytes() above 4 MiB: T*k beyond about 4.1
- * million slots with 256 experts, about 1 million with 1024) is rejected
+ * than that (moe_prepare_workspace_bytes() above 4 MiB: T*k beyond about 3.6
+ * million slots with 256 experts, about 0.9 million with 1024) is rejected
  * with MOE_ERR_UNSUPPORTED before anything is launched.  The call allocates
  * nothing: it clears the part of the array it needs with cudaMemsetAsync on
  * `stream`, then launches the same kernels as moe_prepare.
@@ -417,10 +417,11 @@ moe_status_t moe_output_memset(void *out, moe_dtype_t dtype, int64_t num_tokens,
  * All calls on one device share the array and it keeps the last call's
  * contents, so two calls whose work overlaps on the GPU (different streams
  * with no ordering between them) race and produce wrong results: order them
- * on one stream, or use moe_prepare with separate workspaces.  The first
- * call on a device that needs the scratch (T*k above 4096) looks up the
- * array's device address, once per device; make that first call before any
- * stream capture begins.
+ * on one stream, or use moe_prepare with separate workspaces.  A call that
+ * needs the scratch (T*k above 4096) looks up the array's device address on
+ * its device whenever its stream is not being captured; a call made during
+ * stream capture uses the address found by an earlier call, so make one
+ * such call on the device before any stream capture begins.
  */
 moe_status_t moe_prepare_no_alloc(const int32_t *topk_ids, int64_t num_tokens, int32_t top_k,
                                   int32_t num_experts, int32_t *expert_counts,
@@ -428,6 +429,53 @@ moe_status_t moe_prepare_no_alloc(const int32_t *topk_ids, int64_t num_tokens, i
                                   int32_t blockscale_align, int32_t *input_permutation,
                                   int32_t *output_permutation, int32_t *diag,
                                   moe_stream_t stream);
+
+/* Largest num_ranks * num_local_experts of moe_ep_recv_layout. */
+#define MOE_EP_MAX_GROUPS 8192
+
+/*
+ * Expert-parallel exchange between GPUs, the receiving rank's layout
+ * (Mooncake PR #4581: dispatch / combine across ranks, "dispatch and combine
+ * kernel implementations"; TensorRT-LLM PR #9592: "Alltoall comm", and one
+ * rank's experts being the window local_expert_offset .. +
+ * num_local_experts).
+ *
+ * R = num_ranks ranks each own El = num_local_experts consecutive experts
+ * (rank r: experts [r*El, (r+1)*El)).  A source rank runs moe_prepare over
+ * all R*El experts and dispatches; its dispatched rows are sorted by
+ * expert, so rows [expert_offsets[r*El], expert_offsets[(r+1)*El]) go to
+ * rank r as one block ordered by local expert, and its expert_counts,
+ * viewed [R][El], are what it tells each rank.  This rank receives:
+ *
+ *   recv_expert_counts [R, El] int32  rows source s sends for local expert le
+ *   (the received buffer holds the source blocks in source order)
+ *
+ * and this call writes
+ *
+ *   recv_offsets   [R+1]  int32  first received row of each source block
+ *   local_offsets  [El+1] int32  expert offsets of the grouped layout (by
+ *                                local expert, then source, then the
+ *                                source's own order): what the expert
+ *                                stage's grouped GEMM takes
+ *   recv_to_local  [N]    int32  grouped row of every received row
+ *   local_to_recv  [N]    int32  its inverse
+ *   num_recv       [1]    int32  N, the number of received rows
+ *
+ * The maps are written only when N <= capacity (their allocated length);
+ * otherwise only the offsets and num_recv are, so the caller can size them.
+ * Received rows move into the grouped layout with moe_dispatch_rows(recv,
+ * top_k = 1, input_permutation = local_to_recv) and expert outputs back to
+ * the received order with input_permutation = recv_to_local.  All pointers
+ * are device memory; nothing is allocated.  Errors: MOE_ERR_INVALID_ARG for
+ * num_ranks or num_local_experts < 1, capacity < 0, a NULL offset / count
+ * output or a NULL map with capacity > 0; MOE_ERR_UNSUPPORTED when
+ * num_ranks * num_local_experts > MOE_EP_MAX_GROUPS.
+ */
+moe_status_t moe_ep_recv_layout(const int32_t *recv_expert_counts, int32_t num_ranks,
+                                int32_t num_local_experts, int64_t capacity,
+                                int32_t *recv_offsets, int32_t *local_offsets,
+                                int32_t *recv_to_local, int32_t *local_to_recv,
+                                int32_t *num_recv, moe_stream_t stream);
 
 /* Largest T*k that moe_prepare_dispatch accepts. */
 #define MOE_FUSED_MAX_SLOTS 4096

@@ -1,0 +1,145 @@
+"""Expert-parallel exchange on the GPU: the receive-layout kernel against
+the oracle, the exchange of R ranks emulated on one GPU through the
+library's kernels, and combine_permute_b200.ep over a one-rank NCCL group.
+
+The emulation moves each source's row block to its destination with a
+device copy (what the all-to-all does between GPUs), so every per-rank step
+runs in the library's kernels: prepare, dispatch, the receive layout, the
+regroup gathers and combine.  The result must be bit-exact against the
+single-GPU answer of the oracle over all ranks' tokens taken together.
+"""
+
+import ctypes
+import dataclasses
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import combine_permute_b200 as moe
+import oracle
+from combine_permute_b200 import _lib
+from tests._helpers import bits
+from workloads import CONFIGS, make_workload
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+def _counts(R, El, seed, zero_frac=0.3, hi=50):
+    rng = np.random.default_rng(seed)
+    c = rng.integers(0, hi, size=(R, El)).astype(np.int32)
+    c[rng.random((R, El)) < zero_frac] = 0
+    return c
+
+
+@pytest.mark.parametrize("R,El,seed", [(1, 1, 0), (2, 128, 1), (8, 32, 2), (4, 288, 3),
+                                       (64, 128, 4), (8, 1024, 5), (3, 7, 6)])
+def test_recv_layout_matches_oracle(R, El, seed):
+    c = _counts(R, El, seed, hi=30 if R * El > 2000 else 200)
+    ref = oracle.ep_recv_layout(c)
+    n = int(c.sum())
+    lay = moe.moe_ep_recv_layout(torch.from_numpy(c).to(DEV), n)
+    torch.cuda.synchronize()
+    assert int(lay.num_recv.item()) == n
+    for key in ("recv_offsets", "local_offsets", "recv_to_local", "local_to_recv"):
+        assert np.array_equal(getattr(lay, key).cpu().numpy(), ref[key]), key
+
+
+def test_recv_layout_empty_and_capacity_overflow():
+    c = np.zeros((4, 16), np.int32)
+    lay = moe.moe_ep_recv_layout(torch.from_numpy(c).to(DEV), 0)
+    torch.cuda.synchronize()
+    assert int(lay.num_recv.item()) == 0 and not lay.recv_offsets.any() and not lay.local_offsets.any()
+    # too small a capacity: offsets and the count only, maps untouched
+    c = _counts(4, 16, 9)
+    n = int(c.sum())
+    lib = _lib.load()
+    i32 = dict(dtype=torch.int32, device=DEV)
+    ro, lo, num = torch.empty(5, **i32), torch.empty(17, **i32), torch.empty(1, **i32)
+    r2l, l2r = torch.full((n,), -5, **i32), torch.full((n,), -5, **i32)
+    st = lib.moe_ep_recv_layout(torch.from_numpy(c).to(DEV).data_ptr(), 4, 16, n - 1,
+                                ro.data_ptr(), lo.data_ptr(), r2l.data_ptr(), l2r.data_ptr(),
+                                num.data_ptr(), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.synchronize()
+    ref = oracle.ep_recv_layout(c)
+    assert int(num.item()) == n and np.array_equal(ro.cpu().numpy(), ref["recv_offsets"])
+    assert np.array_equal(lo.cpu().numpy(), ref["local_offsets"])
+    assert (r2l == -5).all() and (l2r == -5).all()
+
+
+@pytest.mark.parametrize("R,T,seed", [(2, 700, 0), (4, 1500, 1), (8, 300, 2)])
+def test_exchange_of_emulated_ranks_matches_single_gpu(R, T, seed):
+    """R ranks of the uniform workload's shape (E = 256 experts, top-8,
+    H = 7168, bf16), each with its own tokens; rank r owns 256 / R experts."""
+    base = CONFIGS["uniform_t4096_h7168_e256_k8"]
+    E, k, H = base.E, base.k, base.H
+    El = E // R
+    ranks = []
+    for r in range(R):
+        w = dataclasses.replace(base, T=T + 37 * r, seed=seed * 100 + r, name=f"rank{r}")
+        ids_np, wt_np, x, _ = make_workload(w, device=DEV, with_y=False)
+        ids_np[::53, 0] = -1  # a few invalid ids
+        meta = moe.moe_prepare(torch.from_numpy(ids_np).to(DEV), E)
+        xd = moe.moe_dispatch_rows(x, k, meta.input_permutation, meta.output_permutation)
+        ranks.append(dict(T=w.T, ids=ids_np, wt=wt_np, x=x, meta=meta, xd=xd,
+                          bounds=meta.expert_offsets[::El].tolist()))
+    # one-GPU answer over every rank's tokens (oracle)
+    g = oracle.prepare(np.concatenate([r["ids"] for r in ranks]), E)
+    xg = np.concatenate([bits(r["x"]) for r in ranks])
+    want = oracle.dispatch(xg, k, g["input_perm"])
+    S = sum(r["T"] for r in ranks) * k
+    y_global = torch.randn(S, H, generator=torch.Generator().manual_seed(seed)).to(torch.bfloat16)
+    backs = [torch.zeros(r["T"] * k, H, dtype=torch.bfloat16, device=DEV) for r in ranks]
+    for dst in range(R):
+        counts = torch.stack([r["meta"].expert_counts[dst * El:(dst + 1) * El] for r in ranks])
+        blocks = [r["xd"][r["bounds"][dst]:r["bounds"][dst + 1]] for r in ranks]
+        recv = torch.cat(blocks)  # the all-to-all, as device copies
+        lay = moe.moe_ep_recv_layout(counts.contiguous(), recv.shape[0])
+        grouped = moe.moe_dispatch_rows(recv, 1, input_permutation=lay.local_to_recv)
+        lo, hi = g["offsets"][dst * El], g["offsets"][(dst + 1) * El]
+        assert np.array_equal(bits(grouped), want[lo:hi]), dst
+        assert np.array_equal(lay.local_offsets.cpu().numpy(),
+                              g["offsets"][dst * El:(dst + 1) * El + 1] - lo)
+        # expert outputs of this window back to the sources' dispatched order
+        y_recv = moe.moe_dispatch_rows(y_global[lo:hi].to(DEV).contiguous(), 1,
+                                       input_permutation=lay.recv_to_local)
+        q = 0
+        for s, r in enumerate(ranks):
+            m = r["bounds"][dst + 1] - r["bounds"][dst]
+            backs[s][r["bounds"][dst]:r["bounds"][dst + 1]] = y_recv[q:q + m]
+            q += m
+    full = oracle.combine(bits(y_global), "bf16", g["output_perm"],
+                          np.concatenate([r["wt"] for r in ranks]), "bf16")
+    t0 = 0
+    for s, r in enumerate(ranks):
+        out = moe.moe_combine(backs[s], r["meta"].output_permutation,
+                              torch.from_numpy(r["wt"]).to(DEV))
+        assert np.array_equal(bits(out), full[t0:t0 + r["T"]]), s
+        t0 += r["T"]
+
+
+def test_ep_module_over_a_one_rank_nccl_group():
+    import torch.distributed as dist
+    from combine_permute_b200 import ep
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=DEV)
+    try:
+        w = CONFIGS["uniform_t4096_h7168_e256_k8"].scaled(900)
+        ids_np, wt_np, x, y = make_workload(w, device=DEV)
+        grouped, local_offsets, handle = ep.ep_dispatch(x, torch.from_numpy(ids_np).to(DEV), w.E)
+        out = ep.ep_combine(y, torch.from_numpy(wt_np).to(DEV), handle)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    ref = oracle.prepare(ids_np, w.E)
+    # one rank owns every expert: the grouped rows are the dispatched rows
+    assert np.array_equal(bits(grouped), oracle.dispatch(bits(x), w.k, ref["input_perm"]))
+    assert np.array_equal(local_offsets.cpu().numpy(), ref["offsets"])
+    assert np.array_equal(bits(out), oracle.combine(bits(y), "bf16", ref["output_perm"], wt_np,
+                                                    "bf16"))

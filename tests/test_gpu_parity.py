@@ -133,6 +133,21 @@ def test_prepare_deterministic_and_workspace_reusable(T):
     assert runs[-1].diag.cpu().tolist() == [0, 0]
 
 
+def test_one_workspace_shared_by_both_tiled_paths():
+    """One workspace, calls alternating between the one-launch path (grid
+    barrier, histogram rows) and the two-kernel path (look-back words) with
+    different sizes and expert counts: neither path may read the other's
+    data (or an earlier call's) as its own."""
+    rng = np.random.default_rng(4242)
+    shapes = [(15000, 8, 5), (170000, 8, 288), (40000, 3, 64), (300000, 6, 64),
+              (60000, 8, 288), (170000, 8, 288), (9000, 8, 256)]
+    need = max(moe.moe_prepare_workspace_bytes(T, k, E) for T, k, E in shapes)
+    ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
+    for T, k, E in shapes:
+        ids = _ids_random(rng, T, k, E, p_invalid=0.02, distinct=False)
+        _check_prepare(ids, E, A=64, workspace=ws)
+
+
 # ---------------------------------------------------------------------------
 # dispatch (same dtype)
 # ---------------------------------------------------------------------------
