@@ -548,6 +548,14 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
         per_graph = time_calls_in_graph(step, dev, K, n_graph)
     except Exception as exc:
         print(f"in-graph call timing unavailable: {exc}", file=sys.stderr)
+    # ---- timed region 4: every call alone, as its average launch time over
+    #      a graph of n back-to-back launches with events only around the
+    #      graph (no event between launches, so nothing separates them)
+    alone = None
+    try:
+        alone = time_calls_alone(step, dev, K, n_graph)
+    except Exception as exc:
+        print(f"back-to-back call timing unavailable: {exc}", file=sys.stderr)
 
     counts = step.meta_bufs["expert_counts"].cpu().numpy()
     diag = step.meta_bufs["diag"].cpu().numpy().tolist()
@@ -571,6 +579,8 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
         if per_graph is not None:
             per_graph = {"prepare_dispatch": per_graph["prepare"],
                          "combine": per_graph["combine"], "step": per_graph["step"]}
+        if alone is not None:
+            alone = {"prepare_dispatch": alone["prepare"], "combine": alone["combine"]}
     calls = [c for c in ("prepare", "dispatch", "prepare_dispatch", "combine") if c in alg]
     # the breakdown and the roofline use the in-graph times (the calls as the
     # headline's graph runs them); the eager ones add each launch's host and
@@ -592,6 +602,11 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
                         "frac_of_8tbs_spec": gbs / SPEC_HBM_GBS,
                         "eager_us_mean": eager_kern[k] * 1e3,
                         "eager_latency_ms": percentiles(per[k])}
+        if alone is not None:
+            a_gbs = alg[k] / (alone[k] * 1e-3) / 1e9
+            breakdown[k].update({"alone_us_mean": alone[k] * 1e3, "alone_effective_gbs": a_gbs,
+                                 "alone_frac_of_measured_peak": a_gbs / peak,
+                                 "alone_frac_of_8tbs_spec": a_gbs / SPEC_HBM_GBS})
     step_alg = sum(alg.values())
     breakdown["end_to_end"] = {
         "latency_ms": percentiles(timed["step"]),
@@ -600,6 +615,11 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
         "graph_ms_per_step": None if graph_ms is None else graph_ms / K,
         "effective_gbs": step_alg / (elapsed_ms / K * 1e-3) / 1e9,
         "frac_of_measured_peak": step_alg / (elapsed_ms / K * 1e-3) / 1e9 / peak}
+    if per_graph is not None and graph_ms is not None:
+        # what the timing events between the calls add to a step: the calls
+        # timed with events, summed, against the event-free graph's step
+        breakdown["end_to_end"]["event_overhead_us_per_step"] = (
+            (sum(kern[c] for c in calls) - graph_ms / K) * 1e3)
     return {
         "value": whole_job_tokens_per_s(w.T, K, world, elapsed_ms),
         "ms_per_step": elapsed_ms / K,
@@ -626,7 +646,23 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
     }
 
 
-def run_gpu(args, names):
+def profile_run(args, workloads):
+    """W warm-up and K eager steps of each workload, nothing else: the
+    program the ncu captures run."""
+    import torch
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    for w in workloads:
+        step = Step(w, dev)
+        for _ in range(args.warmup + args.steps):
+            step.run()
+        torch.cuda.synchronize(dev)
+        del step
+        torch.cuda.empty_cache()
+    print("profile run done", flush=True)
+
+
+def run_gpu(args, names, workloads=None):
     """Every workload in ``names`` on this rank's GPU; the first is the
     headline, the others go under "per_workload"."""
     import torch
@@ -638,15 +674,16 @@ def run_gpu(args, names):
     if ranks.world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={ranks.world}")
     results = {}
+    workloads = workloads or {n: CONFIGS[n] for n in names}
     for i, name in enumerate(names):
         budget = 0.0 if args.no_cpu_baseline else args.cpu_budget * (1.0 if i == 0 else 0.5)
-        results[name] = bench_workload(args, CONFIGS[name], dev, ranks, budget)
+        results[name] = bench_workload(args, workloads[name], dev, ranks, budget)
     world = ranks.world
     ranks.close()
     if ranks.rank != 0:
         return
     head_name = names[0]
-    w = CONFIGS[head_name]
+    w = workloads[head_name]
     r = results[head_name]
     line = {
         "metric": METRIC, "value": r["value"], "unit": "tokens/s", "n_gpus": world,
@@ -658,8 +695,8 @@ def run_gpu(args, names):
     line.update({k: v for k, v in r.items() if k not in ("value", "ms_per_step", "launch")})
     if len(names) > 1:
         line["per_workload"] = {
-            n: dict(results[n], config=dict(_config(CONFIGS[n], world), launch=results[n]["launch"]),
-                    dtype=_dtype_tag(CONFIGS[n]))
+            n: dict(results[n], config=dict(_config(workloads[n], world), launch=results[n]["launch"]),
+                    dtype=_dtype_tag(workloads[n]))
             for n in names[1:]}
     print(json.dumps(line), flush=True)
 
@@ -702,6 +739,44 @@ def time_calls_in_graph(step, dev, K, n_graph):
             per["step"].append(m[0].elapsed_time(m[3]))
     del g
     return per
+
+
+def time_calls_alone(step, dev, K, n):
+    """Average launch time (ms) of each call of the step, alone: a CUDA graph
+    of n back-to-back launches of that call on the step's buffers (the
+    metadata of one prepare), events only around the graph, replayed K / n
+    times."""
+    import torch
+    meta = step.prepare_dispatch() if step.fused else step.prepare()
+    torch.cuda.synchronize(dev)
+    calls = {"combine": lambda: step.combine(meta)}
+    if step.fused:
+        calls["prepare"] = step.prepare_dispatch
+    else:
+        calls["prepare"] = step.prepare
+        calls["dispatch"] = lambda: step.dispatch(meta)
+    out = {}
+    for name, fn in calls.items():
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            fn()
+            with torch.cuda.graph(g, stream=side):
+                for _ in range(n):
+                    fn()
+        torch.cuda.synchronize(dev)
+        g.replay()
+        torch.cuda.synchronize(dev)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(max(1, K // n)):
+            g.replay()
+        e.record()
+        torch.cuda.synchronize(dev)
+        out[name] = s.elapsed_time(e) / (max(1, K // n) * n)
+        del g
+    return out
 
 
 def time_next_rows(step, w, dev, reps=20):
@@ -860,6 +935,12 @@ def main():
                     help="seconds of oracle time per workload (headline); half that for the others")
     ap.add_argument("--ref-budget", type=float, default=90.0,
                     help="seconds of oracle time for the whole reference run")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="run the workload's routing, shapes and dtypes at this many tokens "
+                         "(smaller cases for profiling)")
+    ap.add_argument("--profile-run", action="store_true",
+                    help="only the warm-up and K eager steps of each workload, no JSON line "
+                         "(a short program for ncu)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -867,10 +948,14 @@ def main():
         names = [HEADLINE_WORKLOAD] + [n for n in CONFIGS if n != HEADLINE_WORKLOAD]
     else:
         names = [args.workload]
+    workloads = {n: CONFIGS[n] if args.tokens is None else CONFIGS[n].scaled(args.tokens)
+                 for n in names}
     if args.impl == "reference":
-        run_reference(args, CONFIGS[names[0]])
+        run_reference(args, workloads[names[0]])
+    elif args.profile_run:
+        profile_run(args, [workloads[n] for n in names])
     else:
-        run_gpu(args, names)
+        run_gpu(args, names, workloads)
 
 
 if __name__ == "__main__":
