@@ -1,6 +1,7 @@
-"""The stored expected values of tests/golden/ (written by the oracle, see
-tests/golden/README.md): the oracle still produces them (CPU), and the CUDA
-path, called through the C ABI, reproduces them bit for bit (GPU)."""
+"""The stored expected values of tests/golden/, written by
+tests/golden/make_golden.py from the oracle and the seeded generators alone:
+the oracle still produces them (CPU), and the CUDA path, called through the
+C ABI, reproduces them bit for bit (GPU)."""
 
 import json
 import os
