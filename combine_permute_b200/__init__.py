@@ -40,6 +40,10 @@ __all__ = [
     "moe_output_memset",
     "moe_ep_recv_layout",
     "EpRecvLayout",
+    "moe_ep_peer_layout",
+    "EpPeerLayout",
+    "moe_ep_dispatch_peer",
+    "moe_ep_combine_peer",
     "TileLayout",
     "library_path",
 ]
@@ -67,6 +71,13 @@ class EpRecvLayout(NamedTuple):
     recv_to_local: torch.Tensor   # [N] int32
     local_to_recv: torch.Tensor   # [N] int32
     num_recv: torch.Tensor        # [1] int32
+
+
+class EpPeerLayout(NamedTuple):
+    dest_rank: torch.Tensor       # [T*k] int32: rank owning each slot's expert (-1: none)
+    dest_row: torch.Tensor        # [T*k] int32: the slot's row in that rank's grouped buffer
+    recv_rows: torch.Tensor       # [R] int32: rows of each rank's grouped buffer
+    local_offsets: torch.Tensor   # [El+1] int32: this rank's grouped expert offsets
 
 
 class PrepareResult(NamedTuple):
@@ -481,3 +492,82 @@ def moe_ep_recv_layout(recv_expert_counts: torch.Tensor, num_recv: int) -> EpRec
             _ptr(lay.local_to_recv) if num_recv else None, lay.num_recv.data_ptr(), _stream(dev))
     _lib.check("moe_ep_recv_layout", st)
     return lay
+
+
+def moe_ep_peer_layout(all_expert_counts: torch.Tensor, rank: int, topk_ids: torch.Tensor,
+                       meta: PrepareResult) -> EpPeerLayout:
+    """Every slot's destination rank and row in the owners' grouped buffers
+    (see include/moe.h).  ``all_expert_counts`` [R, E] int32 holds every
+    rank's expert counts; ``meta`` is this rank's moe_prepare over all E
+    experts of ``topk_ids`` [T, k]."""
+    _need(all_expert_counts, "all_expert_counts", torch.int32)
+    if all_expert_counts.dim() != 2:
+        raise ValueError("all_expert_counts must be [num_ranks, num_experts]")
+    R, E = all_expert_counts.shape
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    _need(topk_ids, "topk_ids", torch.int32, (T, k), dev)
+    i32 = dict(dtype=torch.int32, device=dev)
+    lay = EpPeerLayout(torch.empty(T * k, **i32), torch.empty(T * k, **i32), torch.empty(R, **i32),
+                       torch.empty(E // R + 1 if R and E % R == 0 else 1, **i32))
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_ep_peer_layout(
+            all_expert_counts.data_ptr(), R, rank, E, topk_ids.data_ptr(), T, k,
+            meta.expert_offsets.data_ptr(), meta.output_permutation.data_ptr(),
+            lay.dest_rank.data_ptr(), lay.dest_row.data_ptr(), lay.recv_rows.data_ptr(),
+            lay.local_offsets.data_ptr(), _stream(dev))
+    _lib.check("moe_ep_peer_layout", st)
+    return lay
+
+
+def _pointer_array(buffers, dev) -> torch.Tensor:
+    """A device array of the buffers' addresses (tensors, or raw device
+    addresses valid in this process, e.g. another GPU's memory mapped in)."""
+    ptrs = [b.data_ptr() if isinstance(b, torch.Tensor) else int(b) for b in buffers]
+    return torch.tensor(ptrs, dtype=torch.int64).to(dev)
+
+
+def moe_ep_dispatch_peer(x: torch.Tensor, top_k: int, layout: EpPeerLayout, recv_buffers) -> None:
+    """Stores every row of x [T, H] into the grouped buffers of the ranks
+    owning its experts (``recv_buffers``: one per rank, tensors or device
+    addresses; see include/moe.h)."""
+    _need(x, "x")
+    T, H = x.shape
+    dev = x.device
+    R = layout.recv_rows.numel()
+    if len(recv_buffers) != R:
+        raise ValueError(f"{len(recv_buffers)} buffers for {R} ranks")
+    ptrs = _pointer_array(recv_buffers, dev)
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_ep_dispatch_peer(
+            x.data_ptr(), _dtype_code(x.dtype), T, H, top_k, layout.dest_rank.data_ptr(),
+            layout.dest_row.data_ptr(), ptrs.data_ptr(), layout.recv_rows.data_ptr(), R,
+            _stream(dev))
+    _lib.check("moe_ep_dispatch_peer", st)
+    ptrs.record_stream(torch.cuda.current_stream(dev))
+
+
+def moe_ep_combine_peer(out_buffers, y_dtype: torch.dtype, hidden: int, layout: EpPeerLayout,
+                        weights: torch.Tensor, *, out_dtype: Optional[torch.dtype] = None,
+                        out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out[t] = sum_j weights[t, j] * (expert output of slot (t, j), read from
+    its owner's buffer ``out_buffers[rank]``), fp32 accumulation in slot
+    order (see include/moe.h)."""
+    _need(weights, "weights", torch.float32)
+    T, k = weights.shape
+    dev = weights.device
+    R = layout.recv_rows.numel()
+    if len(out_buffers) != R:
+        raise ValueError(f"{len(out_buffers)} buffers for {R} ranks")
+    if out is None:
+        out = torch.empty((T, hidden), dtype=out_dtype or y_dtype, device=dev)
+    _need(out, "out", None, (T, hidden), dev)
+    ptrs = _pointer_array(out_buffers, dev)
+    with torch.cuda.device(dev):
+        st = _lib.load().moe_ep_combine_peer(
+            ptrs.data_ptr(), layout.recv_rows.data_ptr(), R, _dtype_code(y_dtype), T, hidden, k,
+            layout.dest_rank.data_ptr(), layout.dest_row.data_ptr(), weights.data_ptr(),
+            out.data_ptr(), _dtype_code(out.dtype), _stream(dev))
+    _lib.check("moe_ep_combine_peer", st)
+    ptrs.record_stream(torch.cuda.current_stream(dev))
+    return out

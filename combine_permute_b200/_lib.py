@@ -42,6 +42,9 @@ EXPORTED = (
     "moe_prepare_local",
     "moe_output_memset",
     "moe_ep_recv_layout",
+    "moe_ep_peer_layout",
+    "moe_ep_dispatch_peer",
+    "moe_ep_combine_peer",
 )
 
 _vp = ctypes.c_void_p
@@ -75,6 +78,11 @@ _SIGNATURES = {
                                  _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "moe_output_memset": (_int, [_vp, _int, _i64, _i64, _i32, _vp, _vp]),
     "moe_ep_recv_layout": (_int, [_vp, _i32, _i32, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_ep_peer_layout": (_int, [_vp, _i32, _i32, _i32, _vp, _i64, _i32, _vp, _vp, _vp, _vp, _vp,
+                                  _vp, _vp]),
+    "moe_ep_dispatch_peer": (_int, [_vp, _int, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _i32, _vp]),
+    "moe_ep_combine_peer": (_int, [_vp, _vp, _i32, _int, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _int,
+                                   _vp]),
 }
 
 _lib = None

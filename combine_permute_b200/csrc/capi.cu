@@ -301,4 +301,67 @@ moe_status_t moe_ep_recv_layout(const int32_t *recv_expert_counts, int32_t num_r
                                              local_to_recv, num_recv, (cudaStream_t)stream));
 }
 
+moe_status_t moe_ep_peer_layout(const int32_t *all_expert_counts, int32_t num_ranks,
+                                int32_t rank, int32_t num_experts, const int32_t *topk_ids,
+                                int64_t num_tokens, int32_t top_k,
+                                const int32_t *expert_offsets,
+                                const int32_t *output_permutation, int32_t *dest_rank,
+                                int32_t *dest_row, int32_t *recv_rows, int32_t *local_offsets,
+                                moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (num_ranks < 1 || rank < 0 || rank >= num_ranks || num_experts < 1 ||
+        num_experts % num_ranks != 0)
+        return MOE_ERR_INVALID_ARG;
+    if (num_experts > moe::kMaxExperts) return MOE_ERR_UNSUPPORTED;
+    if (!all_expert_counts || !expert_offsets || !recv_rows || !local_offsets)
+        return MOE_ERR_INVALID_ARG;
+    const int64_t S = num_tokens * (int64_t)top_k;
+    if (S > 0 && (!topk_ids || !output_permutation || !dest_rank || !dest_row))
+        return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_ep_peer_layout(all_expert_counts, num_ranks, rank, num_experts,
+                                             topk_ids, S, expert_offsets, output_permutation,
+                                             dest_rank, dest_row, recv_rows, local_offsets,
+                                             (cudaStream_t)stream));
+}
+
+moe_status_t moe_ep_dispatch_peer(const void *x, moe_dtype_t dtype, int64_t num_tokens,
+                                  int64_t hidden, int32_t top_k, const int32_t *dest_rank,
+                                  const int32_t *dest_row, void *const *recv_buffers,
+                                  const int32_t *recv_rows, int32_t num_ranks,
+                                  moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (!io_dtype(dtype) || hidden < 1 || num_ranks < 1) return MOE_ERR_INVALID_ARG;
+    const int64_t row_bytes = hidden * moe::dtype_bytes(dt(dtype));
+    if (row_bytes % 16 != 0) return MOE_ERR_INVALID_ARG;
+    if (num_tokens == 0) return MOE_OK;
+    if (!x || !dest_rank || !dest_row || !recv_buffers || !recv_rows || !aligned16(x))
+        return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_dispatch_peer(x, num_tokens, row_bytes, top_k, dest_rank, dest_row,
+                                            recv_buffers, recv_rows, num_ranks,
+                                            (cudaStream_t)stream));
+}
+
+moe_status_t moe_ep_combine_peer(const void *const *out_buffers, const int32_t *recv_rows,
+                                 int32_t num_ranks, moe_dtype_t y_dtype, int64_t num_tokens,
+                                 int64_t hidden, int32_t top_k, const int32_t *dest_rank,
+                                 const int32_t *dest_row, const float *weights, void *out,
+                                 moe_dtype_t out_dtype, moe_stream_t stream) {
+    moe_status_t st = check_tk(num_tokens, top_k);
+    if (st != MOE_OK) return st;
+    if (!io_dtype(y_dtype) || !io_dtype(out_dtype) || hidden < 1 || num_ranks < 1)
+        return MOE_ERR_INVALID_ARG;
+    if ((hidden * moe::dtype_bytes(dt(y_dtype))) % 16 != 0 ||
+        (hidden * moe::dtype_bytes(dt(out_dtype))) % 16 != 0)
+        return MOE_ERR_INVALID_ARG;
+    if (num_tokens == 0) return MOE_OK;
+    if (!out_buffers || !recv_rows || !dest_rank || !dest_row || !weights || !out)
+        return MOE_ERR_INVALID_ARG;
+    if (!aligned16(out) || ((uintptr_t)weights & 3u)) return MOE_ERR_INVALID_ARG;
+    return from_cuda(moe::run_combine_peer(out_buffers, recv_rows, num_ranks, dt(y_dtype),
+                                           num_tokens, hidden, top_k, dest_rank, dest_row,
+                                           weights, out, dt(out_dtype), (cudaStream_t)stream));
+}
+
 }  // extern "C"

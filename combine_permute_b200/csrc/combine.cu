@@ -21,6 +21,7 @@ namespace {
 constexpr int kCombineThreads = 128;
 constexpr int kBatch = 8;  // slots whose loads are in flight together
 
+
 typedef unsigned long long f32x2;  // two fp32 values, low word = first element
 
 __device__ __forceinline__ f32x2 pack2(float lo, float hi) {
@@ -95,31 +96,75 @@ template <int P> struct Store<float, P> {
     }
 };
 
-// Row indices and weights of slots j0 .. j0+kBatch-1 of one token; an
-// invalid or out-of-range slot gets row -1 and contributes nothing.
-__device__ __forceinline__ void load_batch(int64_t S, const int32_t *rows, const float *wt, int j0,
-                                           int k, int (&row)[kBatch], float (&wj)[kBatch]) {
+// Where the expert output of each slot is read.  LocalRows: row
+// output_permutation[i] of this GPU's y.  PeerRows: the row each slot's
+// destination rank holds in its grouped buffer (the fused exchange between
+// GPUs; a buffer may be another GPU's memory mapped into this process, read
+// with plain loads).  A slot without a valid row contributes nothing.
+struct LocalRows {
+    using Ref = int;
+    static constexpr bool kLocal = true;
+    const char *y;
+    const int32_t *perm;
+    int64_t S, row_bytes;
+    __device__ Ref ref(int64_t i) const {
+        const int p = __ldg(perm + i);
+        return p >= 0 && p < S ? p : -1;
+    }
+    __device__ static Ref none() { return -1; }
+    __device__ static bool valid(Ref r) { return r >= 0; }
+    __device__ const char *addr(Ref r, int64_t coff) const {
+        return y + (int64_t)r * row_bytes + coff;
+    }
+};
+
+struct PeerRows {
+    using Ref = const char *;
+    static constexpr bool kLocal = false;
+    const char *const *bufs;  // [R] each rank's grouped buffer of expert outputs
+    const int32_t *rank;      // [S] destination rank of every slot (-1: none)
+    const int32_t *row;       // [S] and its row there
+    const int32_t *nrows;     // [R] rows of each buffer
+    int R;
+    int64_t row_bytes;
+    __device__ Ref ref(int64_t i) const {
+        const int r = __ldg(rank + i);
+        if (r < 0 || r >= R) return nullptr;
+        const int q = __ldg(row + i);
+        if (q < 0 || q >= __ldg(nrows + r)) return nullptr;
+        return bufs[r] + (int64_t)q * row_bytes;
+    }
+    __device__ static Ref none() { return nullptr; }
+    __device__ static bool valid(Ref r) { return r != nullptr; }
+    __device__ const char *addr(Ref r, int64_t coff) const { return r + coff; }
+};
+
+// Rows and weights of slots j0 .. j0+kBatch-1 of one token (slot index
+// `first` + j); a slot without a valid row gets weight 0 and is skipped.
+template <typename Rows>
+__device__ __forceinline__ void load_batch(const Rows &rows, int64_t first, const float *wt, int j0,
+                                           int k, typename Rows::Ref (&row)[kBatch],
+                                           float (&wj)[kBatch]) {
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
-        const int p = (j0 + b < k) ? __ldg(rows + j0 + b) : -1;
-        row[b] = (p >= 0 && p < S) ? p : -1;
-        wj[b] = row[b] >= 0 ? __ldg(wt + j0 + b) : 0.0f;
+        row[b] = (j0 + b < k) ? rows.ref(first + j0 + b) : Rows::none();
+        wj[b] = Rows::valid(row[b]) ? __ldg(wt + j0 + b) : 0.0f;
     }
 }
 
 // acc += w_j * y_j for one batch of slots, in slot order, at byte offset
 // `coff` of the rows.
-template <typename YT, int P>
-__device__ __forceinline__ void accumulate_batch(f32x2 (&acc)[P], const char *y, int64_t row_bytes,
-                                                 const int (&row)[kBatch],
+template <typename YT, int P, typename Rows>
+__device__ __forceinline__ void accumulate_batch(f32x2 (&acc)[P], const Rows &rows,
+                                                 const typename Rows::Ref (&row)[kBatch],
                                                  const float (&wj)[kBatch], int64_t coff) {
     uint4 v[kBatch];
 #pragma unroll
     for (int b = 0; b < kBatch; ++b)
-        if (row[b] >= 0) v[b] = ld_stream_v4(y + (int64_t)row[b] * row_bytes + coff);
+        if (Rows::valid(row[b])) v[b] = ld_stream_v4(rows.addr(row[b], coff));
 #pragma unroll
     for (int b = 0; b < kBatch; ++b) {
-        if (row[b] < 0) continue;
+        if (!Rows::valid(row[b])) continue;
         f32x2 yv[P];
         Unpack<YT>::run(v[b], yv);
 #pragma unroll
@@ -136,45 +181,48 @@ __device__ __forceinline__ void accumulate_batch(f32x2 (&acc)[P], const char *y,
 // spread evenly over the persistent grid.  kSmallK: k <= kBatch, and every
 // slot's row and weight stay in registers for the unit; otherwise they are
 // re-read (L1) per column vector.
-template <typename YT, typename OT, bool kSmallK>
-__global__ void __launch_bounds__(kCombineThreads)
-    combine_kernel(const YT *__restrict__ y, int64_t T, int64_t H, int k,
-                   const int32_t *__restrict__ out_perm, const float *__restrict__ w,
+// Resident blocks per SM the compiler must leave room for, for rows read from
+// this GPU: eight for 16-bit expert outputs summed into fp32 (at most 64
+// registers a thread), seven for the others (72); six for rows in other
+// ranks' buffers.  The kernels the workloads use spill nothing.
+template <typename YT, typename OT, typename Rows> constexpr int combine_min_blocks() {
+    return !Rows::kLocal ? 6 : (sizeof(YT) == 2 && sizeof(OT) == 4 ? 8 : 7);
+}
+
+template <typename YT, typename OT, bool kSmallK, typename Rows>
+__global__ void __launch_bounds__(kCombineThreads, combine_min_blocks<YT, OT, Rows>())
+    combine_kernel(const Rows rows, int64_t T, int64_t H, int k, const float *__restrict__ w,
                    OT *__restrict__ out, int64_t nsplit, int64_t vpu) {
     constexpr int VE = 16 / sizeof(YT);    // elements per 16-byte load
     constexpr int P = Unpack<YT>::kPairs;  // fp32 pairs per load
     pdl_wait();
-    pdl_launch_dependents();
     const int64_t nvec = H / VE;
-    const int64_t S = T * k;
-    const int64_t row_bytes = H * (int64_t)sizeof(YT);
-    const char *yb = reinterpret_cast<const char *>(y);
     const int64_t units = T * nsplit;
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
         const int64_t t = u / nsplit;
         const int64_t cbeg = (u - t * nsplit) * vpu;
         const int64_t cend = min(nvec, cbeg + vpu);
-        const int32_t *rows = out_perm + t * k;
         const float *wt = w + t * k;
         char *orow = reinterpret_cast<char *>(out + t * H);
-        int row[kBatch];
+        typename Rows::Ref row[kBatch];
         float wj[kBatch];
-        if (kSmallK) load_batch(S, rows, wt, 0, k, row, wj);
+        if (kSmallK) load_batch(rows, t * k, wt, 0, k, row, wj);
         for (int64_t c = cbeg + threadIdx.x; c < cend; c += kCombineThreads) {
             f32x2 acc[P];
 #pragma unroll
             for (int i = 0; i < P; ++i) acc[i] = 0ull;  // +0.0f, +0.0f
             if (kSmallK) {
-                accumulate_batch<YT, P>(acc, yb, row_bytes, row, wj, c * 16);
+                accumulate_batch<YT, P>(acc, rows, row, wj, c * 16);
             } else {
                 for (int j0 = 0; j0 < k; j0 += kBatch) {
-                    load_batch(S, rows, wt, j0, k, row, wj);
-                    accumulate_batch<YT, P>(acc, yb, row_bytes, row, wj, c * 16);
+                    load_batch(rows, t * k, wt, j0, k, row, wj);
+                    accumulate_batch<YT, P>(acc, rows, row, wj, c * 16);
                 }
             }
             Store<OT, P>::run(orow + c * (int64_t)(VE * sizeof(OT)), acc);
         }
     }
+    pdl_launch_dependents();  // after the work loop: see pdl_launch_dependents
 }
 
 // Column split of the token rows: the number of parts that minimises
@@ -198,29 +246,41 @@ inline int64_t combine_split(int64_t T, int64_t nvec, int64_t grid_max) {
     return best_n;
 }
 
-template <typename YT, typename OT>
-cudaError_t launch_combine(const void *y, int64_t T, int64_t H, int k, const int32_t *out_perm,
-                           const float *w, void *out, int64_t nsplit, cudaStream_t stream) {
-    auto kern = k <= kBatch ? combine_kernel<YT, OT, true> : combine_kernel<YT, OT, false>;
+template <typename YT, typename OT, typename Rows>
+cudaError_t launch_combine(const Rows &rows, int64_t T, int64_t H, int k, const float *w,
+                           void *out, int64_t nsplit, cudaStream_t stream) {
+    auto kern =
+        k <= kBatch ? combine_kernel<YT, OT, true, Rows> : combine_kernel<YT, OT, false, Rows>;
     const int64_t nvec = H / (16 / (int64_t)sizeof(YT));
     const int64_t grid_max = (int64_t)sm_count() * blocks_per_sm(kern, kCombineThreads, 0);
     if (nsplit <= 0) nsplit = combine_split(T, nvec, grid_max);
     const int64_t vpu = (nvec + nsplit - 1) / nsplit;
     const int64_t parts = (nvec + vpu - 1) / vpu;
     const int64_t grid = persistent_grid(kern, kCombineThreads, 0, T * parts);
-    return launch(kern, grid, kCombineThreads, 0, stream, (const YT *)y, T, H, k, out_perm, w,
-                  (OT *)out, parts, vpu);
+    const Start start = streaming_start(T * k * H * (int64_t)sizeof(YT));
+    return launch(kern, grid, kCombineThreads, 0, stream, start, rows, T, H, k, w, (OT *)out, parts,
+                  vpu);
 }
 
-template <typename YT>
-cudaError_t dispatch_out(DType out_dtype, const void *y, int64_t T, int64_t H, int k,
-                         const int32_t *out_perm, const float *w, void *out, int64_t nsplit,
-                         cudaStream_t stream) {
-    switch (out_dtype) {
-    case DType::F32: return launch_combine<YT, float>(y, T, H, k, out_perm, w, out, nsplit, stream);
-    case DType::F16: return launch_combine<YT, __half>(y, T, H, k, out_perm, w, out, nsplit, stream);
-    default:
-        return launch_combine<YT, __nv_bfloat16>(y, T, H, k, out_perm, w, out, nsplit, stream);
+// The combine of element types (y_dtype, out_dtype) over rows made by
+// make_rows(sizeof the y element).
+template <typename MakeRows>
+cudaError_t combine_typed(DType y_dtype, DType out_dtype, int64_t T, int64_t H, int k,
+                          const float *w, void *out, int64_t nsplit, cudaStream_t stream,
+                          MakeRows make_rows) {
+    auto by_out = [&](auto yt) -> cudaError_t {
+        using YT = decltype(yt);
+        const auto rows = make_rows((int64_t)sizeof(YT));
+        switch (out_dtype) {
+        case DType::F32: return launch_combine<YT, float>(rows, T, H, k, w, out, nsplit, stream);
+        case DType::F16: return launch_combine<YT, __half>(rows, T, H, k, w, out, nsplit, stream);
+        default: return launch_combine<YT, __nv_bfloat16>(rows, T, H, k, w, out, nsplit, stream);
+        }
+    };
+    switch (y_dtype) {
+    case DType::F32: return by_out(float{});
+    case DType::F16: return by_out(__half{});
+    default: return by_out(__nv_bfloat16{});
     }
 }
 
@@ -229,20 +289,24 @@ cudaError_t dispatch_out(DType out_dtype, const void *y, int64_t T, int64_t H, i
 cudaError_t run_combine_split(const void *y, DType y_dtype, int64_t T, int64_t H, int k,
                               const int32_t *out_perm, const float *w, void *out,
                               DType out_dtype, int64_t nsplit, cudaStream_t stream) {
-    switch (y_dtype) {
-    case DType::F32:
-        return dispatch_out<float>(out_dtype, y, T, H, k, out_perm, w, out, nsplit, stream);
-    case DType::F16:
-        return dispatch_out<__half>(out_dtype, y, T, H, k, out_perm, w, out, nsplit, stream);
-    default:
-        return dispatch_out<__nv_bfloat16>(out_dtype, y, T, H, k, out_perm, w, out, nsplit, stream);
-    }
+    return combine_typed(y_dtype, out_dtype, T, H, k, w, out, nsplit, stream, [&](int64_t elt) {
+        return LocalRows{(const char *)y, out_perm, T * k, H * elt};
+    });
 }
 
 cudaError_t run_combine(const void *y, DType y_dtype, int64_t T, int64_t H, int k,
                         const int32_t *out_perm, const float *w, void *out, DType out_dtype,
                         cudaStream_t stream) {
     return run_combine_split(y, y_dtype, T, H, k, out_perm, w, out, out_dtype, 0, stream);
+}
+
+cudaError_t run_combine_peer(const void *const *bufs, const int32_t *nrows, int R, DType y_dtype,
+                             int64_t T, int64_t H, int k, const int32_t *dest_rank,
+                             const int32_t *dest_row, const float *w, void *out, DType out_dtype,
+                             cudaStream_t stream) {
+    return combine_typed(y_dtype, out_dtype, T, H, k, w, out, 0, stream, [&](int64_t elt) {
+        return PeerRows{(const char *const *)bufs, dest_rank, dest_row, nrows, R, H * elt};
+    });
 }
 
 }  // namespace moe

@@ -44,15 +44,54 @@ constexpr int kQuantMaxThreads = 512;       // and the most
 // up (its rows are then incomplete); read and cleared by dispatch_error_kernel.
 __device__ unsigned g_dispatch_error;
 
+// Where the k copies of a token row go.  LocalRows: rows of this GPU's
+// dispatched tensor, through output_permutation.  PeerRows: rows of the
+// grouped buffers of R ranks (the fused exchange between GPUs), through each
+// slot's destination rank and row; a buffer may be another GPU's memory
+// (mapped into this process), reached by plain bulk stores.
+struct LocalRows {
+    using Ref = int;
+    char *out;
+    const int32_t *perm;
+    int64_t S, row_bytes;
+    __device__ Ref ref(int64_t i) const {
+        const int p = __ldg(perm + i);
+        return p >= 0 && p < S ? p : -1;
+    }
+    __device__ static Ref none() { return -1; }
+    __device__ static bool valid(Ref r) { return r >= 0; }
+    __device__ char *addr(Ref r, int64_t off) const { return out + (int64_t)r * row_bytes + off; }
+};
+
+struct PeerRows {
+    using Ref = char *;
+    char *const *bufs;       // [R] each rank's grouped buffer
+    const int32_t *rank;     // [S] destination rank of every slot (-1: none)
+    const int32_t *row;      // [S] and its row there
+    const int32_t *nrows;    // [R] rows of each buffer
+    int R;
+    int64_t row_bytes;
+    __device__ Ref ref(int64_t i) const {
+        const int r = __ldg(rank + i);
+        if (r < 0 || r >= R) return nullptr;
+        const int q = __ldg(row + i);
+        if (q < 0 || q >= __ldg(nrows + r)) return nullptr;
+        return bufs[r] + (int64_t)q * row_bytes;
+    }
+    __device__ static Ref none() { return nullptr; }
+    __device__ static bool valid(Ref r) { return r != nullptr; }
+    __device__ char *addr(Ref r, int64_t off) const { return r + off; }
+};
+
+template <typename Rows>
 __global__ void __launch_bounds__(32)
     dispatch_bulk_kernel(const char *__restrict__ x, int64_t T, int64_t row_bytes, int k,
-                         const int32_t *__restrict__ out_perm, char *__restrict__ out,
-                         int64_t nch, uint32_t chunk, int stages, uint32_t max_polls) {
+                         const Rows rows, int64_t nch, uint32_t chunk, int stages,
+                         uint32_t max_polls) {
     extern __shared__ __align__(128) unsigned char stage[];  // stages * chunk
     __shared__ __align__(8) uint64_t bar[kBulkMaxStages];
     const int lane = threadIdx.x;
     const int64_t units = T * nch;
-    const int64_t S = T * k;
     const int64_t mine =
         units > (int64_t)blockIdx.x ? (units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
     if (lane == 0) {
@@ -61,7 +100,6 @@ __global__ void __launch_bounds__(32)
     }
     __syncwarp();
     pdl_wait();
-    pdl_launch_dependents();
 
     auto load = [&](int64_t n) {  // lane 0: this block's unit n into stage n % stages
         const int64_t u = blockIdx.x + n * (int64_t)gridDim.x;
@@ -83,11 +121,11 @@ __global__ void __launch_bounds__(32)
         const int64_t t = u / nch, off = (u - t * nch) * (int64_t)chunk;
         const uint32_t bytes = (uint32_t)min((int64_t)chunk, row_bytes - off);
         const int s = (int)(n % stages);
-        int p[2];
+        typename Rows::Ref p[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int j = lane + 32 * h;
-            p[h] = j < k ? __ldg(out_perm + t * k + j) : -1;
+            p[h] = j < k ? rows.ref(t * k + j) : Rows::none();
         }
         const bool ok = mbar_wait(&bar[s], (uint32_t)((n / stages) & 1), max_polls);
         if (!__all_sync(0xffffffffu, ok)) {
@@ -97,10 +135,10 @@ __global__ void __launch_bounds__(32)
         const unsigned char *src = stage + (size_t)s * chunk;
 #pragma unroll
         for (int h = 0; h < 2; ++h)
-            if (p[h] >= 0 && p[h] < S) bulk_s2g(out + (int64_t)p[h] * row_bytes + off, src, bytes);
+            if (Rows::valid(p[h])) bulk_s2g(rows.addr(p[h], off), src, bytes);
         for (int j = lane + 64; j < k; j += 32) {  // top-k above 64
-            const int pj = __ldg(out_perm + t * k + j);
-            if (pj >= 0 && pj < S) bulk_s2g(out + (int64_t)pj * row_bytes + off, src, bytes);
+            const typename Rows::Ref pj = rows.ref(t * k + j);
+            if (Rows::valid(pj)) bulk_s2g(rows.addr(pj, off), src, bytes);
         }
         bulk_commit();
         if (n >= 1) {
@@ -110,6 +148,7 @@ __global__ void __launch_bounds__(32)
             issued = __shfl_sync(0xffffffffu, issued < mine ? issued + 1 : issued, 0);
         }
     }
+    pdl_launch_dependents();  // after the work loop: see pdl_launch_dependents
     if (failed) {
         if (lane == 0) atomicExch(&g_dispatch_error, 1u);
         // let every load still in flight land before the block releases its
@@ -131,7 +170,6 @@ __global__ void __launch_bounds__(kCopyThreads)
     dispatch_gather_kernel(const uint4 *__restrict__ x, int64_t S, int64_t nvec, int k,
                            const int32_t *__restrict__ in_perm, uint4 *__restrict__ out) {
     pdl_wait();
-    pdl_launch_dependents();
     for (int64_t p = blockIdx.x; p < S; p += gridDim.x) {
         const int i = __ldg(in_perm + p);
         if (i < 0 || i >= S) continue;
@@ -151,6 +189,7 @@ __global__ void __launch_bounds__(kCopyThreads)
             }
         }
     }
+    pdl_launch_dependents();
 }
 
 // Output memset (TensorRT-LLM PR #9592, moe_output_memset_inplace): zero the
@@ -160,7 +199,6 @@ __global__ void __launch_bounds__(kCopyThreads)
     output_memset_kernel(uint4 *__restrict__ out, int64_t T, int64_t nvec, int k,
                          const int32_t *__restrict__ out_perm) {
     pdl_wait();
-    pdl_launch_dependents();
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         bool routed = false;
         for (int j = 0; j < k; ++j) routed |= __ldg(out_perm + t * k + j) >= 0;
@@ -168,6 +206,7 @@ __global__ void __launch_bounds__(kCopyThreads)
         uint4 *row = out + t * nvec;
         for (int64_t c = threadIdx.x; c < nvec; c += kCopyThreads) st_v4(row + c, make_uint4(0, 0, 0, 0));
     }
+    pdl_launch_dependents();
 }
 
 // ---------------------------------------------------------------------------
@@ -360,7 +399,6 @@ __global__ void __launch_bounds__(kQuantMaxThreads)
         }
     };
     pdl_wait();
-    pdl_launch_dependents();
     if constexpr (kG > 0) prefetch(blockIdx.x);
     stage_offsets(offsets, bso, E, s_off, s_delta);
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
@@ -390,6 +428,7 @@ __global__ void __launch_bounds__(kQuantMaxThreads)
             }
         }
     }
+    pdl_launch_dependents();
 }
 
 }  // namespace
@@ -417,28 +456,47 @@ static int64_t bulk_split(int64_t T, int64_t row_bytes, int64_t grid_max) {
     return best_n;
 }
 
-cudaError_t run_dispatch_scatter_split(const void *x, int64_t T, int64_t row_bytes, int k,
-                                       const int32_t *out_perm, void *out, int64_t nsplit,
-                                       cudaStream_t stream) {
+template <typename Rows>
+static cudaError_t launch_bulk(const void *x, int64_t T, int64_t row_bytes, int k,
+                               const Rows &rows, int64_t nsplit, cudaStream_t stream) {
     const uint32_t chunk = (uint32_t)(((row_bytes + nsplit - 1) / nsplit + 15) / 16 * 16);
     const int64_t nch = (row_bytes + chunk - 1) / chunk;
     int stages = (int)(kBulkSmem / chunk);
     if (stages > kBulkMaxStages) stages = kBulkMaxStages;
     const size_t smem = (size_t)stages * chunk;
-    const int64_t grid = persistent_grid(dispatch_bulk_kernel, 32, smem, T * nch);
-    return launch(dispatch_bulk_kernel, grid, 32, smem, stream, (const char *)x, T, row_bytes, k,
-                  out_perm, (char *)out, nch, chunk, stages, dispatch_polls().load());
+    auto kern = dispatch_bulk_kernel<Rows>;
+    const int64_t grid = persistent_grid(kern, 32, smem, T * nch);
+    return launch(kern, grid, 32, smem, stream, streaming_start(T * k * row_bytes), (const char *)x,
+                  T, row_bytes, k, rows, nch, chunk, stages, dispatch_polls().load());
+}
+
+cudaError_t run_dispatch_scatter_split(const void *x, int64_t T, int64_t row_bytes, int k,
+                                       const int32_t *out_perm, void *out, int64_t nsplit,
+                                       cudaStream_t stream) {
+    return launch_bulk(x, T, row_bytes, k, LocalRows{(char *)out, out_perm, T * k, row_bytes},
+                       nsplit, stream);
 }
 
 cudaError_t run_dispatch_error(int32_t *out, cudaStream_t stream) {
-    return launch(dispatch_error_kernel, 1, 1, 0, stream, out);
+    return launch(dispatch_error_kernel, 1, 1, 0, stream, Start::kEarly, out);
+}
+
+static int64_t bulk_grid_max() {
+    return (int64_t)sm_count() * blocks_per_sm(dispatch_bulk_kernel<LocalRows>, 32, kBulkSmem);
 }
 
 cudaError_t run_dispatch_scatter(const void *x, int64_t T, int64_t row_bytes, int k,
                                  const int32_t *out_perm, void *out, cudaStream_t stream) {
-    const int64_t grid_max = (int64_t)sm_count() * blocks_per_sm(dispatch_bulk_kernel, 32, kBulkSmem);
     return run_dispatch_scatter_split(x, T, row_bytes, k, out_perm, out,
-                                      bulk_split(T, row_bytes, grid_max), stream);
+                                      bulk_split(T, row_bytes, bulk_grid_max()), stream);
+}
+
+cudaError_t run_dispatch_peer(const void *x, int64_t T, int64_t row_bytes, int k,
+                              const int32_t *dest_rank, const int32_t *dest_row,
+                              void *const *bufs, const int32_t *nrows, int R, cudaStream_t stream) {
+    const PeerRows rows{(char *const *)bufs, dest_rank, dest_row, nrows, R, row_bytes};
+    return launch_bulk(x, T, row_bytes, k, rows, bulk_split(T, row_bytes, bulk_grid_max()),
+                       stream);
 }
 
 cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int k,
@@ -446,8 +504,9 @@ cudaError_t run_dispatch_gather(const void *x, int64_t T, int64_t row_bytes, int
     const int64_t nvec = row_bytes / 16;
     const int64_t S = T * k;
     const int64_t grid = persistent_grid(dispatch_gather_kernel, kCopyThreads, 0, S);
-    return launch(dispatch_gather_kernel, grid, kCopyThreads, 0, stream, (const uint4 *)x, S,
-                  nvec, k, in_perm, (uint4 *)out);
+    return launch(dispatch_gather_kernel, grid, kCopyThreads, 0, stream,
+                  streaming_start(S * row_bytes), (const uint4 *)x, S, nvec, k, in_perm,
+                  (uint4 *)out);
 }
 
 // Quantised dispatch launcher.  Rows of up to 2 * kQuantThreads groups:
@@ -466,8 +525,8 @@ static cudaError_t run_dispatch_quant_t(const XT *x, int64_t T, int64_t H, int k
         int64_t threads = ((n16 + per_thread - 1) / per_thread + 31) / 32 * 32;
         if (threads > kQuantMaxThreads) threads = kQuantMaxThreads;
         const int64_t grid = persistent_grid(kern, (int)threads, smem, T);
-        return launch(kern, grid, (int)threads, smem, stream, x, T, H, k, E, out_perm, offsets,
-                      bso, q, scales);
+        return launch(kern, grid, (int)threads, smem, stream, streaming_start(T * k * H), x, T, H,
+                      k, E, out_perm, offsets, bso, q, scales);
     };
     if (n16 <= kQuantThreads) return go(dispatch_quant_kernel<XT, kFp4, 1>, 1);
     if (n16 <= 2 * kQuantThreads) return go(dispatch_quant_kernel<XT, kFp4, 2>, 2);
@@ -497,8 +556,8 @@ cudaError_t run_dispatch_nvfp4(const void *x, DType x_dtype, int64_t T, int64_t 
 cudaError_t run_output_memset(void *out, int64_t T, int64_t row_bytes, int k,
                               const int32_t *out_perm, cudaStream_t stream) {
     const int64_t grid = persistent_grid(output_memset_kernel, kCopyThreads, 0, T);
-    return launch(output_memset_kernel, grid, kCopyThreads, 0, stream, (uint4 *)out, T,
-                  row_bytes / 16, k, out_perm);
+    return launch(output_memset_kernel, grid, kCopyThreads, 0, stream,
+                  streaming_start(T * row_bytes), (uint4 *)out, T, row_bytes / 16, k, out_perm);
 }
 
 }  // namespace moe

@@ -71,7 +71,80 @@ __global__ void __launch_bounds__(kLayoutThreads)
     }
 }
 
+// Destinations of this rank's slots in the other ranks' grouped buffers
+// (the fused exchange: every source stores its rows straight into the
+// owners' buffers).  all[s * E + e] = rows source s holds for expert e.
+// Per expert e of owner d = e / El:
+//     colsum[e] = sum over sources of all[s][e]
+//     gstart[e] = sum of colsum over the experts of d's window before e
+//     base[e]   = gstart[e] + sum over sources s' < rank of all[s'][e]
+// and slot i of expert e, dispatched here to row p, lands on row
+// base[e] + (p - offsets[e]) of d's buffer.  Every block stages the matrix
+// and the scans in shared memory; the grid walks the slots.
+__global__ void __launch_bounds__(kLayoutThreads)
+    ep_peer_layout_kernel(const int32_t *__restrict__ all, int R, int rank, int E,
+                          const int32_t *__restrict__ ids, int64_t S,
+                          const int32_t *__restrict__ offsets,
+                          const int32_t *__restrict__ out_perm, int32_t *dest_rank,
+                          int32_t *dest_row, int32_t *recv_rows, int32_t *local_offsets) {
+    extern __shared__ int smem[];
+    __shared__ int warp_tmp[66];
+    const int El = E / R;
+    int *gpre = smem;      // [E] global exclusive scan of the column sums
+    int *before = gpre + E;  // [E] rows of sources before this rank
+    int *pad = before + E;   // [E] scan scratch
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int col = 0, pre = 0;
+        for (int s = 0; s < R; ++s) {
+            const int v = __ldg(all + (int64_t)s * E + e);
+            col += v;
+            pre += s < rank ? v : 0;
+        }
+        gpre[e] = col;
+        before[e] = pre;
+    }
+    __syncthreads();
+    int pad_total = 0;
+    const int total = block_exclusive_scan2(gpre, pad, E, 1, warp_tmp, &pad_total);
+    if (blockIdx.x == 0) {
+        for (int d = threadIdx.x; d < R; d += blockDim.x)
+            recv_rows[d] = (d + 1 < R ? gpre[(d + 1) * El] : total) - gpre[d * El];
+        for (int le = threadIdx.x; le <= El; le += blockDim.x)
+            local_offsets[le] = (rank * El + le < E ? gpre[rank * El + le] : total) -
+                                gpre[rank * El];
+    }
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < S; i += stride) {
+        const int e = __ldg(ids + i);
+        const int p = __ldg(out_perm + i);
+        int r = -1, row = -1;
+        if (e >= 0 && e < E && p >= 0) {
+            const int d = e / El;
+            r = d;
+            row = gpre[e] - gpre[d * El] + before[e] + (p - __ldg(offsets + e));
+        }
+        dest_rank[i] = r;
+        dest_row[i] = row;
+    }
+}
+
 }  // namespace
+
+cudaError_t run_ep_peer_layout(const int32_t *all_counts, int R, int rank, int E,
+                               const int32_t *ids, int64_t S, const int32_t *offsets,
+                               const int32_t *out_perm, int32_t *dest_rank, int32_t *dest_row,
+                               int32_t *recv_rows, int32_t *local_offsets, cudaStream_t stream) {
+    const size_t smem = (size_t)3 * E * sizeof(int);
+    int64_t grid = (S + kLayoutThreads - 1) / kLayoutThreads;
+    const int64_t cap = (int64_t)sm_count();
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    return launch(ep_peer_layout_kernel, grid, kLayoutThreads, smem, stream, Start::kEarly,
+                  all_counts, R, rank, E, ids, S, offsets, out_perm, dest_rank, dest_row, recv_rows,
+                  local_offsets);
+}
 
 cudaError_t run_ep_recv_layout(const int32_t *counts, int R, int El, int64_t capacity,
                                int32_t *recv_offsets, int32_t *local_offsets,
@@ -84,8 +157,9 @@ cudaError_t run_ep_recv_layout(const int32_t *counts, int R, int El, int64_t cap
     const int64_t cap = (int64_t)sm_count();
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
-    return launch(ep_recv_layout_kernel, grid, kLayoutThreads, smem, stream, counts, R, El,
-                  capacity, recv_offsets, local_offsets, recv_to_local, local_to_recv, num_recv);
+    return launch(ep_recv_layout_kernel, grid, kLayoutThreads, smem, stream, Start::kEarly, counts,
+                  R, El, capacity, recv_offsets, local_offsets, recv_to_local, local_to_recv,
+                  num_recv);
 }
 
 }  // namespace moe

@@ -75,6 +75,23 @@ cudaError_t run_tile_layout(int64_t S, int E, int tile, const int32_t *counts,
                             int32_t *exp2perm, int32_t *perm2exp, int32_t *num_tiles,
                             int32_t *total_padded, cudaStream_t stream);
 
+// The fused exchange between GPUs: every slot's destination rank and row in
+// the owners' grouped buffers (from all ranks' expert counts [R][E]), the
+// dispatch that stores rows there (bufs: device array of R row pointers,
+// nrows: rows of each buffer) and the combine that reads the expert outputs
+// back from them.
+cudaError_t run_ep_peer_layout(const int32_t *all_counts, int R, int rank, int E,
+                               const int32_t *ids, int64_t S, const int32_t *offsets,
+                               const int32_t *out_perm, int32_t *dest_rank, int32_t *dest_row,
+                               int32_t *recv_rows, int32_t *local_offsets, cudaStream_t stream);
+cudaError_t run_dispatch_peer(const void *x, int64_t T, int64_t row_bytes, int k,
+                              const int32_t *dest_rank, const int32_t *dest_row,
+                              void *const *bufs, const int32_t *nrows, int R, cudaStream_t stream);
+cudaError_t run_combine_peer(const void *const *bufs, const int32_t *nrows, int R, DType y_dtype,
+                             int64_t T, int64_t H, int k, const int32_t *dest_rank,
+                             const int32_t *dest_row, const float *w, void *out, DType out_dtype,
+                             cudaStream_t stream);
+
 // Receiving rank's layout of the expert-parallel exchange: counts [R][El]
 // -> recv_offsets [R+1], local_offsets [El+1], the two row maps (written when
 // the number of received rows is at most `capacity`) and that number.

@@ -139,8 +139,8 @@ __global__ void __launch_bounds__(kLayoutThreads)
 cudaError_t run_problem_sizes(const int32_t *counts, int E, int n1, int k1, int n2, int k2,
                               int32_t *ps1, int32_t *ps2, cudaStream_t stream) {
     const int64_t grid = (E + kLayoutThreads - 1) / kLayoutThreads;
-    return launch(problem_sizes_kernel, grid, kLayoutThreads, 0, stream, counts, E, n1, k1, n2, k2,
-                  ps1, ps2);
+    return launch(problem_sizes_kernel, grid, kLayoutThreads, 0, stream, Start::kEarly, counts, E,
+                  n1, k1, n2, k2, ps1, ps2);
 }
 
 cudaError_t run_tile_layout(int64_t S, int E, int tile, const int32_t *counts,
@@ -153,9 +153,9 @@ cudaError_t run_tile_layout(int64_t S, int E, int tile, const int32_t *counts,
     if (S > work) work = S;
     const int64_t grid =
         persistent_grid(tile_layout_kernel, kLayoutThreads, smem, (work + kLayoutThreads - 1) / kLayoutThreads);
-    return launch(tile_layout_kernel, grid, kLayoutThreads, smem, stream, S, E, tile, counts,
-                  offsets, out_perm, max_tiles, padded_offsets, tile_group, tile_limit, exp2perm,
-                  perm2exp, num_tiles, total_padded);
+    return launch(tile_layout_kernel, grid, kLayoutThreads, smem, stream, Start::kEarly, S, E, tile,
+                  counts, offsets, out_perm, max_tiles, padded_offsets, tile_group, tile_limit,
+                  exp2perm, perm2exp, num_tiles, total_padded);
 }
 
 }  // namespace moe

@@ -13,7 +13,13 @@ constexpr int kWarp = 32;
 // ---------------------------------------------------------------------------
 // Programmatic dependent launch (PTX griddepcontrol, sm_90+).  Every kernel
 // waits for its stream predecessor before touching global memory the
-// predecessor may write or read, and lets its own dependents launch early.
+// predecessor may write or read, and lets its dependents launch before it
+// ends: the short kernels (prepare, layouts) at their start, the streaming
+// ones (dispatch, combine, gathers, memset) only after their work loop.
+// Measured on B200: with the early signal, the next kernel's blocks sit on
+// the SMs for the whole of a long streaming kernel and slowed the large
+// workload's step by about 80 us in 1.3 ms; signalled after the loop, the
+// next launch still overlaps the tail.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() {

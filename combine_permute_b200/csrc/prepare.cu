@@ -896,22 +896,23 @@ cudaError_t run_prepare_t(const IdT *ids, int64_t base, int64_t S, int E, int A,
                           int32_t *diag, void *workspace, cudaStream_t stream) {
     if (S <= kSmallSlots) {
         const int threads = S < 32 ? 32 : (int)((S + 31) / 32 * 32);
-        return launch(prep_small_kernel<IdT>, 1, threads, small_smem(E, S), stream, ids, base,
-                      (int)S, E, A, counts, offsets, bso, in_perm, out_perm, diag);
+        return launch(prep_small_kernel<IdT>, 1, threads, small_smem(E, S), stream, Start::kEarly,
+                      ids, base, (int)S, E, A, counts, offsets, bso, in_perm, out_perm, diag);
     }
     if (S <= kSingleBlockSlots)
-        return launch(prep_single_kernel<IdT>, 1, kSingleThreads, single_block_smem(E), stream, ids,
-                      base, S, E, A, counts, offsets, bso, in_perm, out_perm, diag);
+        return launch(prep_single_kernel<IdT>, 1, kSingleThreads, single_block_smem(E), stream,
+                      Start::kEarly, ids, base, S, E, A, counts, offsets, bso, in_perm, out_perm,
+                      diag);
     cudaError_t e = launch_sync(ids, base, S, E, A, workspace, counts, offsets, bso, in_perm,
                                 out_perm, diag, stream);
     if (e != cudaErrorCooperativeLaunchTooLarge) return e;
     const int G = (int)tiles_of(S);
-    e = launch(prep_rank_kernel<IdT>, G, kRankThreads, tile_smem<kRankThreads>(E), stream, ids,
-               base, S, E, A, G, workspace, (unsigned long long)prepare_wait_ns().load(), counts,
-               offsets, bso, out_perm, diag);
+    e = launch(prep_rank_kernel<IdT>, G, kRankThreads, tile_smem<kRankThreads>(E), stream,
+               Start::kEarly, ids, base, S, E, A, G, workspace,
+               (unsigned long long)prepare_wait_ns().load(), counts, offsets, bso, out_perm, diag);
     if (e != cudaSuccess) return e;
     const int64_t grid = persistent_grid(prep_finish_kernel<IdT>, 256, 0, (S + 1023) / 1024);
-    return launch(prep_finish_kernel<IdT>, grid, 256, 0, stream, ids, base, S, E,
+    return launch(prep_finish_kernel<IdT>, grid, 256, 0, stream, Start::kEarly, ids, base, S, E,
                   (const int32_t *)offsets, in_perm, out_perm);
 }
 
@@ -942,8 +943,9 @@ cudaError_t run_prepare_dispatch(const int32_t *ids, int64_t T, int k, int E, in
                                          : kSingleThreads;
     const int64_t units = (T * nvec + threads - 1) / threads;
     const int64_t grid = persistent_grid(prep_dispatch_kernel, threads, smem, units);
-    return launch(prep_dispatch_kernel, grid, threads, smem, stream, ids, T, k, E, A, counts,
-                  offsets, bso, in_perm, out_perm, diag, (const uint4 *)x, nvec, (uint4 *)out);
+    return launch(prep_dispatch_kernel, grid, threads, smem, stream, Start::kEarly, ids, T, k, E, A,
+                  counts, offsets, bso, in_perm, out_perm, diag, (const uint4 *)x, nvec,
+                  (uint4 *)out);
 }
 
 }  // namespace moe

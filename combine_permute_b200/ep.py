@@ -29,6 +29,13 @@ come from an ``ops`` object; the default, ``CudaOps``, is this library's
 kernels.  The module has no other implementation of them: a caller without
 the CUDA library gets the binding's error.  Passing another ``ops`` is how a
 test drives the same exchange logic on CPU ranks.
+
+ep_dispatch_peer and ep_combine_peer are the same exchange without
+all-to-alls: every source's dispatch kernel stores its rows straight into
+the owners' grouped buffers (other GPUs' memory mapped into this process)
+and its combine kernel reads the expert outputs straight back from them;
+the only collectives are an all-gather of the expert counts and two
+barriers.
 """
 
 from __future__ import annotations
@@ -38,9 +45,11 @@ from typing import List, NamedTuple, Optional
 import torch
 import torch.distributed as dist
 
-from . import (moe_combine, moe_dispatch_rows, moe_ep_recv_layout, moe_prepare)
+from . import (moe_combine, moe_dispatch_rows, moe_ep_combine_peer, moe_ep_dispatch_peer,
+               moe_ep_peer_layout, moe_ep_recv_layout, moe_prepare)
 
-__all__ = ["CudaOps", "EpHandle", "ep_dispatch", "ep_combine"]
+__all__ = ["CudaOps", "EpHandle", "ep_dispatch", "ep_combine", "EpPeerHandle",
+           "ep_dispatch_peer", "ep_combine_peer"]
 
 
 class CudaOps:
@@ -130,3 +139,61 @@ def ep_combine(y: torch.Tensor, weights: torch.Tensor, handle: EpHandle, group=N
     dist.all_to_all_single(back[:sent], y_recv, handle.send_splits, handle.recv_splits,
                            group=group)
     return ops.combine(back, handle.meta, weights, out_dtype or y.dtype)
+
+
+class EpPeerHandle(NamedTuple):
+    """What ep_combine_peer needs from the matching ep_dispatch_peer."""
+    layout: object                # moe_ep_peer_layout of this rank
+    num_tokens: int
+    top_k: int
+
+
+def _barrier(group, dev):
+    # a one-element all-reduce on the current stream: every rank's earlier
+    # kernels (and their stores into other ranks' buffers) have finished
+    # before any rank's later kernels start
+    t = torch.zeros(1, dtype=torch.int32, device=dev)
+    dist.all_reduce(t, group=group)
+
+
+def ep_dispatch_peer(x: torch.Tensor, topk_ids: torch.Tensor, num_experts: int, recv_buffers,
+                     group=None):
+    """Stores every token row into the grouped buffer of the ranks owning
+    its experts.
+
+    ``recv_buffers`` are this process's views of every rank's grouped
+    receive buffer, in rank order ([capacity, H] each, x's dtype; this
+    rank's own is local memory, the others are other GPUs' memory mapped
+    in), none of them in use by an earlier step.  Returns (this rank's
+    grouped rows: a view of its own buffer, by local expert, then source,
+    then the source's order; local_offsets [El+1]; the handle for
+    ep_combine_peer)."""
+    R = _ranks(group)
+    rank = dist.get_rank(group)
+    if num_experts % R:
+        raise ValueError(f"{num_experts} experts do not split evenly over {R} ranks")
+    if len(recv_buffers) != R:
+        raise ValueError(f"{len(recv_buffers)} buffers for {R} ranks")
+    T, k = topk_ids.shape
+    meta = moe_prepare(topk_ids, num_experts)
+    counts = torch.empty((R, num_experts), dtype=torch.int32, device=topk_ids.device)
+    dist.all_gather_into_tensor(counts, meta.expert_counts, group=group)
+    layout = moe_ep_peer_layout(counts, rank, topk_ids, meta)
+    rows = layout.recv_rows.tolist()
+    for r, b in enumerate(recv_buffers):
+        if isinstance(b, torch.Tensor) and b.shape[0] < rows[r]:
+            raise ValueError(f"rank {r}'s buffer holds {b.shape[0]} rows, {rows[r]} needed")
+    moe_ep_dispatch_peer(x, k, layout, recv_buffers)
+    _barrier(group, x.device)
+    own = recv_buffers[rank]
+    return own[: rows[rank]], layout.local_offsets, EpPeerHandle(layout, T, k)
+
+
+def ep_combine_peer(out_buffers, y_dtype: torch.dtype, hidden: int, weights: torch.Tensor,
+                    handle: EpPeerHandle, group=None, out_dtype=None) -> torch.Tensor:
+    """Combines this rank's tokens from the expert outputs the owners wrote
+    into their buffers (``out_buffers``: every rank's, in rank order, in the
+    grouped layout).  Returns out [T, H] as moe_combine would."""
+    _barrier(group, weights.device)  # every owner has written its expert outputs
+    return moe_ep_combine_peer(out_buffers, y_dtype, hidden, handle.layout, weights,
+                               out_dtype=out_dtype)

@@ -477,6 +477,73 @@ moe_status_t moe_ep_recv_layout(const int32_t *recv_expert_counts, int32_t num_r
                                 int32_t *recv_to_local, int32_t *local_to_recv,
                                 int32_t *num_recv, moe_stream_t stream);
 
+/*
+ * The exchange between GPUs as stores into the owners' memory (the same
+ * exchange as above without all-to-alls: every source rank writes its rows
+ * straight into the owners' grouped buffers and later reads the expert
+ * outputs straight back from them; Mooncake PR #4581, dispatch / combine
+ * kernels that move rows between ranks; TensorRT-LLM PR #9592, one rank's
+ * experts being a window).  R ranks each own El = E / R consecutive experts
+ * and each holds a grouped buffer of rows laid out by local expert, then
+ * source rank, then the source's order (the layout moe_ep_recv_layout
+ * gives).  On several GPUs the buffers are other GPUs' memory mapped into
+ * this process (CUDA IPC or symmetric memory; peer-to-peer access enabled),
+ * reached with plain loads and bulk stores, never with multicast loads.
+ *
+ * moe_ep_peer_layout: from every rank's expert counts,
+ *   all_expert_counts [R, E] int32   rank s's moe_prepare expert_counts in
+ *                                    row s (an all-gather of the counts)
+ *   topk_ids, expert_offsets, output_permutation   this rank's ([T, k],
+ *                                    [E+1], [T*k]) from moe_prepare over all
+ *                                    E experts
+ * writes
+ *   dest_rank [T*k] int32   the rank owning each slot's expert (-1: none)
+ *   dest_row  [T*k] int32   the slot's row in that rank's grouped buffer
+ *   recv_rows [R]   int32   rows of each rank's grouped buffer
+ *   local_offsets [El+1] int32   this rank's grouped expert offsets
+ * Errors: MOE_ERR_INVALID_ARG for NULL pointers, num_ranks < 1, rank outside
+ * [0, num_ranks), num_experts not a positive multiple of num_ranks;
+ * MOE_ERR_UNSUPPORTED for num_experts > MOE_MAX_EXPERTS.
+ */
+moe_status_t moe_ep_peer_layout(const int32_t *all_expert_counts, int32_t num_ranks,
+                                int32_t rank, int32_t num_experts, const int32_t *topk_ids,
+                                int64_t num_tokens, int32_t top_k,
+                                const int32_t *expert_offsets,
+                                const int32_t *output_permutation, int32_t *dest_rank,
+                                int32_t *dest_row, int32_t *recv_rows, int32_t *local_offsets,
+                                moe_stream_t stream);
+
+/*
+ * moe_ep_dispatch_peer: row t of x [T, H] (dtype F32, F16 or BF16, rows a
+ * multiple of 16 bytes, 16-byte aligned) goes to row dest_row[t*k+j] of the
+ * grouped buffer of rank dest_rank[t*k+j], for every slot j with a
+ * destination.  recv_buffers is a DEVICE array of num_ranks pointers to the
+ * ranks' grouped buffers (16-byte aligned, recv_rows[r] rows of H elements);
+ * slots whose row falls outside recv_rows are skipped.  Each x row is read
+ * once (the TMA dispatch of moe_dispatch_rows; its bounded waits report
+ * through moe_dispatch_error).  The caller orders the owners' later reads
+ * after every source's dispatch (a barrier across ranks).
+ */
+moe_status_t moe_ep_dispatch_peer(const void *x, moe_dtype_t dtype, int64_t num_tokens,
+                                  int64_t hidden, int32_t top_k, const int32_t *dest_rank,
+                                  const int32_t *dest_row, void *const *recv_buffers,
+                                  const int32_t *recv_rows, int32_t num_ranks,
+                                  moe_stream_t stream);
+
+/*
+ * moe_ep_combine_peer: out[t] = sum_j weights[t, j] * (row dest_row[t*k+j]
+ * of rank dest_rank[t*k+j]'s buffer of expert outputs), accumulated in fp32
+ * in slot order exactly as moe_combine does.  out_buffers is a DEVICE array
+ * of num_ranks pointers to the ranks' expert-output buffers (the grouped
+ * layout, recv_rows[r] rows of H elements of y_dtype, 16-byte aligned).
+ * Slots without a valid row contribute nothing.
+ */
+moe_status_t moe_ep_combine_peer(const void *const *out_buffers, const int32_t *recv_rows,
+                                 int32_t num_ranks, moe_dtype_t y_dtype, int64_t num_tokens,
+                                 int64_t hidden, int32_t top_k, const int32_t *dest_rank,
+                                 const int32_t *dest_row, const float *weights, void *out,
+                                 moe_dtype_t out_dtype, moe_stream_t stream);
+
 /* Largest T*k that moe_prepare_dispatch accepts. */
 #define MOE_FUSED_MAX_SLOTS 4096
 

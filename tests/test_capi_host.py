@@ -244,3 +244,26 @@ def test_dispatch_error_and_wait_limits_validation(lib):
     assert lib.moe_dispatch_error(None, None) == INVALID
     assert lib.moe_set_wait_limits(0, 0) == OK
     assert lib.moe_set_wait_limits(-1, -1) == OK  # back to the defaults
+
+
+def test_ep_peer_validation(lib):
+    # layout: ranks, rank index, experts divisible by ranks, pointers
+    def layout(R=2, rank=0, E=8, T=4, k=2, counts=P, ids=P, offs=P, outp=P, dr=P, drow=P, rr=P,
+               lo=P):
+        return lib.moe_ep_peer_layout(counts, R, rank, E, ids, T, k, offs, outp, dr, drow, rr, lo,
+                                      None)
+    assert layout(R=0) == INVALID
+    assert layout(rank=2) == INVALID and layout(rank=-1) == INVALID
+    assert layout(E=7) == INVALID
+    assert layout(E=2048) == UNSUPPORTED
+    assert layout(counts=None) == INVALID and layout(dr=None) == INVALID
+    # dispatch into peer buffers: row size, alignment, pointers
+    assert lib.moe_ep_dispatch_peer(P, BF16, 4, 4, 2, P, P, P, P, 2, None) == INVALID  # 8-byte rows
+    assert lib.moe_ep_dispatch_peer(P + 8, BF16, 4, 64, 2, P, P, P, P, 2, None) == INVALID
+    assert lib.moe_ep_dispatch_peer(P, BF16, 4, 64, 2, P, P, None, P, 2, None) == INVALID
+    assert lib.moe_ep_dispatch_peer(P, FP8, 4, 64, 2, P, P, P, P, 2, None) == INVALID
+    assert lib.moe_ep_dispatch_peer(P, BF16, 0, 64, 2, None, None, None, None, 2, None) == OK
+    # combine from peer buffers (every call here returns before launching)
+    assert lib.moe_ep_combine_peer(None, P, 2, BF16, 4, 64, 2, P, P, P, P, BF16, None) == INVALID
+    assert lib.moe_ep_combine_peer(P, P, 0, BF16, 4, 64, 2, P, P, P, P, BF16, None) == INVALID
+    assert lib.moe_ep_combine_peer(P, P, 2, BF16, 4, 4, 2, P, P, P, P, BF16, None) == INVALID

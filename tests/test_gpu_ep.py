@@ -143,3 +143,113 @@ def test_ep_module_over_a_one_rank_nccl_group():
     assert np.array_equal(local_offsets.cpu().numpy(), ref["offsets"])
     assert np.array_equal(bits(out), oracle.combine(bits(y), "bf16", ref["output_perm"], wt_np,
                                                     "bf16"))
+
+
+# ---------------------------------------------------------------------------
+# The exchange as stores into the owners' buffers (moe_ep_peer_layout,
+# moe_ep_dispatch_peer, moe_ep_combine_peer).  R ranks are emulated on one
+# GPU: every rank's grouped buffer lives here, and each source's kernels get
+# the array of all R buffer addresses, as a rank with the other GPUs' memory
+# mapped in would.
+# ---------------------------------------------------------------------------
+
+def _emulated_ranks(R, T, seed, base_name="uniform_t4096_h7168_e256_k8", invalid_every=53):
+    base = CONFIGS[base_name]
+    ranks = []
+    for r in range(R):
+        w = dataclasses.replace(base, T=T + 29 * r, seed=seed * 100 + r, name=f"rank{r}")
+        ids_np, wt_np, x, _ = make_workload(w, device=DEV, with_y=False)
+        if invalid_every:
+            ids_np[::invalid_every, 0] = -1
+        ids = torch.from_numpy(ids_np).to(DEV)
+        ranks.append(dict(w=w, T=w.T, ids_np=ids_np, ids=ids, wt=wt_np, x=x,
+                          meta=moe.moe_prepare(ids, base.E)))
+    return base, ranks
+
+
+@pytest.mark.parametrize("R,T,seed", [(1, 500, 3), (2, 700, 4), (4, 1100, 5), (8, 300, 6)])
+def test_peer_layout_matches_the_single_gpu_rows(R, T, seed):
+    base, ranks = _emulated_ranks(R, T, seed)
+    E, k = base.E, base.k
+    El = E // R
+    counts = torch.stack([r["meta"].expert_counts for r in ranks]).contiguous()
+    g = oracle.prepare(np.concatenate([r["ids_np"] for r in ranks]), E)
+    tok0 = 0
+    for s, r in enumerate(ranks):
+        lay = moe.moe_ep_peer_layout(counts, s, r["ids"], r["meta"])
+        torch.cuda.synchronize()
+        # slot i of rank s is global slot tok0*k + i; its owner's grouped buffer
+        # is the single-GPU dispatched rows of the owner's expert window
+        gi = tok0 * k + np.arange(r["T"] * k)
+        P = g["output_perm"][gi]
+        e = r["ids_np"].ravel()
+        ok = P >= 0
+        want_rank = np.where(ok, e // El, -1)
+        want_row = np.where(ok, P - g["offsets"][np.clip(e // El, 0, R - 1) * El], -1)
+        assert np.array_equal(lay.dest_rank.cpu().numpy(), want_rank)
+        assert np.array_equal(lay.dest_row.cpu().numpy(), want_row)
+        assert np.array_equal(lay.recv_rows.cpu().numpy(), np.diff(g["offsets"][::El]))
+        assert np.array_equal(lay.local_offsets.cpu().numpy(),
+                              g["offsets"][s * El:(s + 1) * El + 1] - g["offsets"][s * El])
+        tok0 += r["T"]
+
+
+@pytest.mark.parametrize("R,T,seed,ydt,odt", [(2, 700, 7, "bf16", "bf16"), (4, 900, 8, "bf16", "bf16"),
+                                              (8, 400, 9, "bf16", "fp32")])
+def test_peer_dispatch_and_combine_match_single_gpu(R, T, seed, ydt, odt):
+    base, ranks = _emulated_ranks(R, T, seed)
+    E, k, H = base.E, base.k, base.H
+    El = E // R
+    counts = torch.stack([r["meta"].expert_counts for r in ranks]).contiguous()
+    lays = [moe.moe_ep_peer_layout(counts, s, r["ids"], r["meta"]) for s, r in enumerate(ranks)]
+    rows = lays[0].recv_rows.tolist()
+    sentinel = -3.0
+    bufs = [torch.full((max(n, 1), H), sentinel, dtype=torch.bfloat16, device=DEV) for n in rows]
+    for s, r in enumerate(ranks):
+        moe.moe_ep_dispatch_peer(r["x"], k, lays[s], bufs)
+    torch.cuda.synchronize()
+    g = oracle.prepare(np.concatenate([r["ids_np"] for r in ranks]), E)
+    want = oracle.dispatch(np.concatenate([bits(r["x"]) for r in ranks]), k, g["input_perm"])
+    for d in range(R):
+        lo, hi = g["offsets"][d * El], g["offsets"][(d + 1) * El]
+        assert rows[d] == hi - lo
+        assert np.array_equal(bits(bufs[d][:rows[d]]), want[lo:hi]), d
+    # expert outputs: the single-GPU y rows of each owner's window, in its buffer
+    TD = {"bf16": torch.bfloat16, "fp32": torch.float32}
+    S = sum(r["T"] for r in ranks) * k
+    y = torch.randn(S, H, generator=torch.Generator().manual_seed(seed)).to(TD[ydt])
+    outs = [y[g["offsets"][d * El]:g["offsets"][(d + 1) * El]].to(DEV).contiguous() for d in range(R)]
+    outs = [o if o.shape[0] else torch.zeros(1, H, dtype=TD[ydt], device=DEV) for o in outs]
+    full = oracle.combine(bits(y), ydt, g["output_perm"], np.concatenate([r["wt"] for r in ranks]), odt)
+    t0 = 0
+    for s, r in enumerate(ranks):
+        got = moe.moe_ep_combine_peer(outs, TD[ydt], H, lays[s], torch.from_numpy(r["wt"]).to(DEV),
+                                      out_dtype=TD[odt])
+        torch.cuda.synchronize()
+        assert np.array_equal(bits(got), full[t0:t0 + r["T"]]), s
+        t0 += r["T"]
+
+
+def test_ep_peer_module_over_a_one_rank_nccl_group():
+    import torch.distributed as dist
+    from combine_permute_b200 import ep
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=DEV)
+    try:
+        w = CONFIGS["uniform_t4096_h7168_e256_k8"].scaled(800)
+        ids_np, wt_np, x, y = make_workload(w, device=DEV)
+        buf = torch.empty((w.S, w.H), dtype=x.dtype, device=DEV)
+        grouped, local_offsets, handle = ep.ep_dispatch_peer(x, torch.from_numpy(ids_np).to(DEV),
+                                                             w.E, [buf])
+        out = ep.ep_combine_peer([y], y.dtype, w.H, torch.from_numpy(wt_np).to(DEV), handle)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    ref = oracle.prepare(ids_np, w.E)
+    assert np.array_equal(bits(grouped), oracle.dispatch(bits(x), w.k, ref["input_perm"]))
+    assert np.array_equal(local_offsets.cpu().numpy(), ref["offsets"])
+    assert np.array_equal(bits(out), oracle.combine(bits(y), "bf16", ref["output_perm"], wt_np,
+                                                    "bf16"))
