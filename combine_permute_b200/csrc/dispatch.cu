@@ -433,10 +433,21 @@ __global__ void __launch_bounds__(kQuantMaxThreads)
 
 }  // namespace
 
-// Row split for the bulk dispatch: the number of chunks per row that
-// minimises (units per block) x (bytes per unit + a per-unit overhead), the
-// makespan of a persistent grid of `grid_max` blocks.
+// Row split for the bulk dispatch.  When the batch fills the persistent
+// grid, chunks of about kBulkChunkTarget bytes (16 stages in the ring):
+// measured on B200, 14336-byte rows ran at 0.757 of 8 TB/s cut in four
+// (3584-byte chunks) against 0.694-0.705 whole or cut in two, three or
+// seven, and 4096-byte rows were best whole.  Otherwise (few tokens) the
+// number of chunks per row that minimises (units per block) x (bytes per
+// unit + a per-unit overhead), the makespan of a persistent grid of
+// `grid_max` blocks.
+constexpr int64_t kBulkChunkTarget = 4096;
+
 static int64_t bulk_split(int64_t T, int64_t row_bytes, int64_t grid_max) {
+    int64_t target = (row_bytes + kBulkChunkTarget / 2) / kBulkChunkTarget;
+    if (target < 1) target = 1;
+    if (target > 16) target = 16;
+    if (T * target >= grid_max) return target;
     constexpr int64_t kUnitOverheadBytes = 1024;
     int64_t best_n = 1, best_cost = -1;
     for (int64_t n = 1; n <= 16; ++n) {
