@@ -690,13 +690,12 @@ def run_gpu(args, names, workloads=None):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": _dtype_tag(w),
         "data": "synthetic",
-        "config": dict(_config(w, world), launch=r["launch"]),
+        "config": _config(w, world),
     }
-    line.update({k: v for k, v in r.items() if k not in ("value", "ms_per_step", "launch")})
+    line.update({k: v for k, v in r.items() if k not in ("value", "ms_per_step")})
     if len(names) > 1:
         line["per_workload"] = {
-            n: dict(results[n], config=dict(_config(workloads[n], world), launch=results[n]["launch"]),
-                    dtype=_dtype_tag(workloads[n]))
+            n: dict(results[n], config=_config(workloads[n], world), dtype=_dtype_tag(workloads[n]))
             for n in names[1:]}
     print(json.dumps(line), flush=True)
 
