@@ -487,3 +487,20 @@ def test_chained_step_on_one_stream():
     np.testing.assert_array_equal(meta.output_permutation.cpu().numpy(), ref["output_perm"])
     np.testing.assert_array_equal(bits(xd), oracle.dispatch(bits(x), w.k, ref["input_perm"]))
     _combine_check(y, ref["output_perm"], wt_np, "bf16", out)
+
+
+@pytest.mark.parametrize("S,E", [
+    (4097, 511),            # one-launch path, widest expert range it takes (E + 1 = 512)
+    (4097, 512),            # one expert more: the two-kernel path
+    (32768, 511),           # 2 rounds, 32 blocks
+    (65536, 255),           # last size at 2 rounds (64 rows of 256 staged counts)
+    (65537, 255),           # first at 3 rounds
+    (1212416, 64),          # the largest one-launch problem on 148 SMs (16 rounds)
+    (1212417, 64),          # one slot more: the two-kernel path
+])
+def test_prepare_path_boundaries(S, E):
+    """Sizes on each side of the rules that pick the prepare path and the
+    one-launch path's rounds, with k = 1 (S tokens) and 2 % invalid ids."""
+    rng = np.random.default_rng(S + E)
+    ids = _ids_random(rng, S, 1, E, p_invalid=0.02, distinct=False)
+    _check_prepare(ids, E, A=8)
