@@ -72,24 +72,24 @@ __device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned *p) {
     return v;
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
 // Atomic add with acquire-release semantics at GPU scope; returns the old value.
-__device__ __forceinline__ unsigned long long atom_add_acq_rel_u64(unsigned long long *p,
-                                                                  unsigned long long v) {
-    unsigned long long old;
-    asm volatile("atom.acq_rel.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v)
+__device__ __forceinline__ unsigned atom_add_acq_rel_u32(unsigned *p, unsigned v) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
                  : "memory");
     return old;
 }
 
 // Atomic add with release semantics at GPU scope, no result.
-__device__ __forceinline__ void red_add_release_u64(unsigned long long *p, unsigned long long v) {
-    asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+__device__ __forceinline__ void red_add_release_u32(unsigned *p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// A hint to bring the 128-byte line holding p into L2; it returns nothing
+// and orders nothing, so it may run before the wait on the producing grid
+// (L2 is where every SM's writes meet, so a later write updates the line).
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // Wrapping increment (atomicInc semantics) with acquire-release semantics.

@@ -13,20 +13,22 @@
 //    rank counted directly over the earlier slots (prep_small_kernel);
 //  * up to kSingleBlockSlots slots: one block does it all
 //    (prep_single_kernel);
-//  * above that, tiles of kTileSlots slots, each ranked by one block, which
-//    publishes its per-expert histogram and runs a decoupled look-back over
-//    the earlier tiles' (bounded waits, a window of predecessors read
-//    together); the last tile holds the totals and writes counts and
-//    offsets.  When every tile fits on the GPU at once this is one
-//    cooperative launch (prep_onepass_kernel, 512-thread tiles, tile =
-//    block index): the other tiles wait, bounded, for the last one's offsets
-//    and write both permutations.  Otherwise prep_rank_kernel (256-thread
-//    tiles, two per SM) takes tiles by an atomic ticket, so a tile only ever
-//    waits on tiles already running, and stores rank(i) in
-//    output_permutation; the element-wise prep_finish_kernel then adds the
-//    expert offset and writes both permutations.  A wait that gives up
-//    reports through diag[1].  Words in the workspace carry the epoch of the
-//    call that wrote them, so the workspace needs zeroing once, not per call.
+//  * above that, when every block fits on the GPU at once: one cooperative
+//    launch (prep_sync_kernel, 512-thread blocks of 2 to 16 rounds).  Each
+//    block ranks its slots, publishes its per-expert histogram row and meets
+//    the others at a grid barrier (bounded wait); every block then stages
+//    all rows, scans them into the expert offsets and its own prefix, and
+//    writes both permutations for its slots;
+//  * otherwise two kernels: prep_rank_kernel takes tiles of kTileSlots slots
+//    by an atomic ticket (so a tile only ever waits on tiles already
+//    running), publishes each tile's histogram and runs a decoupled
+//    look-back over the earlier tiles' (bounded waits, a window of
+//    predecessors read together); the last tile holds the totals and writes
+//    counts and offsets, and every slot's rank(i) goes to output_permutation.
+//    The element-wise prep_finish_kernel then adds the expert offset and
+//    writes both permutations.  Look-back words carry the epoch of the call
+//    that wrote them, so the workspace needs zeroing once, not per call.
+// A wait that gives up reports through diag[1].
 #include "kernels.h"
 #include "launch.h"
 #include "moe_device.cuh"
@@ -149,14 +151,15 @@ __host__ __device__ inline size_t align256(size_t b) { return (b + 255) & ~size_
 
 // Workspace of the tiled paths, in three fixed parts: a 256-byte header
 // (counters), the one-launch path's histogram rows (a fixed kSyncHistBytes,
-// int32 rows of E+1 counts, one per block), then one 64-bit look-back word
+// one row of E+1 16-bit counts per block), then one 64-bit look-back word
 // per (tile, expert column) of the two-kernel path.  The parts never move
 // with the problem size, so no call reads another path's data as its own.
 // A look-back word holds epoch << 34 | flag << 32 | value; it counts as
 // published by this call only when its epoch field is this call's epoch, so
 // words left by earlier calls need no clearing.  The epoch advances once per
 // two-kernel call (by its last block); the ticket, done and barrier-arrival
-// counters return to zero at the end of every call.  The histogram rows are
+// counters return to zero at the end of every call (the last block to
+// finish clears them, once every block is past its waits).  The histogram rows are
 // written before the grid barrier and read after it, so they need no
 // clearing either.
 struct PrepWs {
@@ -164,16 +167,21 @@ struct PrepWs {
     unsigned *done;       // blocks finished, wraps at G
     unsigned *epoch;      // this call's epoch
     unsigned *timeout;    // set when a bounded wait gave up
-    unsigned long long *bar;    // one-launch path: generation << 32 | blocks arrived
-    int *hist;                  // [G][E+1] histogram rows of the one-launch path
+    unsigned *arrive;           // one-launch path: blocks arrived at the grid barrier
+    unsigned short *hist;       // [G][sync_stride(E)] histogram rows, one-launch path
     unsigned long long *state;  // [G][E+1] look-back words of the two-kernel path
 };
 
 // Most blocks of one one-launch prepare (one block per SM on B200, with room
-// for parts with more SMs) and, with at most kSyncThreads columns a row, the
-// fixed size of its histogram rows.
+// for parts with more SMs) and the fixed size of its histogram rows.  A row
+// holds E+1 counts of at most kSyncMaxRounds * kSyncThreads = 8192 slots,
+// so 16 bits each, padded to a multiple of 8 (16 bytes) so that rows are
+// staged with 16-byte loads; at most kSyncThreads columns.  The region keeps
+// room for 32-bit counts (512 KB), so that the workspace layout and size do
+// not depend on the width of a count.
 constexpr int kMaxSyncTiles = 256;
 constexpr size_t kSyncHistBytes = (size_t)kMaxSyncTiles * 512 * sizeof(int);
+__host__ __device__ inline int sync_stride(int E) { return (E + 1 + 7) & ~7; }
 
 __host__ __device__ inline int64_t tiles_of(int64_t S) { return (S + kTileSlots - 1) / kTileSlots; }
 
@@ -184,8 +192,8 @@ __host__ __device__ inline PrepWs carve(void *ws) {
     w.done = (unsigned *)(b + 4);
     w.epoch = (unsigned *)(b + 8);
     w.timeout = (unsigned *)(b + 16);
-    w.bar = (unsigned long long *)(b + 24);
-    w.hist = (int *)(b + 256);
+    w.arrive = (unsigned *)(b + 24);
+    w.hist = (unsigned short *)(b + 256);
     w.state = (unsigned long long *)(b + 256 + kSyncHistBytes);
     return w;
 }
@@ -498,29 +506,32 @@ constexpr int kSyncThreads = 512;                  // one-launch tiles: 16 warps
 static_assert(kSyncThreads <= 512, "a histogram row of the one-launch path fits kSyncHistBytes");
 constexpr int kSyncMaxRounds = 16;                 // of up to 16 rounds (8192 slots)
 constexpr int kSyncMinRounds = 4;
+static_assert(kSyncMaxRounds * kSyncThreads <= 65535, "a block's count of one expert fits 16 bits");
 
 // Shared memory of the two-kernel tiles: per-warp rows, then hist, excl,
 // off, pad (one column per expert plus one for invalid ids each).
 template <int NT> size_t tile_smem(int E) { return (size_t)(NT / 32 + 4) * (E + 1) * sizeof(int); }
 
 // One-launch prepare (a cooperative launch: every block resident, so blocks
-// may wait on one another; E + 1 <= kSyncThreads).  Block b ranks slots
-// [b*nr*NT, (b+1)*nr*NT) within each warp's run, folds the warps into its
-// histogram row, publishes the row and arrives at a grid barrier (one 64-bit
-// word, generation << 32 | arrivals: the last arrival resets the count and
-// advances the generation in one atomic; the others wait for the generation
-// to move, bounded).  Then every block stages all G rows in shared memory;
-// thread c sums column c into the total and this block's prefix over earlier
-// blocks, and three exclusive scans over the experts run in registers: the
-// expert offsets, the block-scale offsets (block 0 writes both and the
-// counts) and this block's own offsets.  Every slot's row goes to
-// output_permutation; the block's slots are also staged in shared memory in
-// dispatched order, so that input_permutation is written in runs of
-// consecutive rows rather than one scattered word per slot.  Blocks count
-// themselves out on a second word whose high half counts the waits that gave
-// up; the last one reports them in diag[1].
+// may wait on one another; E + 1 <= kSyncThreads).  Before the wait on the
+// producing grid, each block asks L2 for the lines of its ids.  Block b ranks
+// slots [b*nr*NT, (b+1)*nr*NT) within each warp's run, folds the warps into
+// its histogram row (16-bit counts), publishes the row and arrives at a grid
+// barrier: one release reduction on an arrival counter, then a bounded
+// acquire poll until the counter reads G.  Then every block stages all G
+// rows in shared memory; thread c sums column c into the total and this
+// block's prefix over earlier blocks (eight rows in flight), and three
+// exclusive scans over the experts run in registers: the expert offsets, the
+// block-scale offsets (block 0 writes both and the counts) and this block's
+// own offsets.  Every slot's row goes to output_permutation; the block's
+// slots are also staged in shared memory in dispatched order, so that
+// input_permutation is written in runs of consecutive rows rather than one
+// scattered word per slot.  Blocks count themselves out on a second word
+// whose high half counts the waits that gave up; the last one clears both
+// counters and reports the waits in diag[1].
 template <int NT> size_t sync_smem(int E, int G, int nr) {
-    return ((size_t)(NT / 32 + 4 + G) * (E + 1) + 2 * (size_t)nr * NT) * sizeof(int);
+    return (size_t)(NT / 32 + 4) * (E + 1) * sizeof(int) +
+           (size_t)G * sync_stride(E) * sizeof(unsigned short) + 2 * (size_t)nr * NT * sizeof(int);
 }
 
 template <typename IdT>
@@ -533,18 +544,28 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     extern __shared__ int smem[];
     __shared__ int s_wsum[3][NW];
     __shared__ int s_invalid;
-    const int C = E + 1;
+    const int C = E + 1, Cp = sync_stride(E);
     int *wcnt = smem;            // [NW][C] per-warp counts, then exclusive prefixes
-    int *excl = wcnt + NW * C;   // [C] earlier blocks' counts
-    int *off = excl + C;         // [C] expert offsets
-    int *lofs = off + C;         // [C] this block's offsets of its own slots
-    int *rows = wcnt + (NW + 4) * C;  // [G][C] every block's counts (16-byte aligned)
-    int *s_slot = rows + G * C;       // [nr*NT] this block's slots in dispatched order
-    int *s_row = s_slot + nr * NT;    // [nr*NT] and their rows
+    int *base_row = wcnt + NW * C;  // [C] expert offset + earlier blocks' counts
+    int *lofs = base_row + C;       // [C] this block's offsets of its own slots
+    // [G][Cp] every block's counts (16-byte aligned: (NW + 4) * 4 is a multiple of 16)
+    unsigned short *rows = reinterpret_cast<unsigned short *>(wcnt + (NW + 4) * C);
+    int *s_slot = reinterpret_cast<int *>(rows + (size_t)G * Cp);  // [nr*NT] slots, dispatched order
+    int *s_row = s_slot + nr * NT;                                 // [nr*NT] and their rows
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x;
     const int64_t first = (int64_t)tile * nr * NT;
     const PrepWs ws = carve(workspace);
+    {
+        // a hint only: the ids are read after the wait below
+        const int64_t hi = first + (int64_t)nr * NT < S ? first + (int64_t)nr * NT : S;
+        if (first < hi) {
+            const uintptr_t a0 = reinterpret_cast<uintptr_t>(ids + first) & ~uintptr_t(127);
+            const uintptr_t a1 = reinterpret_cast<uintptr_t>(ids + hi);
+            for (uintptr_t a = a0 + (uintptr_t)tid * 128; a < a1; a += (uintptr_t)NT * 128)
+                prefetch_l2(reinterpret_cast<const void *>(a));
+        }
+    }
     for (int x = tid; x < NW * C; x += NT) wcnt[x] = 0;  // shared memory only: before the wait
     if (tid == 0) s_invalid = 0;
     pdl_wait();
@@ -572,6 +593,7 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     __syncthreads();
 
     // fold the warps: column c becomes exclusive over warps; publish the row
+    // (a block has at most nr * NT <= 8192 slots, so every count fits 16 bits)
     if (tid < C) {
         int run = 0;
 #pragma unroll
@@ -580,52 +602,58 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
             wcnt[w * C + tid] = run;
             run += v;
         }
-        ws.hist[(size_t)tile * C + tid] = tid < E ? run : s_invalid;
+        ws.hist[(size_t)tile * Cp + tid] = (unsigned short)(tid < E ? run : s_invalid);
     }
     __syncthreads();
     unsigned done_old = 0, gave_up = 0;
     if (tid == 0) {
         // grid barrier: the arrival releases this block's row (published
-        // before the block barrier above) and, for the last arrival,
-        // acquires every other row
-        const unsigned long long old = atom_add_acq_rel_u64(ws.bar, 1ull);
-        const unsigned gen = (unsigned)(old >> 32);
-        if ((unsigned)old == (unsigned)(G - 1)) {
-            red_add_release_u64(ws.bar, (1ull << 32) - (unsigned long long)G);
-        } else {
-            const unsigned long long t0 = globaltimer_ns();
-            while ((unsigned)(ld_acquire_u64(ws.bar) >> 32) == gen) {
-                if (globaltimer_ns() - t0 >= wait_ns) {
-                    gave_up = 1;
-                    break;
-                }
-                __nanosleep(32);
+        // before the block barrier above); reading G acquires every row
+        red_add_release_u32(ws.arrive, 1u);
+        const unsigned long long t0 = globaltimer_ns();
+        while (ld_acquire_u32(ws.arrive) != (unsigned)G) {
+            if (globaltimer_ns() - t0 >= wait_ns) {
+                gave_up = 1;
+                break;
             }
+            __nanosleep(32);
         }
-        // count this block out; the result is needed only at the end
-        done_old = atomicAdd(ws.done, 1u + (gave_up << 16));
+        // count this block out (ordered after its arrival); the result is
+        // needed only at the end
+        done_old = atom_add_acq_rel_u32(ws.done, 1u + (gave_up << 16));
     }
     __syncthreads();
 
-    // stage the G rows (L2 only: other SMs wrote them), then per column the
-    // total, the prefix over earlier blocks and this block's own count
-    const int n = G * C;
-    if ((n & 3) == 0) {
+    // stage the G rows (L2 only: other SMs wrote them; a row is a multiple
+    // of 16 bytes), then per column the total, the prefix over earlier
+    // blocks and this block's own count
+    {
         const int4 *s4 = reinterpret_cast<const int4 *>(ws.hist);
         int4 *d4 = reinterpret_cast<int4 *>(rows);
-        for (int x = tid; x < (n >> 2); x += NT) d4[x] = __ldcg(s4 + x);
-    } else {
-        for (int x = tid; x < n; x += NT) rows[x] = __ldcg(ws.hist + x);
+        const int n4 = G * Cp / 8;
+        for (int x = tid; x < n4; x += NT) d4[x] = __ldcg(s4 + x);
     }
     __syncthreads();
     int before = 0, all = 0, mine = 0;
     if (tid < C) {
-        for (int t = 0; t < G; ++t) {
-            const int v = rows[t * C + tid];
-            before += t < tile ? v : 0;
-            all += v;
+        const unsigned short *col = rows + tid;
+        int t = 0;
+        for (; t + 8 <= G; t += 8) {
+            int v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) v[q] = col[(t + q) * Cp];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                all += v[q];
+                before += t + q < tile ? v[q] : 0;
+            }
         }
-        mine = rows[tile * C + tid];
+        for (; t < G; ++t) {
+            const int v = col[t * Cp];
+            all += v;
+            before += t < tile ? v : 0;
+        }
+        mine = col[tile * Cp];
     }
     // three exclusive scans over the experts: counts, counts rounded up to
     // A, this block's counts (warp shuffles, then the warp sums)
@@ -665,8 +693,7 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     }
     const int ex_off = ba + ia - cnt;
     if (tid < C) {
-        excl[tid] = before;
-        off[tid] = ex_off;
+        base_row[tid] = ex_off + before;
         lofs[tid] = bo + io - own;
     }
     if (tile == 0) {
@@ -694,7 +721,7 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
             int p = -1;
             if (e >= 0) {
                 const int lr = row[e] + rank[r];
-                p = off[e] + excl[e] + lr;
+                p = base_row[e] + lr;
                 const int lp = lofs[e] + lr;
                 if (lp >= 0 && lp < nr * NT) {
                     s_slot[lp] = (int)i;
@@ -715,7 +742,9 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     const int64_t hi = end < S ? end : S;
     for (int64_t p = lo + tid; p < hi; p += NT) in_perm[p] = -1;
     if (tid == 0 && (done_old & 0xffffu) == (unsigned)(G - 1)) {
+        // every block is past its wait: the counters can start over
         const unsigned to = (done_old >> 16) + gave_up;
+        atomicExch(ws.arrive, 0u);
         atomicExch(ws.done, 0u);
         if (diag) diag[1] = to ? 1 : 0;
     }

@@ -83,7 +83,7 @@ def test_prepare_grid_barrier_that_never_fills_gives_up(wait_us):
     ids_np, _, _, _ = make_workload(w, with_x=False, with_y=False)
     ids = torch.from_numpy(ids_np).to(DEV)
     ws = _ws(w)
-    ws.view(torch.int32)[6] = 1 << 20  # barrier arrivals: no arrival is ever the last one
+    ws.view(torch.int32)[6] = 1 << 20  # barrier arrivals: the count never reads the block count
     moe.moe_set_wait_limits(wait_us, -1)
     meta = moe.moe_prepare(ids, w.E, workspace=ws)
     torch.cuda.synchronize(DEV)  # the kernel ended
