@@ -618,8 +618,12 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
     if per_graph is not None and graph_ms is not None:
         # what the timing events between the calls add to a step: the calls
         # timed with events, summed, against the event-free graph's step
-        breakdown["end_to_end"]["event_overhead_us_per_step"] = (
-            (sum(kern[c] for c in calls) - graph_ms / K) * 1e3)
+        overhead = (sum(kern[c] for c in calls) - graph_ms / K) * 1e3
+        breakdown["end_to_end"]["event_overhead_us_per_step"] = overhead
+        # each call's share of the event-free step, the overhead split
+        # equally between the calls (the shares sum to the step's time)
+        for c in calls:
+            breakdown[c]["us_net_of_events"] = kern[c] * 1e3 - overhead / len(calls)
     return {
         "value": whole_job_tokens_per_s(w.T, K, world, elapsed_ms),
         "ms_per_step": elapsed_ms / K,

@@ -85,13 +85,6 @@ __device__ __forceinline__ void red_add_release_u32(unsigned *p, unsigned v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// A hint to bring the 128-byte line holding p into L2; it returns nothing
-// and orders nothing, so it may run before the wait on the producing grid
-// (L2 is where every SM's writes meet, so a later write updates the line).
-__device__ __forceinline__ void prefetch_l2(const void *p) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
 // Wrapping increment (atomicInc semantics) with acquire-release semantics.
 __device__ __forceinline__ unsigned atom_inc_acq_rel_u32(unsigned *p, unsigned limit) {
     unsigned old;

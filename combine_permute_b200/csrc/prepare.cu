@@ -14,7 +14,7 @@
 //  * up to kSingleBlockSlots slots: one block does it all
 //    (prep_single_kernel);
 //  * above that, when every block fits on the GPU at once: one cooperative
-//    launch (prep_sync_kernel, 512-thread blocks of 2 to 16 rounds).  Each
+//    launch (prep_sync_kernel, 512-thread blocks of 1 to 16 rounds).  Each
 //    block ranks its slots, publishes its per-expert histogram row and meets
 //    the others at a grid barrier (bounded wait); every block then stages
 //    all rows, scans them into the expert offsets and its own prefix, and
@@ -512,11 +512,16 @@ static_assert(kSyncMaxRounds * kSyncThreads <= 65535, "a block's count of one ex
 // off, pad (one column per expert plus one for invalid ids each).
 template <int NT> size_t tile_smem(int E) { return (size_t)(NT / 32 + 4) * (E + 1) * sizeof(int); }
 
+// A slot's expert e (-2..E-1) and its rank within its warp's run (-1..511)
+// in one int.
+__device__ __forceinline__ int pack_key_rank(int e, int rank) { return (rank + 1) << 12 | (e + 2); }
+__device__ __forceinline__ int packed_key(int v) { return (v & 4095) - 2; }
+__device__ __forceinline__ int packed_rank(int v) { return (v >> 12) - 1; }
+
 // One-launch prepare (a cooperative launch: every block resident, so blocks
-// may wait on one another; E + 1 <= kSyncThreads).  Before the wait on the
-// producing grid, each block asks L2 for the lines of its ids.  Block b ranks
-// slots [b*nr*NT, (b+1)*nr*NT) within each warp's run, folds the warps into
-// its histogram row (16-bit counts), publishes the row and arrives at a grid
+// may wait on one another; E + 1 <= kSyncThreads).  Block b ranks slots
+// [b*nr*NT, (b+1)*nr*NT) within each warp's run, folds the warps into its
+// histogram row (16-bit counts), publishes the row and arrives at a grid
 // barrier: one release reduction on an arrival counter, then a bounded
 // acquire poll until the counter reads G.  Then every block stages all G
 // rows in shared memory; thread c sums column c into the total and this
@@ -531,7 +536,7 @@ template <int NT> size_t tile_smem(int E) { return (size_t)(NT / 32 + 4) * (E + 
 // counters and reports the waits in diag[1].
 template <int NT> size_t sync_smem(int E, int G, int nr) {
     return (size_t)(NT / 32 + 4) * (E + 1) * sizeof(int) +
-           (size_t)G * sync_stride(E) * sizeof(unsigned short) + 2 * (size_t)nr * NT * sizeof(int);
+           (size_t)G * sync_stride(E) * sizeof(unsigned short) + 3 * (size_t)nr * NT * sizeof(int);
 }
 
 template <typename IdT>
@@ -540,7 +545,7 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
                      int nr, void *workspace, unsigned long long wait_ns, int32_t *counts,
                      int32_t *offsets, int32_t *bso, int32_t *in_perm, int32_t *out_perm,
                      int32_t *diag) {
-    constexpr int NT = kSyncThreads, NW = NT / 32, NR = kSyncMaxRounds;
+    constexpr int NT = kSyncThreads, NW = NT / 32;
     extern __shared__ int smem[];
     __shared__ int s_wsum[3][NW];
     __shared__ int s_invalid;
@@ -552,20 +557,11 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     unsigned short *rows = reinterpret_cast<unsigned short *>(wcnt + (NW + 4) * C);
     int *s_slot = reinterpret_cast<int *>(rows + (size_t)G * Cp);  // [nr*NT] slots, dispatched order
     int *s_row = s_slot + nr * NT;                                 // [nr*NT] and their rows
+    int *s_kr = s_row + nr * NT;  // [nr*NT] each slot's expert and rank, warp by warp
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x;
     const int64_t first = (int64_t)tile * nr * NT;
     const PrepWs ws = carve(workspace);
-    {
-        // a hint only: the ids are read after the wait below
-        const int64_t hi = first + (int64_t)nr * NT < S ? first + (int64_t)nr * NT : S;
-        if (first < hi) {
-            const uintptr_t a0 = reinterpret_cast<uintptr_t>(ids + first) & ~uintptr_t(127);
-            const uintptr_t a1 = reinterpret_cast<uintptr_t>(ids + hi);
-            for (uintptr_t a = a0 + (uintptr_t)tid * 128; a < a1; a += (uintptr_t)NT * 128)
-                prefetch_l2(reinterpret_cast<const void *>(a));
-        }
-    }
     for (int x = tid; x < NW * C; x += NT) wcnt[x] = 0;  // shared memory only: before the wait
     if (tid == 0) s_invalid = 0;
     pdl_wait();
@@ -575,17 +571,22 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     const unsigned lt = lanemask_lt();
     const int nbits = key_bits(E);
     const int64_t wbase = first + (int64_t)warp * 32 * nr;
-    int key[NR], rank[NR];
-#pragma unroll
-    for (int r = 0; r < NR; ++r)
-        key[r] = r < nr ? load_key(ids, wbase + r * 32 + lane, S, base, E) : -2;
+    // Round r of this lane is slot wbase + r*32 + lane; its expert, then its
+    // rank, live in shared memory at kr[r*32] (read and written by this lane
+    // only).  The loops stay rolled: fully unrolled over the largest round
+    // count, the kernel's code ran slower than its work (each launch fetches
+    // it anew).
+    int *kr = s_kr + warp * 32 * nr + lane;
+#pragma unroll 4
+    for (int r = 0; r < nr; ++r) kr[r * 32] = load_key(ids, wbase + r * 32 + lane, S, base, E);
     __syncthreads();
     int *row = wcnt + warp * C;
     int bad = 0;
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-        if (r < nr) rank[r] = rank_round(key[r], E, nbits, row, lt);
-        bad += key[r] == -1;
+#pragma unroll 1
+    for (int r = 0; r < nr; ++r) {
+        const int e = kr[r * 32];
+        kr[r * 32] = pack_key_rank(e, rank_round(e, E, nbits, row, lt));
+        bad += e == -1;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
@@ -713,14 +714,15 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     // rows: slot i of expert e is this block's lr-th slot of e, lr = earlier
     // warps + its rank in the warp's run; output_permutation directly,
     // input_permutation through the staged dispatched order
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
+#pragma unroll 1
+    for (int r = 0; r < nr; ++r) {
         const int64_t i = wbase + r * 32 + lane;
-        if (r < nr && i < S) {
-            const int e = key[r];
+        if (i < S) {
+            const int v = kr[r * 32];
+            const int e = packed_key(v);
             int p = -1;
             if (e >= 0) {
-                const int lr = row[e] + rank[r];
+                const int lr = row[e] + packed_rank(v);
                 p = base_row[e] + lr;
                 const int lp = lofs[e] + lr;
                 if (lp >= 0 && lp < nr * NT) {
@@ -866,23 +868,23 @@ namespace {
 
 // Tile shape of the one-launch path: nr rounds of kSyncThreads slots per
 // block, G = ceil(S / (nr * kSyncThreads)) blocks.  nr is the fewest rounds
-// from 2 to kSyncMinRounds that keeps the histogram rows every block stages
+// from 1 to kSyncMinRounds that keeps the histogram rows every block stages
 // (G x (E+1) counts) within kSyncStagedCounts, else kSyncMinRounds; more
 // when the blocks would not all be resident.  Fewer rounds shorten the
-// ranking, more blocks lengthen the staging: measured per call, 32768 slots
-// of 256 experts took 9.2 us at 2 rounds against 9.7 at 4, 73728 slots 9.75
-// us at 3 against 10.0-10.1, 131072 slots of 288 experts 11.05 us at 4
-// against 11.7 at 2.  False when the problem needs more than kSyncMaxRounds
-// rounds or kMaxSyncTiles blocks, or has more experts than a block has
-// threads.
-constexpr int64_t kSyncStagedCounts = 16384;
+// ranking, more blocks lengthen the staging: measured per call back to
+// back, 32768 slots of 256 experts took 7.3 us at 1 round against 7.4 at 2
+// and 8.5 at 4, 73728 slots 8.25 us at 2 rounds against 8.55 at 3 and 8.75
+// at 1, 131072 slots of 288 experts 9.4 us at 4 against 9.45 at 2 and 3 and
+// 10.7 at 6.  False when the problem needs more than kSyncMaxRounds rounds
+// or kMaxSyncTiles blocks, or has more experts than a block has threads.
+constexpr int64_t kSyncStagedCounts = 20480;
 
 bool sync_shape(int64_t S, int E, int64_t resident, int *nr_out, int *G_out) {
     if (E + 1 > kSyncThreads) return false;
     const int64_t cap = resident < kMaxSyncTiles ? resident : kMaxSyncTiles;
     if (cap < 1) return false;
     int64_t least = kSyncMinRounds;
-    for (int64_t r = 2; r < kSyncMinRounds; ++r) {
+    for (int64_t r = 1; r < kSyncMinRounds; ++r) {
         const int64_t G = (S + r * kSyncThreads - 1) / (r * kSyncThreads);
         if (G * (E + 1) <= kSyncStagedCounts) {
             least = r;

@@ -78,7 +78,7 @@ def _ws(w):
 
 @pytest.mark.parametrize("wait_us", [-1, 0])
 def test_prepare_grid_barrier_that_never_fills_gives_up(wait_us):
-    # 32768 slots: the one-launch path (16 blocks and one grid barrier)
+    # 32768 slots: the one-launch path (64 blocks and one grid barrier)
     w = CONFIGS["uniform_t4096_h7168_e256_k8"]
     ids_np, _, _, _ = make_workload(w, with_x=False, with_y=False)
     ids = torch.from_numpy(ids_np).to(DEV)

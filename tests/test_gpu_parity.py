@@ -220,9 +220,10 @@ def _fp8_run(ids_np, E, x, A):
 
 
 @pytest.mark.parametrize("xdt", ["bf16", "fp16"])
-@pytest.mark.parametrize("T,H,E,k,A", [(300, 4096, 288, 8, 128), (77, 384, 16, 3, 1),
-                                       (40, 128, 5, 2, 32)])
+@pytest.mark.parametrize("T,H,E,k,A", [(300, 4096, 288, 8, 128), (129, 7168, 64, 4, 8),
+                                       (77, 384, 16, 3, 1), (40, 128, 5, 2, 32)])
 def test_dispatch_fp8_vs_oracle(xdt, T, H, E, k, A):
+    # H = 7168: two 16-element groups a thread; the others one
     rng = np.random.default_rng(T + H)
     ids_np = _ids_random(rng, T, k, E, p_invalid=0.02)
     x = torch.randn(T, H, device=DEV)
@@ -493,8 +494,10 @@ def test_chained_step_on_one_stream():
     (4097, 511),            # one-launch path, widest expert range it takes (E + 1 = 512)
     (4097, 512),            # one expert more: the two-kernel path
     (32768, 511),           # 2 rounds, 32 blocks
-    (65536, 255),           # last size at 2 rounds (64 rows of 256 staged counts)
-    (65537, 255),           # first at 3 rounds
+    (40960, 255),           # last size at 1 round (80 rows of 256 staged counts)
+    (40961, 255),           # first at 2 rounds
+    (81920, 255),           # last size at 2 rounds
+    (81921, 255),           # first at 3 rounds
     (1212416, 64),          # the largest one-launch problem on 148 SMs (16 rounds)
     (1212417, 64),          # one slot more: the two-kernel path
 ])
