@@ -623,7 +623,9 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
         # each call's share of the event-free step, the overhead split
         # equally between the calls (the shares sum to the step's time)
         for c in calls:
-            breakdown[c]["us_net_of_events"] = kern[c] * 1e3 - overhead / len(calls)
+            net = kern[c] * 1e3 - overhead / len(calls)
+            breakdown[c]["us_net_of_events"] = net
+            breakdown[c]["net_frac_of_8tbs_spec"] = alg[c] / (net * 1e-6) / 1e9 / SPEC_HBM_GBS
     return {
         "value": whole_job_tokens_per_s(w.T, K, world, elapsed_ms),
         "ms_per_step": elapsed_ms / K,
