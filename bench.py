@@ -625,7 +625,8 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
         for c in calls:
             net = kern[c] * 1e3 - overhead / len(calls)
             breakdown[c]["us_net_of_events"] = net
-            breakdown[c]["net_frac_of_8tbs_spec"] = alg[c] / (net * 1e-6) / 1e9 / SPEC_HBM_GBS
+            breakdown[c]["net_frac_of_8tbs_spec"] = (
+                alg[c] / (net * 1e-6) / 1e9 / SPEC_HBM_GBS if net > 0 else None)
     return {
         "value": whole_job_tokens_per_s(w.T, K, world, elapsed_ms),
         "ms_per_step": elapsed_ms / K,
