@@ -301,7 +301,7 @@ def _config(w, n):
             "routing": w.routing.mode, "x_dtype": w.x_dtype, "dispatch_dtype": w.dispatch_dtype,
             "y_dtype": w.y_dtype, "out_dtype": w.out_dtype, "seed": w.seed,
             "l2": ("no flush: per-step working set > 126 MB L2" if _step_bytes(w) > L2_BYTES
-                   else "no flush: the working set fits in L2 (a latency figure)"),
+                   else "flushed: a buffer of twice the L2 size written before every timed step"),
             "parallelism": "replicas" if n > 1 else "single GPU"}
 
 
@@ -557,6 +557,27 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
     except Exception as exc:
         print(f"back-to-back call timing unavailable: {exc}", file=sys.stderr)
 
+    # ---- timed region 5, only for a step whose working set fits in L2: K
+    #      eager steps, each after an L2 flush (a buffer of twice the L2
+    #      size written outside the step's events), so that no step finds
+    #      its inputs left in L2 by the one before; their sum is the value
+    flushed_ms, clocks_flushed = None, None
+    if _step_bytes(w) <= L2_BYTES:
+        flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+        fmarks = [(ev(), ev()) for _ in range(K)]
+        barrier()
+        torch.cuda.synchronize(dev)
+        with ClockSampler(local) as clocks_flushed:
+            for i in range(K):
+                flush_buf.fill_(i & 0xff)
+                fmarks[i][0].record(stream)
+                step.run()
+                fmarks[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+        barrier()
+        flushed_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in fmarks))
+        del flush_buf
+
     counts = step.meta_bufs["expert_counts"].cpu().numpy()
     diag = step.meta_bufs["diag"].cpu().numpy().tolist()
 
@@ -627,11 +648,22 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
             breakdown[c]["us_net_of_events"] = net
             breakdown[c]["net_frac_of_8tbs_spec"] = (
                 alg[c] / (net * 1e-6) / 1e9 / SPEC_HBM_GBS if net > 0 else None)
+    launch = (f"cuda_graph of {n_graph} steps, replayed {K // n_graph} times"
+              if graph_ms is not None else "eager")
+    l2_resident = None
+    if flushed_ms is not None:
+        # the flushed steps are the value; the graph's steps, whose inputs
+        # the step before left in L2, are kept beside them
+        l2_resident = {"value": whole_job_tokens_per_s(w.T, K, world, elapsed_ms),
+                       "ms_per_step": elapsed_ms / K, "launch": launch}
+        elapsed_ms, launch = flushed_ms, ("eager steps, each after an L2 flush, CUDA events "
+                                          "around each step")
+        clocks = clocks_flushed
     return {
         "value": whole_job_tokens_per_s(w.T, K, world, elapsed_ms),
         "ms_per_step": elapsed_ms / K,
-        "launch": (f"cuda_graph of {n_graph} steps, replayed {K // n_graph} times"
-                   if graph_ms is not None else "eager"),
+        "launch": launch,
+        "l2_resident": l2_resident,
         "eager_value": whole_job_tokens_per_s(w.T, K, world, eager_ms),
         "roofline": {"bound": "hbm", "kernel": kernel_key, "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
