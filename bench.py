@@ -685,16 +685,22 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
     }
 
 
-def profile_run(args, workloads):
+def profile_run(args, workloads, next_rows=False):
     """W warm-up and K eager steps of each workload, nothing else: the
-    program the ncu captures run."""
+    program the ncu captures run.  With next_rows, one prepare and then W + K
+    eager launches of each call beside the path (next_row_calls) instead."""
     import torch
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     for w in workloads:
         step = Step(w, dev)
-        for _ in range(args.warmup + args.steps):
-            step.run()
+        if next_rows:
+            for fn in next_row_calls(step, w, dev).values():
+                for _ in range(args.warmup + args.steps):
+                    fn()
+        else:
+            for _ in range(args.warmup + args.steps):
+                step.run()
         torch.cuda.synchronize(dev)
         del step
         torch.cuda.empty_cache()
@@ -817,18 +823,50 @@ def time_calls_alone(step, dev, K, n):
     return out
 
 
-def time_next_rows(step, w, dev, reps=20):
-    """The steps beside the timed path: the grouped-GEMM metadata that follows
-    prepare (tile-padded layout with 128-row tiles, per-expert problem
-    sizes) and the NVFP4 dispatch of this workload's activations, each timed
-    as a CUDA graph of `reps` calls."""
+NEXT_TILE = 128  # rows per tile of the grouped-GEMM layout timed beside the path
+
+
+def next_row_bytes(w):
+    """Algorithmic bytes of the calls beside the timed path (next_row_calls)."""
+    S, E = w.S, w.E
+    max_tiles = max(1, -(-S // NEXT_TILE) + min(E, S))
+    x_b = 4 if w.x_dtype == "fp32" else 2
+    return {
+        "tile_layout_t128": (8 * S + 8 * E + 4 * (E + 1) + 8 * max_tiles + 4 * S
+                             + 4 * max_tiles * NEXT_TILE + 8),
+        "problem_sizes": 4 * E + 24 * E,
+        "dispatch_nvfp4": w.T * w.H * x_b + S * (w.H // 2 + w.H // 16) + 4 * S + 8 * (E + 1),
+    }
+
+
+def next_row_calls(step, w, dev):
+    """The calls beside the timed path, on the step's buffers after one
+    prepare: the grouped-GEMM metadata that follows prepare (tile-padded
+    layout with 128-row tiles, per-expert problem sizes) and the NVFP4
+    dispatch of this workload's activations.  Returns name -> call."""
     import torch
     moe = step.moe
     meta = step.prepare()
-    tile = 128
     S, E = w.S, w.E
-    max_tiles = max(1, -(-S // tile) + min(E, S))
-    out = {}
+    max_tiles = max(1, -(-S // NEXT_TILE) + min(E, S))
+    calls = {
+        "tile_layout_t128": lambda: moe.moe_tile_layout(meta, w.k, NEXT_TILE, max_tiles),
+        "problem_sizes": lambda: moe.moe_problem_sizes(meta.expert_counts, 2 * w.H, w.H, w.H, w.H),
+    }
+    if step.x.dtype in (torch.bfloat16, torch.float16) and w.H % 16 == 0:
+        bso = meta.blockscale_offsets if meta.blockscale_offsets is not None else meta.expert_offsets
+        A = step.A or 1
+        q = torch.empty((S, w.H // 2), dtype=torch.uint8, device=dev)
+        sc = torch.empty((S + E * (A - 1), w.H // 16), dtype=torch.uint8, device=dev)
+        calls["dispatch_nvfp4"] = lambda: moe.moe_dispatch_rows_nvfp4(
+            step.x, w.k, meta.output_permutation, meta.expert_offsets, bso, out_q=q,
+            out_scales=sc)
+    return calls
+
+
+def time_next_rows(step, w, dev, reps=20):
+    """Each call of next_row_calls timed as a CUDA graph of `reps` calls."""
+    import torch
 
     def timed(fn):
         fn()
@@ -849,22 +887,13 @@ def time_next_rows(step, w, dev, reps=20):
         torch.cuda.synchronize(dev)
         return s.elapsed_time(e) / reps * 1e3
 
-    us = timed(lambda: moe.moe_tile_layout(meta, w.k, tile, max_tiles))
-    b = 8 * S + 8 * E + 4 * (E + 1) + 8 * max_tiles + 4 * S + 4 * max_tiles * tile + 8
-    out["tile_layout_t128"] = {"us": us, "algorithmic_bytes": b, "effective_gbs": b / us / 1e3}
-    us = timed(lambda: moe.moe_problem_sizes(meta.expert_counts, 2 * w.H, w.H, w.H, w.H))
-    b = 4 * E + 24 * E
-    out["problem_sizes"] = {"us": us, "algorithmic_bytes": b}
-    if step.x.dtype in (torch.bfloat16, torch.float16) and w.H % 16 == 0:
-        bso = meta.blockscale_offsets if meta.blockscale_offsets is not None else meta.expert_offsets
-        A = step.A or 1
-        q = torch.empty((S, w.H // 2), dtype=torch.uint8, device=dev)
-        sc = torch.empty((S + E * (A - 1), w.H // 16), dtype=torch.uint8, device=dev)
-        us = timed(lambda: moe.moe_dispatch_rows_nvfp4(step.x, w.k, meta.output_permutation,
-                                                       meta.expert_offsets, bso, out_q=q,
-                                                       out_scales=sc))
-        b = w.T * w.H * step.x.element_size() + S * (w.H // 2 + w.H // 16) + 4 * S + 8 * (E + 1)
-        out["dispatch_nvfp4"] = {"us": us, "algorithmic_bytes": b, "effective_gbs": b / us / 1e3}
+    nbytes = next_row_bytes(w)
+    out = {}
+    for name, fn in next_row_calls(step, w, dev).items():
+        us = timed(fn)
+        out[name] = {"us": us, "algorithmic_bytes": nbytes[name]}
+        if name != "problem_sizes":
+            out[name]["effective_gbs"] = nbytes[name] / us / 1e3
     return out
 
 
@@ -979,6 +1008,9 @@ def main():
     ap.add_argument("--profile-run", action="store_true",
                     help="only the warm-up and K eager steps of each workload, no JSON line "
                          "(a short program for ncu)")
+    ap.add_argument("--profile-next", action="store_true",
+                    help="like --profile-run, for the calls timed beside the path (tile layout, "
+                         "problem sizes, NVFP4 dispatch)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -990,8 +1022,8 @@ def main():
                  for n in names}
     if args.impl == "reference":
         run_reference(args, workloads[names[0]])
-    elif args.profile_run:
-        profile_run(args, [workloads[n] for n in names])
+    elif args.profile_run or args.profile_next:
+        profile_run(args, [workloads[n] for n in names], next_rows=args.profile_next)
     else:
         run_gpu(args, names, workloads)
 

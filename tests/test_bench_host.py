@@ -59,3 +59,13 @@ def test_traffic_counts_only_for_the_captured_sources(monkeypatch):
     assert bench.committed_traffic(key) == entry["dram_bytes_per_launch"]
     monkeypatch.setattr(bench, "src_hash", lambda step: "0" * 16)
     assert bench.committed_traffic(key) is None
+
+
+def test_next_row_bytes_of_the_fp8_workload():
+    """Worked by hand for T=16384, H=4096, E=288, k=8 (S = 131072): the NVFP4
+    dispatch reads x once (16384 * 4096 * 2), writes 2048 code bytes and 256
+    scale bytes per slot, reads the permutation (4 bytes a slot) and the two
+    offset arrays (8 * 289)."""
+    b = bench.next_row_bytes(CONFIGS["zipf_fp8_t16384_h4096_e288_k8"])
+    assert b["dispatch_nvfp4"] == 134217728 + 131072 * 2304 + 524288 + 2312
+    assert b["problem_sizes"] == 28 * 288

@@ -51,7 +51,8 @@ def _run(ids_np, E, x, A):
 
 @pytest.mark.parametrize("xdt", ["bf16", "fp16"])
 @pytest.mark.parametrize("T,H,E,k,A", [(300, 4096, 288, 8, 128), (77, 48, 16, 3, 1),
-                                       (40, 16, 5, 2, 32), (513, 7168, 64, 6, 4)])
+                                       (40, 16, 5, 2, 32), (513, 7168, 64, 6, 4),
+                                       (50, 4096, 64, 40, 4), (31, 2048, 40, 32, 1)])
 def test_dispatch_nvfp4_vs_oracle(xdt, T, H, E, k, A):
     rng = np.random.default_rng(T + H)
     ids_np = _ids(rng, T, k, E, p_invalid=0.02)

@@ -221,9 +221,10 @@ def _fp8_run(ids_np, E, x, A):
 
 @pytest.mark.parametrize("xdt", ["bf16", "fp16"])
 @pytest.mark.parametrize("T,H,E,k,A", [(300, 4096, 288, 8, 128), (129, 7168, 64, 4, 8),
-                                       (77, 384, 16, 3, 1), (40, 128, 5, 2, 32)])
+                                       (77, 384, 16, 3, 1), (40, 128, 5, 2, 32),
+                                       (50, 4096, 64, 40, 4), (33, 7168, 48, 33, 2)])
 def test_dispatch_fp8_vs_oracle(xdt, T, H, E, k, A):
-    # H = 7168: two 16-element groups a thread; the others one
+    # H = 7168: two 16-element groups a thread; the others one; top-k up to 40
     rng = np.random.default_rng(T + H)
     ids_np = _ids_random(rng, T, k, E, p_invalid=0.02)
     x = torch.randn(T, H, device=DEV)
