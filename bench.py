@@ -824,6 +824,7 @@ def time_calls_alone(step, dev, K, n):
 
 
 NEXT_TILE = 128  # rows per tile of the grouped-GEMM layout timed beside the path
+EP_RANKS = 2     # ranks of the exchange between GPUs, emulated on this GPU
 
 
 def next_row_bytes(w):
@@ -836,14 +837,26 @@ def next_row_bytes(w):
                              + 4 * max_tiles * NEXT_TILE + 8),
         "problem_sizes": 4 * E + 24 * E,
         "dispatch_nvfp4": w.T * w.H * x_b + S * (w.H // 2 + w.H // 16) + 4 * S + 8 * (E + 1),
+        # the exchange's own kernels, both owners' buffers on this GPU
+        "ep_peer_layout_r2": (4 * EP_RANKS * E + 4 * S + 4 * (E + 1) + 4 * S + 8 * S
+                              + 4 * EP_RANKS + 4 * (E // EP_RANKS + 1)),
+        "ep_dispatch_peer_r2": w.T * w.H * x_b + S * w.H * x_b + 8 * S,
+        "ep_combine_peer_r2": S * w.H * x_b + 8 * S + 4 * S + w.T * w.H * _out_bytes(w),
     }
+
+
+def _out_bytes(w):
+    return {"fp32": 4, "bf16": 2, "fp16": 2}[w.out_dtype]
 
 
 def next_row_calls(step, w, dev):
     """The calls beside the timed path, on the step's buffers after one
     prepare: the grouped-GEMM metadata that follows prepare (tile-padded
-    layout with 128-row tiles, per-expert problem sizes) and the NVFP4
-    dispatch of this workload's activations.  Returns name -> call."""
+    layout with 128-row tiles, per-expert problem sizes), the NVFP4 dispatch
+    of this workload's activations, and the exchange between GPUs in its
+    fused form with EP_RANKS ranks emulated on this GPU (both owners'
+    buffers here; every rank routes this step's tokens, and rank 0's layout,
+    dispatch and combine are timed).  Returns name -> call."""
     import torch
     moe = step.moe
     meta = step.prepare()
@@ -861,6 +874,17 @@ def next_row_calls(step, w, dev):
         calls["dispatch_nvfp4"] = lambda: moe.moe_dispatch_rows_nvfp4(
             step.x, w.k, meta.output_permutation, meta.expert_offsets, bso, out_q=q,
             out_scales=sc)
+    if step.x.dtype in (torch.bfloat16, torch.float16) and E % EP_RANKS == 0:
+        counts = torch.stack([meta.expert_counts] * EP_RANKS).contiguous()
+        lay = moe.moe_ep_peer_layout(counts, 0, step.ids, meta)
+        rows = lay.recv_rows.tolist()
+        bufs = [torch.empty((max(n, 1), w.H), dtype=step.x.dtype, device=dev) for n in rows]
+        step.ep_buffers = bufs  # alive as long as the step (the table refers to them too)
+        table = moe.moe_ep_buffer_table(bufs, dev)
+        calls["ep_peer_layout_r2"] = lambda: moe.moe_ep_peer_layout(counts, 0, step.ids, meta)
+        calls["ep_dispatch_peer_r2"] = lambda: moe.moe_ep_dispatch_peer(step.x, w.k, lay, table)
+        calls["ep_combine_peer_r2"] = lambda: moe.moe_ep_combine_peer(
+            table, step.x.dtype, w.H, lay, step.wt, out=step.out)
     return calls
 
 
@@ -892,7 +916,7 @@ def time_next_rows(step, w, dev, reps=20):
     for name, fn in next_row_calls(step, w, dev).items():
         us = timed(fn)
         out[name] = {"us": us, "algorithmic_bytes": nbytes[name]}
-        if name != "problem_sizes":
+        if name not in ("problem_sizes", "ep_peer_layout_r2"):
             out[name]["effective_gbs"] = nbytes[name] / us / 1e3
     return out
 

@@ -44,6 +44,7 @@ __all__ = [
     "EpPeerLayout",
     "moe_ep_dispatch_peer",
     "moe_ep_combine_peer",
+    "moe_ep_buffer_table",
     "TileLayout",
     "library_path",
 ]
@@ -520,17 +521,33 @@ def moe_ep_peer_layout(all_expert_counts: torch.Tensor, rank: int, topk_ids: tor
     return lay
 
 
-def _pointer_array(buffers, dev) -> torch.Tensor:
-    """A device array of the buffers' addresses (tensors, or raw device
-    addresses valid in this process, e.g. another GPU's memory mapped in)."""
+def moe_ep_buffer_table(buffers, device) -> torch.Tensor:
+    """The device array of the ranks' buffer addresses that moe_ep_dispatch_peer
+    and moe_ep_combine_peer read (int64 [R] on ``device``), from tensors or raw
+    device addresses valid in this process (another GPU's memory mapped in).
+    Building it copies from the host; a caller that records the exchange in a
+    CUDA graph builds it once beforehand and passes it in place of the list.
+    The table holds references to the tensors it was built from, so that
+    their memory stays allocated while the table exists (torch may otherwise
+    hand freed blocks back to the driver, e.g. when a graph capture begins);
+    raw addresses stay the caller's to keep valid."""
     ptrs = [b.data_ptr() if isinstance(b, torch.Tensor) else int(b) for b in buffers]
-    return torch.tensor(ptrs, dtype=torch.int64).to(dev)
+    table = torch.tensor(ptrs, dtype=torch.int64).to(device)
+    table._buffers = [b for b in buffers if isinstance(b, torch.Tensor)]
+    return table
+
+
+def _pointer_array(buffers, dev) -> torch.Tensor:
+    if isinstance(buffers, torch.Tensor):  # a table from moe_ep_buffer_table
+        _need(buffers, "buffer table", torch.int64, (buffers.numel(),), dev)
+        return buffers
+    return moe_ep_buffer_table(buffers, dev)
 
 
 def moe_ep_dispatch_peer(x: torch.Tensor, top_k: int, layout: EpPeerLayout, recv_buffers) -> None:
     """Stores every row of x [T, H] into the grouped buffers of the ranks
     owning its experts (``recv_buffers``: one per rank, tensors or device
-    addresses; see include/moe.h)."""
+    addresses, or their moe_ep_buffer_table; see include/moe.h)."""
     _need(x, "x")
     T, H = x.shape
     dev = x.device
@@ -551,8 +568,9 @@ def moe_ep_combine_peer(out_buffers, y_dtype: torch.dtype, hidden: int, layout: 
                         weights: torch.Tensor, *, out_dtype: Optional[torch.dtype] = None,
                         out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """out[t] = sum_j weights[t, j] * (expert output of slot (t, j), read from
-    its owner's buffer ``out_buffers[rank]``), fp32 accumulation in slot
-    order (see include/moe.h)."""
+    its owner's buffer ``out_buffers[rank]``, or through their
+    moe_ep_buffer_table), fp32 accumulation in slot order (see
+    include/moe.h)."""
     _need(weights, "weights", torch.float32)
     T, k = weights.shape
     dev = weights.device

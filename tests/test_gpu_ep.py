@@ -253,3 +253,56 @@ def test_ep_peer_module_over_a_one_rank_nccl_group():
     assert np.array_equal(local_offsets.cpu().numpy(), ref["offsets"])
     assert np.array_equal(bits(out), oracle.combine(bits(y), "bf16", ref["output_perm"], wt_np,
                                                     "bf16"))
+
+
+def test_peer_calls_take_a_prebuilt_buffer_table():
+    """moe_ep_buffer_table built once (as for a CUDA graph) gives the same
+    bytes as the list of buffers, and the peer dispatch records into a graph
+    with it."""
+    base, ranks = _emulated_ranks(2, 600, 11)
+    E, k, H = base.E, base.k, base.H
+    counts = torch.stack([r["meta"].expert_counts for r in ranks]).contiguous()
+    r = ranks[0]
+    lay = moe.moe_ep_peer_layout(counts, 0, r["ids"], r["meta"])
+    rows = lay.recv_rows.tolist()
+    want = [torch.full((n, H), -3.0, dtype=torch.bfloat16, device=DEV) for n in rows]
+    moe.moe_ep_dispatch_peer(r["x"], k, lay, want)
+    got = [torch.full((n, H), -3.0, dtype=torch.bfloat16, device=DEV) for n in rows]
+    table = moe.moe_ep_buffer_table(got, DEV)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(g, stream=side):
+            moe.moe_ep_dispatch_peer(r["x"], k, lay, table)
+    g.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(want, got):
+        assert np.array_equal(bits(a), bits(b))
+    wt = torch.from_numpy(r["wt"]).to(DEV)
+    assert np.array_equal(bits(moe.moe_ep_combine_peer(want, torch.bfloat16, H, lay, wt)),
+                          bits(moe.moe_ep_combine_peer(table, torch.bfloat16, H, lay, wt)))
+
+
+def test_buffer_table_keeps_its_buffers_allocated():
+    """The table refers to the tensors it was built from: dropping the
+    caller's list and emptying torch's cache (as a graph capture does) leaves
+    the memory it points to allocated, so the peer dispatch still has it."""
+    import gc
+    base, ranks = _emulated_ranks(2, 400, 12)
+    counts = torch.stack([r["meta"].expert_counts for r in ranks]).contiguous()
+    r = ranks[0]
+    lay = moe.moe_ep_peer_layout(counts, 0, r["ids"], r["meta"])
+    rows = lay.recv_rows.tolist()
+    bufs = [torch.full((n, base.H), -3.0, dtype=torch.bfloat16, device=DEV) for n in rows]
+    want = [b.clone() for b in bufs]
+    moe.moe_ep_dispatch_peer(r["x"], base.k, lay, want)
+    table = moe.moe_ep_buffer_table(bufs, DEV)
+    kept = table._buffers
+    del bufs
+    gc.collect()
+    torch.cuda.empty_cache()
+    moe.moe_ep_dispatch_peer(r["x"], base.k, lay, table)
+    torch.cuda.synchronize()
+    for a, b in zip(want, kept):
+        assert np.array_equal(bits(a), bits(b))
