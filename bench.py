@@ -867,7 +867,8 @@ def next_row_calls(step, w, dev):
         "problem_sizes": lambda: moe.moe_problem_sizes(meta.expert_counts, 2 * w.H, w.H, w.H, w.H),
     }
     if step.x.dtype in (torch.bfloat16, torch.float16) and w.H % 16 == 0:
-        bso = meta.blockscale_offsets if meta.blockscale_offsets is not None else meta.expert_offsets
+        bso = (meta.blockscale_offsets if meta.blockscale_offsets is not None
+               else meta.expert_offsets)
         A = step.A or 1
         q = torch.empty((S, w.H // 2), dtype=torch.uint8, device=dev)
         sc = torch.empty((S + E * (A - 1), w.H // 16), dtype=torch.uint8, device=dev)

@@ -555,8 +555,8 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     int *lofs = base_row + C;       // [C] this block's offsets of its own slots
     // [G][Cp] every block's counts (16-byte aligned: (NW + 4) * 4 is a multiple of 16)
     unsigned short *rows = reinterpret_cast<unsigned short *>(wcnt + (NW + 4) * C);
-    int *s_slot = reinterpret_cast<int *>(rows + (size_t)G * Cp);  // [nr*NT] slots, dispatched order
-    int *s_row = s_slot + nr * NT;                                 // [nr*NT] and their rows
+    int *s_slot = reinterpret_cast<int *>(rows + (size_t)G * Cp);  // [nr*NT] slots,
+    int *s_row = s_slot + nr * NT;  // [nr*NT] and their rows, in dispatched order
     int *s_kr = s_row + nr * NT;  // [nr*NT] each slot's expert and rank, warp by warp
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x;
