@@ -32,9 +32,9 @@ constexpr int kCopyUnroll = 8;  // 16-byte vectors in flight per thread
 // its previous chunk have finished reading it (bulk async-group wait).  The
 // row is read from HBM once and written k times with one instruction per
 // copy, so the load/store unit queues never throttle.  Each lane loads its
-// destinations for the next unit while the current one is stored.  The host
-// splits rows into `nch` chunks so that the (token, chunk) units spread
-// evenly over the persistent grid.
+// destinations for the next unit while the current one is stored.  The host splits rows
+// into `nch` chunks so that the (token, chunk) units spread evenly over the
+// persistent grid.
 // ---------------------------------------------------------------------------
 constexpr int kBulkMaxStages = 16;
 constexpr uint32_t kBulkSmem = 64 * 1024;   // stage ring per block
