@@ -487,7 +487,15 @@ static int64_t bulk_split(int64_t T, int64_t row_bytes, int64_t grid_max) {
 template <typename Rows>
 static cudaError_t launch_bulk(const void *x, int64_t T, int64_t row_bytes, int k,
                                const Rows &rows, int64_t nsplit, cudaStream_t stream) {
-    const uint32_t chunk = (uint32_t)(((row_bytes + nsplit - 1) / nsplit + 15) / 16 * 16);
+    // chunks of the row, at least two of which fit the stage ring
+    auto chunk_of = [&](int64_t ns) {
+        return (uint32_t)(((row_bytes + ns - 1) / ns + 15) / 16 * 16);
+    };
+    constexpr int64_t kMaxChunk = kBulkSmem / 2;
+    if (nsplit < (row_bytes + kMaxChunk - 1) / kMaxChunk)
+        nsplit = (row_bytes + kMaxChunk - 1) / kMaxChunk;
+    uint32_t chunk = chunk_of(nsplit);
+    while (chunk > kMaxChunk) chunk = chunk_of(++nsplit);  // rounding up to 16 bytes
     const int64_t nch = (row_bytes + chunk - 1) / chunk;
     int stages = (int)(kBulkSmem / chunk);
     if (stages > kBulkMaxStages) stages = kBulkMaxStages;

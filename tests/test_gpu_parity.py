@@ -173,6 +173,27 @@ def test_dispatch_vs_oracle(form, dtype, H):
     np.testing.assert_array_equal(bits(out), ref)
 
 
+@pytest.mark.parametrize("T,H", [(40, 300_000), (32, 600_000)])
+def test_dispatch_rows_wider_than_the_stage_ring(T, H):
+    """bf16 rows of 600 KB and 1.2 MB: the scatter dispatch cuts them into
+    chunks of at most half its 64 KB ring of stages (the chunk rule alone
+    would give one or no stage)."""
+    rng = np.random.default_rng(T)
+    k, E = 3, 16
+    ids_np = _ids_random(rng, T, k, E, p_invalid=0.05)
+    x = torch.randn(T, H, device=DEV).to(torch.bfloat16)
+    meta = moe.moe_prepare(torch.from_numpy(ids_np).to(DEV), E)
+    out = torch.full((T * k, H), -3.0, device=DEV).to(torch.bfloat16)
+    moe.moe_dispatch_rows(x, k, None, meta.output_permutation, out=out)
+    err = moe.moe_dispatch_error()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    ref_meta = oracle.prepare(ids_np, E)
+    ref = bits(torch.full((T * k, H), -3.0).to(torch.bfloat16))
+    oracle.dispatch(bits(x), k, ref_meta["input_perm"], ref)
+    np.testing.assert_array_equal(bits(out), ref)
+
+
 @pytest.mark.parametrize("name", ["uniform_t4096_h7168_e256_k8", "khot_t9216_h7168_e256_k8",
                                   "zipf_fp16_t131072_h2048_e64_k6"])
 def test_dispatch_full_workloads_sampled(name):
