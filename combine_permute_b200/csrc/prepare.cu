@@ -373,37 +373,44 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
 
 size_t single_block_smem(int E) { return (size_t)(kSingleWarps * (E + 1) + 2 * E) * sizeof(int); }
 
+// A slot's expert e (-2..E-1) and its rank within its warp's run (-1..511)
+// in one int.
+__device__ __forceinline__ int pack_key_rank(int e, int rank) { return (rank + 1) << 12 | (e + 2); }
+__device__ __forceinline__ int packed_key(int v) { return (v & 4095) - 2; }
+__device__ __forceinline__ int packed_rank(int v) { return (v >> 12) - 1; }
+
 // ---------------------------------------------------------------------------
 // Tiled paths.  A tile is a run of consecutive slots ranked by one block of
 // NT threads: warp w takes nr rounds of 32 consecutive slots starting at
-// first + w * 32 * nr (nr <= NR, the register capacity).  rank_tile() ranks
-// the slots within each warp's run and folds the warps into the tile
-// histogram: hist[c] for c < E is the tile's count of expert c, hist[E] its
-// count of invalid ids; wcnt holds the per-warp exclusive prefixes and
-// key / rank each thread's slots.
+// first + w * 32 * nr.  Round r of a lane's slots keeps its expert, then its
+// expert and rank packed, at kr[r * 32] in shared memory (this lane's own
+// entries), so that the round loops stay rolled.  rank_tile() ranks the
+// slots within each warp's run and folds the warps into the tile histogram:
+// hist[c] for c < E is the tile's count of expert c, hist[E] its count of
+// invalid ids; wcnt holds the per-warp exclusive prefixes.
 // ---------------------------------------------------------------------------
-template <typename IdT, int NT, int NR>
+template <typename IdT, int NT>
 __device__ __forceinline__ void rank_tile(const IdT *__restrict__ ids, int64_t base, int64_t S,
                                           int E, int64_t first, int nr, int *wcnt, int *hist,
-                                          int *s_invalid, int (&key)[NR], int (&rank)[NR]) {
+                                          int *s_invalid, int *kr) {
     constexpr int NW = NT / 32;
     const int C = E + 1;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned lt = lanemask_lt();
     const int nbits = key_bits(E);
     const int64_t wbase = first + (int64_t)warp * 32 * nr;
-#pragma unroll
-    for (int r = 0; r < NR; ++r)
-        key[r] = r < nr ? load_key(ids, wbase + r * 32 + lane, S, base, E) : -2;
+#pragma unroll 4
+    for (int r = 0; r < nr; ++r) kr[r * 32] = load_key(ids, wbase + r * 32 + lane, S, base, E);
     for (int x = tid; x < NW * C; x += NT) wcnt[x] = 0;
     if (tid == 0) *s_invalid = 0;
     __syncthreads();
     int *row = wcnt + warp * C;
     int bad = 0;
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
-        if (r < nr) rank[r] = rank_round(key[r], E, nbits, row, lt);
-        bad += key[r] == -1;
+#pragma unroll 1
+    for (int r = 0; r < nr; ++r) {
+        const int e = kr[r * 32];
+        kr[r * 32] = pack_key_rank(e, rank_round(e, E, nbits, row, lt));
+        bad += e == -1;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, o);
@@ -417,20 +424,20 @@ __device__ __forceinline__ void rank_tile(const IdT *__restrict__ ids, int64_t b
 // Both permutations of a tile's slots: row = off[e] (expert offset, or 0) +
 // excl[e] (earlier tiles) + wcnt (earlier warps) + rank (earlier lanes and
 // rounds).  When `in_perm` is null only the rank part goes to out_perm.
-template <int NT, int NR>
 __device__ __forceinline__ void write_tile_rows(int64_t S, int E, int64_t first, int nr,
                                                 const int *off, const int *excl, const int *wcnt,
-                                                const int (&key)[NR], const int (&rank)[NR],
-                                                int32_t *in_perm, int32_t *out_perm) {
+                                                const int *kr, int32_t *in_perm,
+                                                int32_t *out_perm) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t wbase = first + (int64_t)warp * 32 * nr;
     const int *row = wcnt + warp * (E + 1);
-#pragma unroll
-    for (int r = 0; r < NR; ++r) {
+#pragma unroll 1
+    for (int r = 0; r < nr; ++r) {
         const int64_t i = wbase + r * 32 + lane;
-        if (r < nr && i < S) {
-            const int e = key[r];
-            const int p = e >= 0 ? (off ? off[e] : 0) + excl[e] + row[e] + rank[r] : -1;
+        if (i < S) {
+            const int v = kr[r * 32];
+            const int e = packed_key(v);
+            const int p = e >= 0 ? (off ? off[e] : 0) + excl[e] + row[e] + packed_rank(v) : -1;
             out_perm[i] = p;
             if (in_perm && p >= 0 && p < S) in_perm[p] = (int)i;
         }
@@ -509,14 +516,11 @@ constexpr int kSyncMinRounds = 4;
 static_assert(kSyncMaxRounds * kSyncThreads <= 65535, "a block's count of one expert fits 16 bits");
 
 // Shared memory of the two-kernel tiles: per-warp rows, then hist, excl,
-// off, pad (one column per expert plus one for invalid ids each).
-template <int NT> size_t tile_smem(int E) { return (size_t)(NT / 32 + 4) * (E + 1) * sizeof(int); }
-
-// A slot's expert e (-2..E-1) and its rank within its warp's run (-1..511)
-// in one int.
-__device__ __forceinline__ int pack_key_rank(int e, int rank) { return (rank + 1) << 12 | (e + 2); }
-__device__ __forceinline__ int packed_key(int v) { return (v & 4095) - 2; }
-__device__ __forceinline__ int packed_rank(int v) { return (v >> 12) - 1; }
+// off, pad (one column per expert plus one for invalid ids each), then the
+// tile's slots (expert and rank packed).
+template <int NT> size_t tile_smem(int E) {
+    return ((size_t)(NT / 32 + 4) * (E + 1) + (size_t)kTileSlots) * sizeof(int);
+}
 
 // One-launch prepare (a cooperative launch: every block resident, so blocks
 // may wait on one another; E + 1 <= kSyncThreads).  Block b ranks slots
@@ -785,6 +789,7 @@ __global__ void __launch_bounds__(kRankThreads, 2)
     int *excl = hist + C;
     int *off = excl + C;
     int *pad = off + C;
+    int *s_kr = pad + C;  // [NR][NT] each slot's expert and rank, warp by warp
     PrepWs ws = carve(workspace);
     pdl_wait();
     pdl_launch_dependents();
@@ -799,10 +804,10 @@ __global__ void __launch_bounds__(kRankThreads, 2)
     const int tile = (int)s_misc[0];
     const unsigned epoch = s_misc[1];
     const int64_t first = (int64_t)tile * kTileSlots;
-    int key[NR], rank[NR];
-    rank_tile<IdT, NT, NR>(ids, base, S, E, first, NR, wcnt, hist, &s_invalid, key, rank);
+    int *kr = s_kr + (threadIdx.x >> 5) * 32 * NR + (threadIdx.x & 31);
+    rank_tile<IdT, NT>(ids, base, S, E, first, NR, wcnt, hist, &s_invalid, kr);
     tile_lookback<NT>(ws, tile, epoch, E, hist, excl, wait_ns);
-    write_tile_rows<NT, NR>(S, E, first, NR, nullptr, excl, wcnt, key, rank, nullptr, out_perm);
+    write_tile_rows(S, E, first, NR, nullptr, excl, wcnt, kr, nullptr, out_perm);
     if (tile == G - 1) {
         for (int c = threadIdx.x; c < C; c += NT) off[c] = excl[c] + hist[c];
         __syncthreads();
