@@ -14,7 +14,7 @@
 //  * up to kSingleBlockSlots slots: one block does it all
 //    (prep_single_kernel);
 //  * above that, when every block fits on the GPU at once: one cooperative
-//    launch (prep_sync_kernel, 512-thread blocks of 1 to 16 rounds).  Each
+//    launch (prep_sync_kernel, 512-thread blocks of 1 to 32 rounds).  Each
 //    block ranks its slots, publishes its per-expert histogram row and meets
 //    the others at a grid barrier (bounded wait); every block then stages
 //    all rows, scans them into the expert offsets and its own prefix, and
@@ -174,7 +174,7 @@ struct PrepWs {
 
 // Most blocks of one one-launch prepare (one block per SM on B200, with room
 // for parts with more SMs) and the fixed size of its histogram rows.  A row
-// holds E+1 counts of at most kSyncMaxRounds * kSyncThreads = 8192 slots,
+// holds E+1 counts of at most kSyncMaxRounds * kSyncThreads = 16384 slots,
 // so 16 bits each, padded to a multiple of 8 (16 bytes) so that rows are
 // staged with 16-byte loads; at most kSyncThreads columns.  The region keeps
 // room for 32-bit counts (512 KB), so that the workspace layout and size do
@@ -511,7 +511,8 @@ constexpr int kRankThreads = 256;                  // two-kernel tiles: 8 warps
 constexpr int kRankRounds = kTileSlots / kRankThreads;  // of 8 rounds
 constexpr int kSyncThreads = 512;                  // one-launch tiles: 16 warps
 static_assert(kSyncThreads <= 512, "a histogram row of the one-launch path fits kSyncHistBytes");
-constexpr int kSyncMaxRounds = 16;                 // of up to 16 rounds (8192 slots)
+constexpr int kSyncStagedRounds = 16;              // staged input_permutation up to 16 rounds
+constexpr int kSyncMaxRounds = 32;                 // of up to 32 rounds (16384 slots)
 constexpr int kSyncMinRounds = 4;
 static_assert(kSyncMaxRounds * kSyncThreads <= 65535, "a block's count of one expert fits 16 bits");
 
@@ -532,18 +533,21 @@ template <int NT> size_t tile_smem(int E) {
 // block's prefix over earlier blocks (eight rows in flight), and three
 // exclusive scans over the experts run in registers: the expert offsets, the
 // block-scale offsets (block 0 writes both and the counts) and this block's
-// own offsets.  Every slot's row goes to output_permutation; the block's
-// slots are also staged in shared memory in dispatched order, so that
-// input_permutation is written in runs of consecutive rows rather than one
-// scattered word per slot.  Blocks count themselves out on a second word
+// own offsets.  Every slot's row goes to output_permutation.  With kStage
+// (up to kSyncStagedRounds rounds) the block's slots are also staged in
+// shared memory in dispatched order, so that input_permutation is written in
+// runs of consecutive rows rather than one scattered word per slot; above
+// that the staging would not fit beside the rows and input_permutation is
+// written slot by slot.  Blocks count themselves out on a second word
 // whose high half counts the waits that gave up; the last one clears both
 // counters and reports the waits in diag[1].
-template <int NT> size_t sync_smem(int E, int G, int nr) {
+template <int NT> size_t sync_smem(int E, int G, int nr, bool stage) {
     return (size_t)(NT / 32 + 4) * (E + 1) * sizeof(int) +
-           (size_t)G * sync_stride(E) * sizeof(unsigned short) + 3 * (size_t)nr * NT * sizeof(int);
+           (size_t)G * sync_stride(E) * sizeof(unsigned short) +
+           (stage ? 3 : 1) * (size_t)nr * NT * sizeof(int);
 }
 
-template <typename IdT>
+template <typename IdT, bool kStage>
 __global__ void __launch_bounds__(kSyncThreads, 1)
     prep_sync_kernel(const IdT *__restrict__ ids, int64_t base, int64_t S, int E, int A, int G,
                      int nr, void *workspace, unsigned long long wait_ns, int32_t *counts,
@@ -559,9 +563,10 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     int *lofs = base_row + C;       // [C] this block's offsets of its own slots
     // [G][Cp] every block's counts (16-byte aligned: (NW + 4) * 4 is a multiple of 16)
     unsigned short *rows = reinterpret_cast<unsigned short *>(wcnt + (NW + 4) * C);
-    int *s_slot = reinterpret_cast<int *>(rows + (size_t)G * Cp);  // [nr*NT] slots,
-    int *s_row = s_slot + nr * NT;  // [nr*NT] and their rows, in dispatched order
-    int *s_kr = s_row + nr * NT;  // [nr*NT] each slot's expert and rank, warp by warp
+    // kStage: [nr*NT] slots and [nr*NT] their rows, in dispatched order
+    int *s_slot = reinterpret_cast<int *>(rows + (size_t)G * Cp);
+    int *s_row = s_slot + (kStage ? nr * NT : 0);
+    int *s_kr = s_row + (kStage ? nr * NT : 0);  // [nr*NT] each slot's expert and rank
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tile = blockIdx.x;
     const int64_t first = (int64_t)tile * nr * NT;
@@ -588,12 +593,13 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
 #pragma unroll 4
         for (int r = 0; r < nr; ++r) kr[r * 32] = load_key(ids, wbase + r * 32 + lane, S, base, E);
     } else {
-        int key[kSyncMaxRounds];  // every round's id in flight at once
+        constexpr int NRMAX = kStage ? kSyncStagedRounds : kSyncMaxRounds;
+        int key[NRMAX];  // every round's id in flight at once
 #pragma unroll
-        for (int r = 0; r < kSyncMaxRounds; ++r)
+        for (int r = 0; r < NRMAX; ++r)
             key[r] = r < nr ? load_key(ids, wbase + r * 32 + lane, S, base, E) : -2;
 #pragma unroll
-        for (int r = 0; r < kSyncMaxRounds; ++r)
+        for (int r = 0; r < NRMAX; ++r)
             if (r < nr) kr[r * 32] = key[r];
     }
     __syncthreads();
@@ -611,7 +617,7 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     __syncthreads();
 
     // fold the warps: column c becomes exclusive over warps; publish the row
-    // (a block has at most nr * NT <= 8192 slots, so every count fits 16 bits)
+    // (a block has at most nr * NT <= 16384 slots, so every count fits 16 bits)
     if (tid < C) {
         int run = 0;
 #pragma unroll
@@ -741,20 +747,26 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
             if (e >= 0) {
                 const int lr = row[e] + packed_rank(v);
                 p = base_row[e] + lr;
-                const int lp = lofs[e] + lr;
-                if (lp >= 0 && lp < nr * NT) {
-                    s_slot[lp] = (int)i;
-                    s_row[lp] = p;
+                if constexpr (kStage) {
+                    const int lp = lofs[e] + lr;
+                    if (lp >= 0 && lp < nr * NT) {
+                        s_slot[lp] = (int)i;
+                        s_row[lp] = p;
+                    }
+                } else if (p < S) {
+                    in_perm[p] = (int)i;
                 }
             }
             out_perm[i] = p;
         }
     }
-    __syncthreads();
-    const int nown = own_total < nr * NT ? own_total : nr * NT;
-    for (int lp = tid; lp < nown; lp += NT) {
-        const int p = s_row[lp];
-        if (p >= 0 && p < S) in_perm[p] = s_slot[lp];
+    if constexpr (kStage) {
+        __syncthreads();
+        const int nown = own_total < nr * NT ? own_total : nr * NT;
+        for (int lp = tid; lp < nown; lp += NT) {
+            const int p = s_row[lp];
+            if (p >= 0 && p < S) in_perm[p] = s_slot[lp];
+        }
     }
     const int64_t lo = first > total ? first : (int64_t)total;
     const int64_t end = first + (int64_t)nr * NT;
@@ -924,10 +936,11 @@ template <typename IdT>
 cudaError_t launch_sync(const IdT *ids, int64_t base, int64_t S, int E, int A, void *workspace,
                         int32_t *counts, int32_t *offsets, int32_t *bso, int32_t *in_perm,
                         int32_t *out_perm, int32_t *diag, cudaStream_t stream) {
-    auto kern = prep_sync_kernel<IdT>;
     int nr = 0, G = 0;
     if (!sync_shape(S, E, (int64_t)sm_count(), &nr, &G)) return cudaErrorCooperativeLaunchTooLarge;
-    const size_t smem = sync_smem<kSyncThreads>(E, G, nr);
+    const bool stage = nr <= kSyncStagedRounds;
+    auto kern = stage ? prep_sync_kernel<IdT, true> : prep_sync_kernel<IdT, false>;
+    const size_t smem = sync_smem<kSyncThreads>(E, G, nr, stage);
     if (smem > 200 * 1024) return cudaErrorCooperativeLaunchTooLarge;
     const int64_t resident = (int64_t)sm_count() * blocks_per_sm(kern, kSyncThreads, smem);
     if (G > resident) return cudaErrorCooperativeLaunchTooLarge;
