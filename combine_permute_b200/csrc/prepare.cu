@@ -511,7 +511,7 @@ constexpr int kRankThreads = 256;                  // two-kernel tiles: 8 warps
 constexpr int kRankRounds = kTileSlots / kRankThreads;  // of 8 rounds
 constexpr int kSyncThreads = 512;                  // one-launch tiles: 16 warps
 static_assert(kSyncThreads <= 512, "a histogram row of the one-launch path fits kSyncHistBytes");
-constexpr int kSyncStagedRounds = 16;              // staged input_permutation up to 16 rounds
+constexpr int kSyncStagedRounds = 16;              // staged input_permutation: 5 to 16 rounds
 constexpr int kSyncMaxRounds = 32;                 // of up to 32 rounds (16384 slots)
 constexpr int kSyncMinRounds = 4;
 static_assert(kSyncMaxRounds * kSyncThreads <= 65535, "a block's count of one expert fits 16 bits");
@@ -534,11 +534,11 @@ template <int NT> size_t tile_smem(int E) {
 // exclusive scans over the experts run in registers: the expert offsets, the
 // block-scale offsets (block 0 writes both and the counts) and this block's
 // own offsets.  Every slot's row goes to output_permutation.  With kStage
-// (up to kSyncStagedRounds rounds) the block's slots are also staged in
+// (from 5 to kSyncStagedRounds rounds) the block's slots are also staged in
 // shared memory in dispatched order, so that input_permutation is written in
-// runs of consecutive rows rather than one scattered word per slot; above
-// that the staging would not fit beside the rows and input_permutation is
-// written slot by slot.  Blocks count themselves out on a second word
+// runs of consecutive rows rather than one scattered word per slot; with
+// fewer rounds that measured slower, with more it would not fit beside the
+// rows, and input_permutation is written slot by slot.  Blocks count themselves out on a second word
 // whose high half counts the waits that gave up; the last one clears both
 // counters and reports the waits in diag[1].
 template <int NT> size_t sync_smem(int E, int G, int nr, bool stage) {
@@ -938,7 +938,10 @@ cudaError_t launch_sync(const IdT *ids, int64_t base, int64_t S, int E, int A, v
                         int32_t *out_perm, int32_t *diag, cudaStream_t stream) {
     int nr = 0, G = 0;
     if (!sync_shape(S, E, (int64_t)sm_count(), &nr, &G)) return cudaErrorCooperativeLaunchTooLarge;
-    const bool stage = nr <= kSyncStagedRounds;
+    // staged from 5 to kSyncStagedRounds rounds: measured per call back to
+    // back, 13.7 against 16.0 us at 11 rounds, while at 1 to 4 rounds the
+    // slot-by-slot form was 0.1-0.2 us faster (7.25 against 7.33 us at 1)
+    const bool stage = nr > 4 && nr <= kSyncStagedRounds;
     auto kern = stage ? prep_sync_kernel<IdT, true> : prep_sync_kernel<IdT, false>;
     const size_t smem = sync_smem<kSyncThreads>(E, G, nr, stage);
     if (smem > 200 * 1024) return cudaErrorCooperativeLaunchTooLarge;

@@ -524,6 +524,8 @@ def test_chained_step_on_one_stream():
     (81920, 255),           # last size at 2 rounds
     (81921, 255),           # first at 3 rounds
     (1212416, 64),          # 148 blocks of 16 rounds: the last with input_permutation staged
+    (303104, 64),           # 148 blocks of 4 rounds: input_permutation slot by slot
+    (303105, 64),           # 5 rounds: input_permutation staged
     (1212417, 64),          # 17 rounds: input_permutation written slot by slot
     (2424832, 64),          # the largest one-launch problem on 148 SMs (32 rounds)
     (2424833, 64),          # one slot more: the two-kernel path
