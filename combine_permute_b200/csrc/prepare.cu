@@ -538,9 +538,9 @@ template <int NT> size_t tile_smem(int E) {
 // shared memory in dispatched order, so that input_permutation is written in
 // runs of consecutive rows rather than one scattered word per slot; with
 // fewer rounds that measured slower, with more it would not fit beside the
-// rows, and input_permutation is written slot by slot.  Blocks count themselves out on a second word
-// whose high half counts the waits that gave up; the last one clears both
-// counters and reports the waits in diag[1].
+// rows, and input_permutation is written slot by slot.  Blocks count
+// themselves out on a second word whose high half counts the waits that gave
+// up; the last one clears both counters and reports the waits in diag[1].
 template <int NT> size_t sync_smem(int E, int G, int nr, bool stage) {
     return (size_t)(NT / 32 + 4) * (E + 1) * sizeof(int) +
            (size_t)G * sync_stride(E) * sizeof(unsigned short) +
