@@ -305,6 +305,15 @@ def _config(w, n):
             "parallelism": "replicas" if n > 1 else "single GPU"}
 
 
+def net_of_events(call_us, step_us):
+    """What the timing events between the calls add to a step (the calls
+    timed with events, summed, against the event-free step), and each call's
+    share of the event-free step: its evented time less an equal share of
+    that overhead, so that the shares sum to the step's time."""
+    overhead = sum(call_us.values()) - step_us
+    return overhead, {c: t - overhead / len(call_us) for c, t in call_us.items()}
+
+
 def _step_bytes(w):
     return sum(algorithmic_bytes(w).values())
 
@@ -637,17 +646,12 @@ def bench_workload(args, w, dev, ranks, cpu_budget_s):
         "effective_gbs": step_alg / (elapsed_ms / K * 1e-3) / 1e9,
         "frac_of_measured_peak": step_alg / (elapsed_ms / K * 1e-3) / 1e9 / peak}
     if per_graph is not None and graph_ms is not None:
-        # what the timing events between the calls add to a step: the calls
-        # timed with events, summed, against the event-free graph's step
-        overhead = (sum(kern[c] for c in calls) - graph_ms / K) * 1e3
+        overhead, net = net_of_events({c: kern[c] * 1e3 for c in calls}, graph_ms / K * 1e3)
         breakdown["end_to_end"]["event_overhead_us_per_step"] = overhead
-        # each call's share of the event-free step, the overhead split
-        # equally between the calls (the shares sum to the step's time)
         for c in calls:
-            net = kern[c] * 1e3 - overhead / len(calls)
-            breakdown[c]["us_net_of_events"] = net
+            breakdown[c]["us_net_of_events"] = net[c]
             breakdown[c]["net_frac_of_8tbs_spec"] = (
-                alg[c] / (net * 1e-6) / 1e9 / SPEC_HBM_GBS if net > 0 else None)
+                alg[c] / (net[c] * 1e-6) / 1e9 / SPEC_HBM_GBS if net[c] > 0 else None)
     launch = (f"cuda_graph of {n_graph} steps, replayed {K // n_graph} times"
               if graph_ms is not None else "eager")
     l2_resident = None

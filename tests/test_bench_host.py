@@ -69,3 +69,12 @@ def test_next_row_bytes_of_the_fp8_workload():
     b = bench.next_row_bytes(CONFIGS["zipf_fp8_t16384_h4096_e288_k8"])
     assert b["dispatch_nvfp4"] == 134217728 + 131072 * 2304 + 524288 + 2312
     assert b["problem_sizes"] == 28 * 288
+
+
+def test_net_of_events_shares_sum_to_the_event_free_step():
+    # three calls timed with events (13.0 + 88.0 + 93.0 = 194 us) in a step
+    # that takes 179.6 us without them: 14.4 us of events, 4.8 a call
+    overhead, net = bench.net_of_events({"prepare": 13.0, "dispatch": 88.0, "combine": 93.0}, 179.6)
+    assert abs(overhead - 14.4) < 1e-9
+    assert abs(net["prepare"] - 8.2) < 1e-9 and abs(net["combine"] - 88.2) < 1e-9
+    assert abs(sum(net.values()) - 179.6) < 1e-9
