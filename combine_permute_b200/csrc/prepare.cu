@@ -853,7 +853,8 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 // Tiny batches: every block recomputes the metadata in shared memory (the
 // batch is at most kFusedMaxSlots slots), block 0 writes it out, and all
-// blocks copy their share of the x rows to their k dispatched rows.
+// blocks copy their share of the x rows to their k dispatched rows (each
+// thread's first x vector is loaded before the metadata is built).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kSingleThreads, 1)
     prep_dispatch_kernel(const int32_t *__restrict__ ids, int64_t T, int k, int E, int A,
@@ -865,6 +866,10 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
     int *pos;  // [S] dispatched row of every slot
     pdl_wait();
     pdl_launch_dependents();
+    // this thread's first x vector, in flight while the metadata is built
+    const int64_t total = T * nvec;
+    const int64_t v0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const uint4 x0 = v0 < total ? ld_stream_v4(x + v0) : make_uint4(0u, 0u, 0u, 0u);
     if (S <= kSmallSlots) {
         pos = smem + small_smem(E, S) / sizeof(int);
         small_prepare(ids, (int64_t)0, (int)S, E, A, smem, pos, blockIdx.x == 0, counts, offsets,
@@ -875,11 +880,9 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
                              offsets, bso, in_perm, out_perm, diag);
     }
     __syncthreads();
-    const int64_t total = T * nvec;
-    for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < total;
-         v += (int64_t)gridDim.x * blockDim.x) {
+    for (int64_t v = v0; v < total; v += (int64_t)gridDim.x * blockDim.x) {
         const int64_t t = v / nvec, c = v - t * nvec;
-        const uint4 val = ld_stream_v4(x + v);
+        const uint4 val = v == v0 ? x0 : ld_stream_v4(x + v);
         for (int j = 0; j < k; ++j) {
             const int p = pos[t * k + j];
             if (p >= 0) st_v4(out + (int64_t)p * nvec + c, val);
