@@ -14,7 +14,7 @@
 //  * up to kSingleBlockSlots slots: one block does it all
 //    (prep_single_kernel);
 //  * above that, when every block fits on the GPU at once: one cooperative
-//    launch (prep_sync_kernel, 512-thread blocks of 1 to 32 rounds).  Each
+//    launch (prep_sync_kernel, 512-thread blocks of 1 to 64 rounds).  Each
 //    block ranks its slots, publishes its per-expert histogram row and meets
 //    the others at a grid barrier (bounded wait); every block then stages
 //    all rows, scans them into the expert offsets and its own prefix, and
@@ -174,7 +174,7 @@ struct PrepWs {
 
 // Most blocks of one one-launch prepare (one block per SM on B200, with room
 // for parts with more SMs) and the fixed size of its histogram rows.  A row
-// holds E+1 counts of at most kSyncMaxRounds * kSyncThreads = 16384 slots,
+// holds E+1 counts of at most kSyncMaxRounds * kSyncThreads = 32768 slots,
 // so 16 bits each, padded to a multiple of 8 (16 bytes) so that rows are
 // staged with 16-byte loads; at most kSyncThreads columns.  The region keeps
 // room for 32-bit counts (512 KB), so that the workspace layout and size do
@@ -373,8 +373,8 @@ __global__ void __launch_bounds__(kSingleThreads, 1)
 
 size_t single_block_smem(int E) { return (size_t)(kSingleWarps * (E + 1) + 2 * E) * sizeof(int); }
 
-// A slot's expert e (-2..E-1) and its rank within its warp's run (-1..511)
-// in one int.
+// A slot's expert e (-2..E-1) and its rank within its warp's run
+// (-1..2047) in one int.
 __device__ __forceinline__ int pack_key_rank(int e, int rank) { return (rank + 1) << 12 | (e + 2); }
 __device__ __forceinline__ int packed_key(int v) { return (v & 4095) - 2; }
 __device__ __forceinline__ int packed_rank(int v) { return (v >> 12) - 1; }
@@ -512,7 +512,8 @@ constexpr int kRankRounds = kTileSlots / kRankThreads;  // of 8 rounds
 constexpr int kSyncThreads = 512;                  // one-launch tiles: 16 warps
 static_assert(kSyncThreads <= 512, "a histogram row of the one-launch path fits kSyncHistBytes");
 constexpr int kSyncStagedRounds = 16;              // staged input_permutation: 5 to 16 rounds
-constexpr int kSyncMaxRounds = 32;                 // of up to 32 rounds (16384 slots)
+constexpr int kSyncUnrolledRounds = 32;            // id loads unrolled: 5 to 32 rounds
+constexpr int kSyncMaxRounds = 64;                 // of up to 64 rounds (32768 slots)
 constexpr int kSyncMinRounds = 4;
 static_assert(kSyncMaxRounds * kSyncThreads <= 65535, "a block's count of one expert fits 16 bits");
 
@@ -584,16 +585,17 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     // rank, live in shared memory at kr[r*32] (read and written by this lane
     // only).  The ranking and row loops stay rolled: fully unrolled over the
     // largest round count, the kernel's code ran slower than its work (each
-    // launch fetches it anew).  Above 4 rounds the loads are unrolled, so
-    // that every round's id is in flight at once: measured at 11 rounds,
+    // launch fetches it anew).  From 5 to kSyncUnrolledRounds rounds the
+    // loads are unrolled, so that every round's id is in flight at once
+    // (above that, four at a time): measured at 11 rounds,
     // 13.6 us a call against 14.0 rolled (16.2 against 17.2 after an L2
     // flush); unrolled at 1 to 4 rounds they cost 0.4-0.6 us more.
     int *kr = s_kr + warp * 32 * nr + lane;
-    if (nr <= 4) {
+    if (nr <= 4 || nr > kSyncUnrolledRounds) {
 #pragma unroll 4
         for (int r = 0; r < nr; ++r) kr[r * 32] = load_key(ids, wbase + r * 32 + lane, S, base, E);
     } else {
-        constexpr int NRMAX = kStage ? kSyncStagedRounds : kSyncMaxRounds;
+        constexpr int NRMAX = kStage ? kSyncStagedRounds : kSyncUnrolledRounds;
         int key[NRMAX];  // every round's id in flight at once
 #pragma unroll
         for (int r = 0; r < NRMAX; ++r)
@@ -617,7 +619,7 @@ __global__ void __launch_bounds__(kSyncThreads, 1)
     __syncthreads();
 
     // fold the warps: column c becomes exclusive over warps; publish the row
-    // (a block has at most nr * NT <= 16384 slots, so every count fits 16 bits)
+    // (a block has at most nr * NT <= 32768 slots, so every count fits 16 bits)
     if (tid < C) {
         int run = 0;
 #pragma unroll

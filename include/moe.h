@@ -141,9 +141,9 @@ size_t moe_prepare_workspace_bytes(int64_t num_tokens, int32_t top_k, int32_t nu
  * Batches of up to 4096 slots run in one block; larger ones as tiles over
  * the whole GPU (the only case that touches the workspace): one cooperative
  * launch with one grid barrier when every tile fits on the GPU at once (up
- * to 32 rounds of 512 slots per SM: about 2.4 million slots on B200 with up
- * to about 300 experts), else two kernels with a decoupled look-back between
- * tiles.
+ * to 64 rounds of 512 slots per SM and the SM's shared memory: about 4.8
+ * million slots on B200 with 64 experts, 3.8 million with 256), else two
+ * kernels with a decoupled look-back between tiles.
  *
  * Dispatched order: by expert ascending, and within an expert by expanded
  * index ascending (token, then slot): a stable counting sort, so the result

@@ -96,12 +96,13 @@ def test_prepare_grid_barrier_that_never_fills_gives_up(wait_us):
 
 
 def test_prepare_lookback_on_an_unscheduled_tile_gives_up():
-    # above 2.4 M slots prepare runs as two kernels of 2048-slot tiles (more
-    # tiles than fit on the GPU at once) with a decoupled look-back.  A ticket
+    # above about 3.9 M slots of 256 experts prepare runs as two kernels of
+    # 2048-slot tiles (more tiles than fit on the GPU at once) with a
+    # decoupled look-back.  A ticket
     # word of 1 hands tile 0 to the block that takes the last ticket; the
     # first wave of resident tiles all wait on it and give up after the
     # default limit.
-    w = CONFIGS["uniform_t4096_h7168_e256_k8"].scaled(310000)  # 2.48 M slots
+    w = CONFIGS["uniform_t4096_h7168_e256_k8"].scaled(500000)  # 4 M slots
     ids_np, _, _, _ = make_workload(w, with_x=False, with_y=False)
     ids = torch.from_numpy(ids_np).to(DEV)
     ws = _ws(w)

@@ -36,10 +36,10 @@ def _check_local(ids_np, base, E, A=16):
 
 @pytest.mark.parametrize("id_dtype", [np.int32, np.int64])
 @pytest.mark.parametrize("T,base,E", [(40, 64, 32), (3000, 0, 256), (3000, 96, 64),
-                                      (40000, 128, 128), (262144, 16, 40), (330000, 16, 40)])
+                                      (40000, 128, 128), (262144, 16, 40), (660000, 16, 40)])
 def test_prepare_local_vs_oracle(id_dtype, T, base, E):
     # top-8 slots: one block, 1 round, 5 rounds (input_permutation staged),
-    # 28 rounds (one launch, slot by slot) and 2.64 M slots (two kernels)
+    # 28 rounds (one launch, slot by slot) and 5.28 M slots (two kernels)
     w = CONFIGS["uniform_t4096_h7168_e256_k8"].scaled(T)
     ids_np, _, _, _ = make_workload(w, with_x=False, with_y=False)
     ids_np = ids_np.astype(id_dtype)

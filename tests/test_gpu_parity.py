@@ -139,11 +139,11 @@ def test_one_workspace_shared_by_both_tiled_paths():
     different sizes and expert counts: neither path may read the other's
     data (or an earlier call's) as its own."""
     rng = np.random.default_rng(4242)
-    # one launch (input_permutation staged, or above 16 rounds not), then
-    # two kernels above 2.4 M slots, in turn
-    shapes = [(15000, 8, 5), (330000, 8, 256), (40000, 3, 64), (320000, 8, 288),
-              (60000, 8, 288), (170000, 8, 288), (300000, 6, 64), (330000, 8, 256),
-              (9000, 8, 256)]
+    # one launch (input_permutation staged or not) and two kernels (more
+    # than 511 experts), in turn
+    shapes = [(15000, 8, 5), (20000, 8, 600), (40000, 3, 64), (30000, 6, 700),
+              (60000, 8, 288), (20000, 8, 600), (320000, 8, 288), (30000, 6, 700),
+              (300000, 6, 64), (9000, 8, 256)]
     need = max(moe.moe_prepare_workspace_bytes(T, k, E) for T, k, E in shapes)
     ws = torch.zeros(need, dtype=torch.uint8, device=DEV)
     for T, k, E in shapes:
@@ -527,8 +527,10 @@ def test_chained_step_on_one_stream():
     (303104, 64),           # 148 blocks of 4 rounds: input_permutation slot by slot
     (303105, 64),           # 5 rounds: input_permutation staged
     (1212417, 64),          # 17 rounds: input_permutation written slot by slot
-    (2424832, 64),          # the largest one-launch problem on 148 SMs (32 rounds)
-    (2424833, 64),          # one slot more: the two-kernel path
+    (2424832, 64),          # 32 rounds: the last with every round's id load unrolled
+    (2424833, 64),          # 33 rounds: id loads four at a time
+    (4849664, 64),          # the largest one-launch problem on 148 SMs (64 rounds)
+    (4849665, 64),          # one slot more: the two-kernel path
 ])
 def test_prepare_path_boundaries(S, E):
     """Sizes on each side of the rules that pick the prepare path and the
